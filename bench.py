@@ -1,0 +1,451 @@
+"""Benchmark of the DV-SSQ layer on B200: one JSON line on rank 0.
+
+A step is one pass of the whole path on the Spark-shaped down_proj layer
+(W 2560 x 10240 BF16, H_256 blocks, 1280 salient columns, rank 16):
+    encode W  ->  forward of 1 token  ->  forward of 16 tokens.
+The metric's unit is GB/s of algorithmic bytes: the encoder reads W once and
+writes the packed form; each forward reads the packed layer once (x and y
+are not counted).  Eight independent copies of the layer (about 1.1 GB) are
+used in rotation so that no step finds its inputs in the 126 MB L2, and the
+forwards of a step read a copy that was encoded four steps earlier.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload spark_down|spark_up_prefill|bulk_encode]
+
+With --gpus N > 1 (under torchrun, one process per GPU) every rank runs the
+same step on its own layers: the path has no data-path exchange, so scaling
+is weak and the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DV-SSQ linear fwd: decode HBM GB/s vs peak; prefill TFLOP/s; encode GB/s"
+N_COPIES = 8
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------- helpers --
+
+def packed_bytes(M, K, rank, n_sal):
+    return M * K // 2 + M * (K // 64) * 2 + M * n_sal + M * 2 + n_sal * 4 + M * rank * 2 + rank * K * 2
+
+
+def encode_bytes(M, K, n_sal):
+    # read W once (BF16) + write q4, s4, q8, s8, sal_idx
+    return M * K * 2 + M * K // 2 + M * (K // 64) * 2 + M * n_sal + M * 2 + n_sal * 4
+
+
+def kernel_bytes(name, M, K, rank, n_sal, T):
+    """Algorithmic bytes of one launch of each kernel (see the design notes)."""
+    if name == "enc_pass1":
+        return M * K * 2
+    if name == "enc_pass2":
+        return encode_bytes(M, K, n_sal)
+    if name == "dec_main":
+        return M * K // 2 + M * (K // 64) * 2 + M * n_sal + M * 2 + M * rank * 2
+    if name == "dec_prologue":
+        return rank * K * 2 + n_sal * 4 + T * K * 2
+    return None
+
+
+def source_hash():
+    d = os.path.join(ROOT, "mixed_precision_weight_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kernel, workload):
+    """Per-launch DRAM bytes from the committed ncu summary, if still current."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    ent = rec.get(f"{kernel}@{workload}")
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc = index, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- workload --
+
+class SparkDownStep:
+    """encode + forward(T=1) + forward(T=16) on rotating copies of one layer."""
+
+    name = "spark_down_proj_2560x10240_r16_encode+fwd_T1+T16"
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv, self.torch = dv, torch
+        wl = synth.WORKLOADS["spark_down"]
+        self.wl = wl
+        M, K, B, r, n = wl.M, wl.K, wl.block, wl.rank, wl.n_sal
+        self.M, self.K, self.r, self.n = M, K, r, n
+        self.shape = dv.Shape.make(M, K, B, r, n)
+        self.copies = []
+        for c in range(N_COPIES):
+            off = 100 * rank_id + c
+            W = wl.weight(seed_offset=off).to(device)
+            act = wl.act_scale(seed_offset=off).to(device)
+            U, V = synth.lowrank_factors(M, K, r, seed=wl.seed + 7 + off)
+            packed = dv.PackedWeights.empty(self.shape, device, U=U.to(device), V=V.to(device))
+            self.copies.append((W, act, packed))
+        self.x1 = wl.activations(1, seed_offset=rank_id).to(device)
+        self.x16 = wl.activations(16, seed_offset=rank_id).to(device)
+        self.ws_enc = torch.empty(dv.dvssq_encode_workspace_size(self.shape), dtype=torch.uint8,
+                                  device=device)
+        self.ws1 = torch.empty(dv.dvssq_forward_workspace_size(self.shape, 1), dtype=torch.uint8,
+                               device=device)
+        self.ws16 = torch.empty(dv.dvssq_forward_workspace_size(self.shape, 16), dtype=torch.uint8,
+                                device=device)
+        self.y1 = torch.empty((1, M), dtype=torch.float32, device=device)
+        self.y16 = torch.empty((16, M), dtype=torch.float32, device=device)
+        for c in range(N_COPIES):   # every copy starts encoded
+            W, act, packed = self.copies[c]
+            dv.dvssq_encode(self.shape, W, act, packed, workspace=self.ws_enc)
+        self.i = 0
+
+    def step(self):
+        dv = self.dv
+        W, act, packed = self.copies[self.i % N_COPIES]
+        dv.dvssq_encode(self.shape, W, act, packed, workspace=self.ws_enc)
+        fwd = self.copies[(self.i + N_COPIES // 2) % N_COPIES][2]
+        dv.dvssq_linear_forward(self.shape, fwd, self.x1, y=self.y1, workspace=self.ws1)
+        dv.dvssq_linear_forward(self.shape, fwd, self.x16, y=self.y16, workspace=self.ws16)
+        self.i += 1
+
+    def bytes_per_step(self):
+        return encode_bytes(self.M, self.K, self.n) + 2 * packed_bytes(self.M, self.K, self.r, self.n)
+
+    def launches_per_step(self):
+        return 4 + 2 + 2
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "K": self.K, "block": 256, "rank": self.r,
+                "n_sal": self.n, "tokens": [1, 16],
+                "step": "dvssq_encode + dvssq_linear_forward(T=1) + dvssq_linear_forward(T=16)",
+                "l2": f"{N_COPIES} rotating layer copies (~{N_COPIES * 70} MB) > 126 MB L2; "
+                      "forwards read a copy encoded 4 steps earlier",
+                "lowrank_factors": "seeded synthetic U, V (values do not change the work)",
+                "parallelism": "replica per GPU (weak scaling, no data-path collective)"}
+
+    # ---- end-to-end through the public API with host buffers ----
+    def e2e_setup(self, synth):
+        torch = self.torch
+        wl = self.wl
+        self.hW = wl.weight(seed_offset=999).pin_memory()
+        self.hact = wl.act_scale(seed_offset=999).pin_memory()
+        U, V = synth.lowrank_factors(self.M, self.K, self.r, seed=1234)
+        self.hU, self.hV = U.pin_memory(), V.pin_memory()
+        self.hx1 = wl.activations(1, seed_offset=77).pin_memory()
+        self.hx16 = wl.activations(16, seed_offset=78).pin_memory()
+        self.hy1 = torch.empty((1, self.M), dtype=torch.float32).pin_memory()
+        self.hy16 = torch.empty((16, self.M), dtype=torch.float32).pin_memory()
+
+    def e2e_step(self):
+        dv = self.dv
+        layer = dv.DvssqLinear.from_weight(self.hW, self.hact, self.hU, self.hV, block=256)
+        self.hy1.copy_(layer(self.hx1), non_blocking=True)
+        self.hy16.copy_(layer(self.hx16), non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in
+                  (self.hW, self.hact, self.hU, self.hV, self.hx1, self.hx16))
+        d2h = (self.hy1.numel() + self.hy16.numel()) * 4
+        return h2d, d2h
+
+    # ---- the oracle on the host cores ----
+    def oracle_sample(self, O, synth):
+        wl = self.wl
+        W = O.torch_bf16_to_f64(wl.weight(seed_offset=555))
+        act = wl.act_scale(seed_offset=555).numpy()
+        U, V = synth.lowrank_factors(self.M, self.K, self.r, seed=55)
+        Uf, Vf = O.torch_bf16_to_f64(U), O.torch_bf16_to_f64(V)
+        x1 = O.torch_bf16_to_f64(wl.activations(1))
+        x16 = O.torch_bf16_to_f64(wl.activations(16))
+
+        def step():
+            enc = O.encode(W, act, wl.block, self.r, with_svd=False)
+            O.forward(enc, x1, U=Uf, V=Vf)
+            O.forward(enc, x16, U=Uf, V=Vf)
+        return step
+
+
+# -------------------------------------------------------------------- main --
+
+def threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_oracle(work, O, synth, budget_s=20.0, min_steps=1, max_steps=10):
+    step = work.oracle_sample(O, synth)
+    t0 = time.perf_counter()
+    n = 0
+    while n < min_steps or (time.perf_counter() - t0 < budget_s and n < max_steps):
+        step()
+        n += 1
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="spark_down")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    import mixed_precision_weight_b200 as pkg
+    from mixed_precision_weight_b200 import synth
+    dv = pkg.binding
+
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(device))
+    work = SparkDownStep(dv, synth, torch, rank, device)
+    W = max(3, args.warmup)
+    for _ in range(W):
+        work.step()
+    torch.cuda.synchronize()
+    dv.dvssq_device_error(clear=True)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            work.step()
+        stop.record(stream)
+        barrier()
+    ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    err = dv.dvssq_device_error(clear=True)
+    ms_step = ms / args.steps
+    bytes_step = work.bytes_per_step()
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+
+    # per-kernel device times: the same K steps again with events around each launch
+    dv.dvssq_profile_reset()
+    dv.dvssq_profile_enable(True)
+    for _ in range(args.steps):
+        work.step()
+    torch.cuda.synchronize()
+    dv.dvssq_profile_collect()
+    dv.dvssq_profile_enable(False)
+    prof = dv.dvssq_profile_read()
+    pk, pk_kind = peaks()
+    kernels = {}
+    M, K, r, n = work.M, work.K, work.r, work.n
+    tot_ms = sum(v[1] for v in prof.values())
+    for name, (cnt, kms) in prof.items():
+        avg = kms / cnt
+        ent = {"launches": cnt, "avg_us": round(avg * 1e3, 3), "share": round(kms / tot_ms, 4)}
+        calls_T = 16 if name == "dec_prologue" else 1
+        b = kernel_bytes(name, M, K, r, n, calls_T)
+        if b is not None:
+            gbs = b / (avg * 1e-3) / 1e9
+            ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
+        kernels[name] = ent
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
+    db = kernel_bytes(dom, M, K, r, n, 16)
+    dom_avg_ms = prof[dom][1] / prof[dom][0]
+    achieved = db / (dom_avg_ms * 1e-3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": pk["hbm_gbs"], "peak_source": pk_kind, "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4),
+                "traffic": dram_traffic(dom, args.workload),
+                "algorithmic_bytes_per_launch": db}
+    # the decode GEMV's own roofline (the headline HBM-bound kernel)
+    dm = kernels.get("dec_main")
+
+    # end-to-end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        work.e2e_setup(synth)
+        for _ in range(2):
+            work.e2e_step()
+        torch.cuda.synchronize()
+        e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        barrier()
+        e_start.record(stream)
+        for _ in range(n_e2e):
+            work.e2e_step()
+        e_stop.record(stream)
+        barrier()
+        ems = e_start.elapsed_time(e_stop) / n_e2e
+        if world > 1:
+            t = torch.tensor([ems], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d, d2h = work.e2e_bytes()
+        e2e = {"value": round(world * bytes_step / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "ms_per_step": round(ems, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import dvssq_oracle as O
+        nst, dt = run_oracle(work, O, synth)
+        cpu = {"value": round(bytes_step * nst / dt / 1e9, 4), "unit": "GB/s",
+               "cores": threads_used(), "kind": "oracle",
+               "sample": f"{nst} full step(s) of the same workload (encode without SVD + "
+                         f"2 forwards) on the host, {dt:.1f} s"}
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": W, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp16",
+            "data": "synthetic (seeded N(0,0.02) weights with outlier columns, N(0,1) tokens)",
+            "config": work.config(), "roofline": roofline, "kernels": kernels,
+            "decode_gemv": dm, "gpu_launches": work.launches_per_step() * args.steps,
+            "e2e": e2e, "cpu_baseline": cpu, "device_error_word": err,
+            "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args, world, rank):
+    """The oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import torch  # noqa: F401  (synth uses torch for BF16 rounding)
+    from mixed_precision_weight_b200 import synth
+    from oracle import dvssq_oracle as O
+
+    class _W(SparkDownStep):
+        def __init__(self):
+            wl = synth.WORKLOADS["spark_down"]
+            self.wl = wl
+            self.M, self.K, self.r, self.n = wl.M, wl.K, wl.rank, wl.n_sal
+    work = _W()
+    step = work.oracle_sample(O, synth)
+    for _ in range(max(0, min(args.warmup, 1))):
+        step()
+    t0 = time.perf_counter()
+    nst = max(1, min(args.steps, 3))
+    for _ in range(nst):
+        step()
+    dt = time.perf_counter() - t0
+    v = work.bytes_per_step() * nst / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": nst, "warmup": min(args.warmup, 1),
+            "ms_per_step": round(dt / nst * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": SparkDownStep.config(work),
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "kind": "oracle",
+                             "cores": threads_used(),
+                             "sample": f"{nst} full steps of the workload on the host"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,227 @@
+/*
+ * dvssq.h -- C ABI of libdvssq.so, a B200 (sm_100a) implementation of the
+ * DV-SSQ compressed linear layer.
+ *
+ * The method (F-Labs model cards "Spark-X2.5-4B-Hadamard-GSQ", section
+ * "Architectural Pillars / 1. DV-SSQ", Tiers A-C, and
+ * "MiniCPM5-2B-Hadamard-GSQ", section "Mathematical Foundations" §1-§2):
+ *
+ *   offline (dvssq_encode):  W_rot = W . H_K, H_K = diag(H_b, ..., H_b), b in
+ *     {128, 256}; the top n_sal rotated columns by salience are kept as INT8
+ *     with one BF16 scale per row; every other rotated weight is quantised
+ *     to symmetric INT4 in groups of 64 contiguous rotated columns with one
+ *     BF16 scale per group.
+ *   online (dvssq_linear_forward):
+ *     y = What4 . (H x) + diag(s8) . Q8 . (H x)_sal + U . (V . (H x)) [+ bias]
+ *     with U, V the BF16 truncated-SVD factors of the INT4 residual (A and B
+ *     of the MiniCPM card's §2), supplied by the caller.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument named as a buffer is a DEVICE pointer on the
+ *   current CUDA device unless documented as host.  Every buffer is owned by
+ *   the caller; the library never allocates or frees device memory.  Scratch
+ *   memory is the caller's "workspace" (size from the *_workspace_size query).
+ * - Matrices are dense and row-major.  BF16 values travel as uint16_t bit
+ *   patterns.
+ * - Every device buffer must be 16-byte aligned (cudaMalloc gives 256 B);
+ *   the workspace must be 256-byte aligned.  Violations return
+ *   DVSSQ_ERR_MISALIGNED before any launch.
+ * - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *   NULL is the legacy default stream).  Argument validation happens on the
+ *   host before any launch and returns an error status with nothing
+ *   launched.  A launch failure returns DVSSQ_ERR_CUDA; dvssq_last_error()
+ *   gives the CUDA message.
+ * - A workspace must not be shared by calls that may run concurrently.
+ * - Kernels never wait without a bound: a wait that runs out sets a device
+ *   error word that dvssq_device_error() reads and clears.
+ */
+#ifndef DVSSQ_H
+#define DVSSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DVSSQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DVSSQ_API __attribute__((visibility("default")))
+#else
+#define DVSSQ_API
+#endif
+
+typedef enum {
+  DVSSQ_OK = 0,
+  DVSSQ_ERR_INVALID_ARG = 1,      /* NULL pointer, negative size, bad enum      */
+  DVSSQ_ERR_UNSUPPORTED_SHAPE = 2,/* shape outside the documented limits        */
+  DVSSQ_ERR_MISALIGNED = 3,       /* a buffer is not 16-byte aligned            */
+  DVSSQ_ERR_WORKSPACE = 4,        /* workspace smaller than the query's answer  */
+  DVSSQ_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed       */
+  DVSSQ_ERR_DEVICE = 6            /* current device is not compute capability 10.0 */
+} dvssq_status;
+
+/* Shape of one compressed linear layer.
+ *   M      out_features (rows of W), 1 <= M <= 2^24
+ *   K      in_features, a multiple of `block`, of 64 and of 128, K <= 65536
+ *   block  Hadamard block size b: 128 or 256
+ *   group  INT4 group size: must be 64
+ *   n_sal  number of salient (INT8) columns: 0 <= n_sal <= K, n_sal % 16 == 0;
+ *          the method uses n_sal = K / 8 (top 12.5 %)
+ *   rank   rank r of the residual factors: 0 <= r <= 64                    */
+typedef struct {
+  int32_t M;
+  int32_t K;
+  int32_t block;
+  int32_t group;
+  int32_t n_sal;
+  int32_t rank;
+} dvssq_shape;
+
+/* The packed layer (all device pointers).  dvssq_encode writes q4, s4,
+ * sal_idx, q8 and s8; U and V are inputs supplied by the caller.
+ *   q4       uint8 [M][K/2]: INT4 codes of the rotated weights, two's
+ *            complement, the even rotated column in the low nibble; codes at
+ *            salient columns are 0 (dense layout over all K)
+ *   s4       bf16 [M][K/64]: one scale per 64 contiguous rotated columns
+ *   sal_idx  int32 [n_sal]: salient rotated-column indices, ascending
+ *   q8       int8 [M][n_sal]: INT8 codes; column k belongs to sal_idx[k]
+ *   s8       bf16 [M]: one INT8 scale per row
+ *   U        bf16 [M][r]: A = U_r sqrt(S_r) of the rotated-domain residual
+ *   V        bf16 [r][K]: B = sqrt(S_r) V_r^T, rotated-domain columns        */
+typedef struct {
+  uint8_t *q4;
+  uint16_t *s4;
+  int32_t *sal_idx;
+  int8_t *q8;
+  uint16_t *s8;
+  const uint16_t *U;
+  const uint16_t *V;
+} dvssq_weights;
+
+/* Diagnostics of one encode (host struct, filled when non-NULL). */
+typedef struct {
+  /* row-blocks whose +-1 Hadamard sums are not provably exact in fp64
+     (BF16 exponent spread above 45 - log2(b) bits); codes of such blocks
+     may differ from an exact-arithmetic encoder in the last rounding     */
+  int64_t inexact_rotation_blocks;
+  /* INT4 groups with a nonzero scale outside [2^-17, 8188] and rows with a
+     nonzero INT8 scale outside [2^-17, 511]: the prefill path stages q*s
+     in FP16, which is exact (INT4) or correctly rounded (INT8) only
+     inside those ranges                                                   */
+  int64_t fp16_unsafe_scales;
+  /* NaN or infinite salience scores (from non-finite W or act_scale)      */
+  int64_t nonfinite_scores;
+} dvssq_encode_info;
+
+/* Output element type of the forward. */
+enum { DVSSQ_Y_F32 = 0, DVSSQ_Y_BF16 = 1 };
+
+/* Kernel choice of the forward: AUTO picks the decode GEMV for T <= 16 and
+ * the tensor-core GEMM above; the others force one (the GEMV accepts
+ * T <= 16, the GEMM any T >= 1).                                          */
+enum { DVSSQ_PATH_AUTO = 0, DVSSQ_PATH_DECODE = 1, DVSSQ_PATH_PREFILL = 2 };
+
+/* ABI version of the loaded library (DVSSQ_ABI_VERSION). */
+DVSSQ_API int32_t dvssq_abi_version(void);
+
+/* Static description of a status code. */
+DVSSQ_API const char *dvssq_status_string(dvssq_status status);
+
+/* Text of the last CUDA error seen by this host thread ("" if none). */
+DVSSQ_API const char *dvssq_last_error(void);
+
+/* Blockwise Walsh-Hadamard rotation of activations, x_rot = H_K x
+ * (MiniCPM card, Mathematical Foundations §1: X' = X H; Spark card, Tier B:
+ * H_K = diag(H_b, ..., H_b)), H_b = S_b / sqrt(b) with S_b Sylvester's
+ * +-1 matrix.
+ *   x      bf16 [rows][cols]  (device)
+ *   y      fp32 [rows][cols]  (device), y[i] = H_K x[i], computed in fp32
+ *   rows   >= 0 (0 is a no-op); cols a multiple of block; block 128 or 256
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, DEVICE, CUDA.        */
+DVSSQ_API dvssq_status dvssq_fwht(const void *x, float *y, int64_t rows, int32_t cols,
+                        int32_t block, void *stream);
+
+/* Bytes of workspace dvssq_encode needs for `shape` (host only; no CUDA). */
+DVSSQ_API dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes);
+
+/* Encoder (Spark card, Tiers A and B; MiniCPM card §1-§2):
+ *   1. W_rot = W . H_K in fp64; each +-1 sum is exact whenever
+ *      inexact_rotation_blocks is 0, the scale 1/sqrt(b) is applied once.
+ *   2. score_j = act_scale_j * sqrt(sum_i W_rot[i,j]^2); the sum runs over
+ *      rows in chunks of 64 (within a chunk acc = acc + w*w, each operation
+ *      rounded), chunk partials added in ascending order.
+ *   3. sal_idx = the n_sal largest scores, ties to the lower index, sorted.
+ *   4. INT8 tier per row: s8 = bf16_rn(max_{j in sal} |W_rot| / 127),
+ *      q8 = clip(rint(w / s8), -128, 127)  (division as w * (1/s8)).
+ *   5. INT4 tier per 64-column group with the salient columns zeroed:
+ *      s4 = bf16_rn(absmax / 7), q = clip(rint(w * (1/s4)), -8, 7).
+ *   Arguments:
+ *   shape      host pointer
+ *   W          bf16 [M][K] (device), original (unrotated) weights
+ *   act_scale  fp32 [K] (device), activation scale per rotated column
+ *   out        host struct of device pointers; q4, s4, sal_idx, q8, s8 are
+ *              written (sal_idx/q8 may be NULL when n_sal == 0)
+ *   resid      fp32 [M][K] (device) or NULL: R = W_bg - What4 in the
+ *              rotated domain, the input of the truncated SVD (Tier C)
+ *   info       host struct or NULL; when given the call synchronises
+ *              `stream` to fill it
+ *   workspace  device scratch of at least dvssq_encode_workspace_size bytes
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_encode(const dvssq_shape *shape, const void *W,
+                          const float *act_scale, const dvssq_weights *out,
+                          float *resid, dvssq_encode_info *info,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace dvssq_linear_forward needs for `shape`, T tokens and
+ * `path` (host only). */
+DVSSQ_API dvssq_status dvssq_forward_workspace_size(const dvssq_shape *shape, int64_t T,
+                                          int32_t path, size_t *bytes);
+
+/* Forward on the packed form (MiniCPM card §2 runtime equation
+ * Y = X What^T + (X B^T) A^T, with the Spark card's INT8 salient tier):
+ *   y[t][i] = sum_j q4_ij s4_i,j/64 xr[t][j] + s8_i sum_k q8_ik xr[t][sal_k]
+ *             + sum_p U_ip (sum_j V_pj xr[t][j]) + bias_i,   xr = H_K x.
+ *   shape    host pointer; w: host struct of device pointers (read only)
+ *   x        bf16 [T][K] (device); T >= 0 (0 is a no-op)
+ *   bias     bf16 [M] (device) or NULL
+ *   y        [T][M] (device), fp32 or bf16 by y_dtype (bf16 = round to
+ *            nearest even of the fp32 result)
+ *   path     DVSSQ_PATH_*
+ *   workspace device scratch of at least dvssq_forward_workspace_size bytes
+ * Arithmetic: the GEMV path multiplies exact FP16 codes by the FP16-rounded
+ * xr on tensor cores with FP32 accumulation and applies s4/s8 in FP32; the
+ * GEMM path stages q*s in FP16 (exact for INT4 inside the ranges of
+ * fp16_unsafe_scales) and xr in FP16, accumulating in FP32.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvssq_weights *w,
+                                  const void *x, int64_t T, const void *bias,
+                                  void *y, int32_t y_dtype, int32_t path,
+                                  void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/* Reads (and clears when `clear` != 0) the device error word of the current
+ * device; synchronises the device.  0 means no kernel gave up a wait.     */
+DVSSQ_API dvssq_status dvssq_device_error(uint32_t *word, int32_t clear);
+
+/* Per-kernel device timing.  While enabled, every launch is bracketed by
+ * CUDA events on its own stream (and launched without programmatic
+ * dependent launch).  dvssq_profile_collect synchronises those events and
+ * adds their elapsed times to per-kernel totals; dvssq_profile_get reads
+ * entry i (i < dvssq_profile_count()): its kernel name (static string),
+ * launch count and total milliseconds.  dvssq_profile_reset clears them. */
+DVSSQ_API dvssq_status dvssq_profile_enable(int32_t on);
+DVSSQ_API dvssq_status dvssq_profile_collect(void);
+DVSSQ_API int32_t dvssq_profile_count(void);
+DVSSQ_API dvssq_status dvssq_profile_get(int32_t i, const char **name, int64_t *launches,
+                               double *total_ms);
+DVSSQ_API dvssq_status dvssq_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DVSSQ_H */

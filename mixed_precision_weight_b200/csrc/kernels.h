@@ -1,0 +1,113 @@
+// Internal interface between the C ABI (dvssq_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+namespace dvssq {
+
+// Largest supported salient set (bounded by the encoder's shared-memory stash).
+constexpr int kMaxSalient = 16384;
+
+// ------------------------------------------------------------ launching ---
+// Launches kernels with optional programmatic dependent launch and, while
+// profiling is enabled, brackets each launch with CUDA events on its stream.
+struct ProfileRecord {
+  const char *name;
+  cudaEvent_t start, stop;
+};
+
+class Launcher {
+ public:
+  bool profiling = false;
+  std::vector<ProfileRecord> pending;
+
+  template <typename... KArgs, typename... Args>
+  cudaError_t launch(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                     size_t smem, cudaStream_t st, bool pdl, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (pdl && !profiling) {
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+    }
+    ProfileRecord rec{name, nullptr, nullptr};
+    if (profiling) {
+      cudaEventCreate(&rec.start);
+      cudaEventCreate(&rec.stop);
+      cudaEventRecord(rec.start, st);
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (profiling) {
+      cudaEventRecord(rec.stop, st);
+      pending.push_back(rec);
+    }
+    return e;
+  }
+};
+
+Launcher &launcher();
+
+// --------------------------------------------------------------- encoder ---
+struct EncodeArgs {
+  int M, K, block, n_sal;
+  const void *W;
+  const float *act_scale;
+  uint8_t *q4;
+  uint16_t *s4;
+  int32_t *sal_idx;
+  int8_t *q8;
+  uint16_t *s8;
+  float *resid;
+  int64_t *info_host;  // 3 counters or nullptr
+  void *workspace;
+};
+size_t encode_workspace_bytes(int M, int K);
+int pass2_rows_per_cta(int block, int n_sal);
+cudaError_t prepare_encode_kernels();
+cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L);
+
+// ------------------------------------------------------------ activations -
+cudaError_t launch_fwht(const uint16_t *x, float *y, int64_t rows, int cols, int block,
+                        cudaStream_t st, Launcher &L);
+
+// ---------------------------------------------------------------- forward -
+struct ForwardArgs {
+  int M, K, block, n_sal, rank;
+  int T;
+  const uint8_t *q4;
+  const uint16_t *s4;
+  const int32_t *sal_idx;
+  const int8_t *q8;
+  const uint16_t *s8;
+  const uint16_t *U;
+  const uint16_t *V;
+  const uint16_t *x;
+  const uint16_t *bias;
+  void *y;
+  int y_bf16;
+  void *workspace;
+};
+
+size_t decode_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T);
+size_t prefill_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T);
+cudaError_t prepare_forward_kernels();
+cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L);
+cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L);
+
+// Tensor-map encoder from the driver (resolved once through the runtime).
+CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                        uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+}  // namespace dvssq

@@ -1,0 +1,7 @@
+// Single translation unit of libdvssq.so: the kernels share device state (the
+// error word) and helpers without relocatable device code.
+#include "dvssq_api.cu"
+#include "fwht.cu"
+#include "encode.cu"
+#include "decode.cu"
+#include "prefill.cu"

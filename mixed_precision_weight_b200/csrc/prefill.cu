@@ -1,0 +1,447 @@
+// Prefill-shaped forward (many tokens) of the DV-SSQ layer on the 5th-
+// generation tensor cores: the MiniCPM5-2B-Hadamard-GSQ card's runtime
+// equation (§2) with the Spark card's INT8 salient tier, as ONE dense
+// contraction over a concatenated reduction axis:
+//
+//   y[t][m] = sum_k A[m][k] * Xc[t][k] + bias[m]
+//   A  = [ q4 . s4 (K cols) | q8 . s8 (n_sal, padded to 64) | U (r, padded to 64) ]
+//   Xc = [ H x             | (H x)[sal_idx]                | V H x                ]
+//
+// pre_act   one CTA per 16 tokens builds Xc in FP16: fp32 Kronecker FWHT of
+//           each Hadamard block, the salient gather, and t = V xr with
+//           mma.sync (fp32 accumulation over all blocks).
+// pre_gemm  CTA tile 128 rows x BN tokens.  Warp 0 streams Xc tiles by TMA
+//           (128B swizzle); warps 2-5 dequantise the packed weights of the
+//           stage straight into the UMMA K-major 128B-swizzled layout (q4 . s4
+//           is exact in FP16 for scales in [2^-17, 8188]; q8 . s8 and U are
+//           rounded once); warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into
+//           a TMEM accumulator and commits each stage back to its producers;
+//           warps 2-5 then read TMEM (tcgen05.ld) and write y.  No TMA
+//           multicast is used anywhere.
+#include "common.cuh"
+#include "fwht_group.cuh"
+#include "kernels.h"
+
+namespace dvssq {
+
+constexpr int kPreBM = 128;
+constexpr int kPreStages = 4;
+constexpr int kPreThreads = 192;
+
+struct PrefillParams {
+  int M, K, T, n_sal, salp, rank, Kc, nstages, nq4, nsal;
+  float c;
+  const uint8_t *q4;
+  const uint16_t *s4;
+  const int32_t *sal_idx;
+  const int8_t *q8;
+  const uint16_t *s8;
+  const uint16_t *U;
+  const uint16_t *V;
+  const uint16_t *x;
+  const uint16_t *bias;
+  void *y;
+  int y_bf16;
+  __half *xc;      // [T][Kc]
+};
+
+// ------------------------------------------------------------------ pre_act
+// Dynamic shared memory of pre_act: fp32 block [16][B+1], FP16 block
+// [16][B+8], FP16 V block [rank][B+8], sal_idx copy [n_sal].
+static size_t pre_act_smem_bytes(int B, int rank, int n_sal) {
+  return (size_t)16 * (B + 1) * 4 + (size_t)16 * (B + 8) * 2 + (size_t)rank * (B + 8) * 2 +
+         (size_t)n_sal * 4;
+}
+
+template <int B>
+__global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
+  constexpr int P = B / 16;
+  constexpr int NW = B / 32;
+  __shared__ float scratch[16][GroupScratch<B>::kElems];
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float (*xr)[B + 1] = reinterpret_cast<float (*)[B + 1]>(dsm);
+  __half (*xh)[B + 8] = reinterpret_cast<__half (*)[B + 8]>(dsm + 16 * (B + 1) * 4);
+  __half (*vh)[B + 8] =
+      reinterpret_cast<__half (*)[B + 8]>(dsm + 16 * (B + 1) * 4 + 16 * (B + 8) * 2);
+  int *sidx = reinterpret_cast<int *>(dsm + 16 * (B + 1) * 4 + 16 * (B + 8) * 2 +
+                                      (size_t)p.rank * (B + 8) * 2);
+
+  const int tid = threadIdx.x, tok = tid / P, t = tid % P;
+  const int t0 = blockIdx.x * 16, gt = t0 + tok;
+  const bool live = gt < p.T;
+  const int nkb = p.K / B;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
+  for (int e = tid; e < p.n_sal; e += B) sidx[e] = p.sal_idx[e];
+
+  // t accumulators: n-tile (8 ranks) nt = warp + NW * j, j = 0, 1
+  float tacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  const int ntiles = (p.rank + 7) / 8;
+
+  for (int kb = 0; kb < nkb; ++kb) {
+    float v[16];
+#pragma unroll
+    for (int a = 0; a < 16; ++a)
+      v[a] = live ? bf16_bits_to_f32(p.x[(size_t)gt * p.K + (size_t)kb * B + P * a + t]) : 0.0f;
+    fwht_group<B>(v, scratch[tok], t);
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      const float a0 = v[j] * p.c, a1 = v[j + 1] * p.c;
+      xr[tok][16 * t + j] = a0;
+      xr[tok][16 * t + j + 1] = a1;
+      h[j / 2] = pack_half2(__float2half_rn(a0), __float2half_rn(a1));
+    }
+    *reinterpret_cast<uint4 *>(&xh[tok][16 * t]) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4 *>(&xh[tok][16 * t + 8]) = make_uint4(h[4], h[5], h[6], h[7]);
+    if (live) {
+      uint4 *dst = reinterpret_cast<uint4 *>(p.xc + (size_t)gt * p.Kc + (size_t)kb * B + 16 * t);
+      dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+    // V block as FP16
+    for (int i = tid; i < p.rank * (B / 8); i += B) {
+      const int rr = i / (B / 8), cc = i % (B / 8);
+      const uint4 raw =
+          *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + (size_t)kb * B + cc * 8);
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        o[u] = pack_half2(__float2half_rn(bf16_bits_to_f32(wv[u] & 0xFFFFu)),
+                          __float2half_rn(bf16_bits_to_f32(wv[u] >> 16)));
+      *reinterpret_cast<uint4 *>(&vh[rr][cc * 8]) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __syncthreads();
+    // salient gather: entries whose column lies in this block (sal_idx sorted)
+    {
+      int lo = 0, hi = p.n_sal;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (sidx[mid] < kb * B) lo = mid + 1; else hi = mid;
+      }
+      const int e_lo = lo;
+      hi = p.n_sal;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (sidx[mid] < (kb + 1) * B) lo = mid + 1; else hi = mid;
+      }
+      const int e_hi = lo;
+      for (int i = tid; i < (e_hi - e_lo) * 16; i += B) {
+        const int e = e_lo + i / 16, q = i % 16;
+        const int col = sidx[e] - kb * B;
+        if (t0 + q < p.T && col >= 0 && col < B)
+          p.xc[(size_t)(t0 + q) * p.Kc + p.K + e] = __float2half_rn(xr[q][col]);
+      }
+    }
+    // t += xr_block (16 x B) . V_block^T (B x 8) per n-tile of 8 ranks
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int nt = warp + NW * j;
+      if (nt >= ntiles) break;
+      const int n = 8 * nt + g;
+#pragma unroll 4
+      for (int k0 = 0; k0 < B; k0 += 16) {
+        uint32_t a[4];
+        a[0] = *reinterpret_cast<const uint32_t *>(&xh[g][k0 + 2 * tig]);
+        a[1] = *reinterpret_cast<const uint32_t *>(&xh[g + 8][k0 + 2 * tig]);
+        a[2] = *reinterpret_cast<const uint32_t *>(&xh[g][k0 + 2 * tig + 8]);
+        a[3] = *reinterpret_cast<const uint32_t *>(&xh[g + 8][k0 + 2 * tig + 8]);
+        const uint32_t b0 = n < p.rank ? *reinterpret_cast<const uint32_t *>(&vh[n][k0 + 2 * tig]) : 0u;
+        const uint32_t b1 =
+            n < p.rank ? *reinterpret_cast<const uint32_t *>(&vh[n][k0 + 2 * tig + 8]) : 0u;
+        mma_16816(tacc[j], a, b0, b1, tacc[j]);
+      }
+    }
+    __syncthreads();
+  }
+  // t and the zero padding of the salient and low-rank sections
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int nt = warp + NW * j;
+    if (nt >= ntiles) break;
+    const int n = 8 * nt + 2 * tig;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int q = g + 8 * (i >> 1), rr = n + (i & 1);
+      if (t0 + q < p.T && rr < p.rank)
+        p.xc[(size_t)(t0 + q) * p.Kc + p.K + p.salp + rr] = __float2half_rn(tacc[j][i]);
+    }
+  }
+  const int npad1 = p.salp - p.n_sal, npad2 = 64 - p.rank;
+  for (int i = tid; i < 16 * (npad1 + npad2); i += B) {
+    const int q = i / (npad1 + npad2), j = i % (npad1 + npad2);
+    if (t0 + q >= p.T) continue;
+    const int col = j < npad1 ? p.K + p.n_sal + j : p.K + p.salp + p.rank + (j - npad1);
+    p.xc[(size_t)(t0 + q) * p.Kc + col] = __float2half_rn(0.0f);
+  }
+}
+
+// ----------------------------------------------------------------- pre_gemm
+// One producer thread per tile row writes the 64 FP16 operands of a stage as
+// eight 16-byte chunks in the 128B-swizzled K-major layout.
+__device__ __forceinline__ void store_row_sw128(uint8_t *stage, int row, const uint32_t h[32]) {
+  uint8_t *rp = stage + row * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+    *reinterpret_cast<uint4 *>(rp + ((c ^ (row & 7)) << 4)) = v;
+  }
+}
+
+// 8 nibbles (two's complement) of word w times scale s -> 4 FP16 pairs in
+// column order (n0,n1), (n2,n3), (n4,n5), (n6,n7); exact for FP16-safe s.
+__device__ __forceinline__ void dequant_q4_scaled(uint32_t w, __half2 s2, uint32_t out[4]) {
+  const uint32_t u = w ^ 0x88888888u;
+  const uint32_t magic = 0x64006400u;
+  const __half2 sub_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  const __half2 mul_hi = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+  const __half2 sub_hi = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+  uint32_t l0 = (u & 0x000F000Fu) | magic;
+  uint32_t h0 = (u & 0x00F000F0u) | magic;
+  uint32_t l1 = ((u >> 8) & 0x000F000Fu) | magic;
+  uint32_t h1 = ((u >> 8) & 0x00F000F0u) | magic;
+  __half2 p0 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&l0), sub_lo), s2);          // (n0,n4)
+  __half2 p1 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&h0), mul_hi, sub_hi), s2);   // (n1,n5)
+  __half2 p2 = __hmul2(__hsub2(*reinterpret_cast<__half2 *>(&l1), sub_lo), s2);          // (n2,n6)
+  __half2 p3 = __hmul2(__hfma2(*reinterpret_cast<__half2 *>(&h1), mul_hi, sub_hi), s2);   // (n3,n7)
+  const uint32_t a = *reinterpret_cast<uint32_t *>(&p0), b = *reinterpret_cast<uint32_t *>(&p1);
+  const uint32_t c = *reinterpret_cast<uint32_t *>(&p2), d = *reinterpret_cast<uint32_t *>(&p3);
+  out[0] = __byte_perm(a, b, 0x5410);   // (n0, n1)
+  out[1] = __byte_perm(c, d, 0x5410);   // (n2, n3)
+  out[2] = __byte_perm(a, b, 0x7632);   // (n4, n5)
+  out[3] = __byte_perm(c, d, 0x7632);   // (n6, n7)
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
+    const __grid_constant__ CUtensorMap mxc, PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  constexpr int A_STAGE = kPreBM * 128;
+  constexpr int B_STAGE = BN * 128;
+  uint8_t *sa = base;
+  uint8_t *sb = base + kPreStages * A_STAGE;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sb + kPreStages * B_STAGE);
+  uint64_t *empty = full + kPreStages;
+  uint64_t *accum = empty + kPreStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * kPreBM, n0 = blockIdx.y * BN;
+  const int S = p.nstages;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPreStages; ++s) {
+      mbar_init(&full[s], 129);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------- activation operand producer (TMA) ----------------
+    if (lane == 0) {
+      prefetch_tensormap(&mxc);
+      for (int s = 0; s < S && ok; ++s) {
+        const int slot = s % kPreStages, round = s / kPreStages;
+        if (!mbar_wait(&empty[slot], (round & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[slot], B_STAGE);
+        tma_load_2d(sb + slot * B_STAGE, &mxc, 64 * s, n0, &full[slot]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------- MMA issuer -----------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_f16(kPreBM, BN);
+      for (int s = 0; s < S && ok; ++s) {
+        const int slot = s % kPreStages, round = s / kPreStages;
+        if (!mbar_wait(&full[slot], round & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sa + slot * A_STAGE), b0 = smem_u32(sb + slot * B_STAGE);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc_mma_f16(tmem, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k), idesc,
+                     (s > 0 || k > 0) ? 1u : 0u);
+        tc_commit(&empty[slot]);
+      }
+      tc_commit(accum);
+    }
+  } else {
+    // ------------- weight operand producers, then the epilogue -------------
+    const int i = tid - 64;              // tile row 0..127
+    const int m = m0 + i;
+    const bool rowok = m < p.M;
+    const int KG = p.K / 64;
+    uint4 cur0 = make_uint4(0, 0, 0, 0), cur1 = cur0;
+    uint16_t cur_s = 0;
+    auto load_q4 = [&](int s, uint4 &w0, uint4 &w1, uint16_t &sc) {
+      if (rowok && s < p.nq4) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.q4 + (size_t)m * (p.K / 2) + 32 * s);
+        w0 = __ldg(src);
+        w1 = __ldg(src + 1);
+        sc = p.s4[(size_t)m * KG + s];
+      }
+    };
+    load_q4(0, cur0, cur1, cur_s);
+    const float s8f = rowok && p.n_sal > 0 ? bf16_bits_to_f32(p.s8[m]) : 0.0f;
+    for (int s = 0; s < S && ok; ++s) {
+      const int slot = s % kPreStages, round = s / kPreStages;
+      uint4 nx0 = make_uint4(0, 0, 0, 0), nx1 = nx0;
+      uint16_t nx_s = 0;
+      load_q4(s + 1, nx0, nx1, nx_s);
+      uint32_t h[32];
+      if (!rowok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) h[j] = 0u;
+      } else if (s < p.nq4) {
+        const __half sh = __float2half_rn(bf16_bits_to_f32(cur_s));
+        const __half2 s2 = __halves2half2(sh, sh);
+        const uint32_t wv[8] = {cur0.x, cur0.y, cur0.z, cur0.w, cur1.x, cur1.y, cur1.z, cur1.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dequant_q4_scaled(wv[q], s2, h + 4 * q);
+      } else if (s < p.nq4 + p.nsal) {
+        const int e0 = 64 * (s - p.nq4);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 raw = make_uint4(0, 0, 0, 0);
+          if (e0 + 16 * q < p.n_sal)
+            raw = __ldg(reinterpret_cast<const uint4 *>(p.q8 + (size_t)m * p.n_sal + e0 + 16 * q));
+          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t w = wv[u];
+            const float f0 = (float)(int8_t)(w & 0xFF) * s8f, f1 = (float)(int8_t)((w >> 8) & 0xFF) * s8f;
+            const float f2 = (float)(int8_t)((w >> 16) & 0xFF) * s8f, f3 = (float)(int8_t)(w >> 24) * s8f;
+            h[8 * q + 2 * u] = pack_half2(__float2half_rn(f0), __float2half_rn(f1));
+            h[8 * q + 2 * u + 1] = pack_half2(__float2half_rn(f2), __float2half_rn(f3));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int r0 = 2 * j, r1 = 2 * j + 1;
+          const float u0 = r0 < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + r0]) : 0.0f;
+          const float u1 = r1 < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + r1]) : 0.0f;
+          h[j] = pack_half2(__float2half_rn(u0), __float2half_rn(u1));
+        }
+      }
+      if (!mbar_wait(&empty[slot], (round & 1) ^ 1)) { ok = false; break; }
+      store_row_sw128(sa + slot * A_STAGE, i, h);
+      fence_proxy_async_smem();
+      mbar_arrive(&full[slot]);
+      cur0 = nx0; cur1 = nx1; cur_s = nx_s;
+    }
+    // ------------------------------ epilogue ------------------------------
+    if (ok && mbar_wait(accum, 0)) {
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int row = m0 + 32 * quarter + lane;
+      const float bv = (p.bias != nullptr && row < p.M) ? bf16_bits_to_f32(p.bias[row]) : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + 16 * c, r);
+        tmem_ld_wait();
+        if (row < p.M) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tok = n0 + 16 * c + j;
+            if (tok < p.T) {
+              const float v = __uint_as_float(r[j]) + bv;
+              if (p.y_bf16)
+                reinterpret_cast<uint16_t *>(p.y)[(size_t)tok * p.M + row] = f32_to_bf16_rn_bits(v);
+              else
+                reinterpret_cast<float *>(p.y)[(size_t)tok * p.M + row] = v;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+// ---------------------------------------------------------------- host ---
+static int pre_bn(int T) { return T > 128 ? 256 : (T > 64 ? 128 : 64); }
+
+static size_t pre_smem_bytes(int BN) {
+  return 1024 + (size_t)kPreStages * (kPreBM * 128 + BN * 128) + 256;
+}
+
+size_t prefill_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T) {
+  (void)M; (void)block; (void)rank;
+  const int salp = (n_sal + 63) / 64 * 64;
+  const size_t Kc = (size_t)K + salp + 64;
+  return ((size_t)T * Kc * 2 + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
+  PrefillParams p;
+  p.M = a.M; p.K = a.K; p.T = a.T; p.n_sal = a.n_sal; p.rank = a.rank;
+  p.salp = (a.n_sal + 63) / 64 * 64;
+  p.Kc = a.K + p.salp + 64;
+  p.nq4 = a.K / 64;
+  p.nsal = p.salp / 64;
+  p.nstages = p.nq4 + p.nsal + (a.rank > 0 ? 1 : 0);
+  p.c = (float)sqrt(1.0 / (double)a.block);
+  p.q4 = a.q4; p.s4 = a.s4; p.sal_idx = a.sal_idx; p.q8 = a.q8; p.s8 = a.s8;
+  p.U = a.U; p.V = a.V; p.x = a.x; p.bias = a.bias; p.y = a.y; p.y_bf16 = a.y_bf16;
+  p.xc = reinterpret_cast<__half *>(a.workspace);
+
+  const size_t act_smem = pre_act_smem_bytes(a.block, a.rank, a.n_sal);
+  cudaError_t e;
+  dim3 ga((a.T + 15) / 16);
+  if (a.block == 256)
+    e = L.launch("pre_act", pre_act_kernel<256>, ga, dim3(256), act_smem, st, false, p);
+  else
+    e = L.launch("pre_act", pre_act_kernel<128>, ga, dim3(128), act_smem, st, false, p);
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap mxc;
+  const int BN = pre_bn(a.T);
+  if (encode_tmap_2d(&mxc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.xc, (uint64_t)p.Kc, (uint64_t)a.T,
+                     (uint64_t)p.Kc * 2, 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  dim3 gg((a.M + kPreBM - 1) / kPreBM, (a.T + BN - 1) / BN);
+  const size_t smem = pre_smem_bytes(BN);
+  if (BN == 256)
+    return L.launch("pre_gemm", pre_gemm_kernel<256>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
+  if (BN == 128)
+    return L.launch("pre_gemm", pre_gemm_kernel<128>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
+  return L.launch("pre_gemm", pre_gemm_kernel<64>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
+}
+
+cudaError_t prepare_prefill_kernels() {
+  cudaError_t e;
+  e = cudaFuncSetAttribute(pre_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)pre_smem_bytes(256));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pre_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)pre_smem_bytes(128));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pre_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)pre_smem_bytes(64));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pre_act_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)pre_act_smem_bytes(256, 64, kMaxSalient));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(pre_act_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)pre_act_smem_bytes(128, 64, kMaxSalient));
+}
+
+}  // namespace dvssq

@@ -10,6 +10,9 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+    # the CUDA library is built in-tree (nvcc cross-compiles without a GPU)
+    from mixed_precision_weight_b200 import build
+    build.build()
 
 
 def pytest_collection_modifyitems(config, items):
