@@ -106,22 +106,27 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.3)   # let the sampler start before the timed region
         return self
 
     def __exit__(self, *a):
-        self.out = ""
+        self.out, self.err = "", ""
         if self.proc is not None:
+            time.sleep(0.25)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.out, self.err = self.proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.out, self.err = self.proc.communicate()
+            if not self.out.strip():
+                print(f"clock sampler produced no samples: {self.err.strip()[:300]}",
+                      file=sys.stderr)
 
     def summary(self):
         sm, mx, reasons = [], [], set()
@@ -352,7 +357,9 @@ def main():
             gbs = b / (avg * 1e-3) / 1e9
             ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
         kernels[name] = ent
-    dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
+    # dominant kernel among those with an algorithmic byte count
+    dom = max((kv for kv in prof.items() if kernel_bytes(kv[0], M, K, r, n, 16) is not None),
+              key=lambda kv: kv[1][1])[0]
     db = kernel_bytes(dom, M, K, r, n, 16)
     dom_avg_ms = prof[dom][1] / prof[dom][0]
     achieved = db / (dom_avg_ms * 1e-3) / 1e9
