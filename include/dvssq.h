@@ -203,6 +203,34 @@ DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvss
                                   void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* Allocation-free decode forward.  The paper has no counterpart: this entry
+ * exists for callers that cannot obtain device memory for a workspace --
+ * for example a host program that links only this library and has no device
+ * allocator of its own, or a plug-in host that hands its plug-ins fixed input
+ * and output buffers and forbids them to allocate.  It computes the same
+ * result as dvssq_linear_forward with path DVSSQ_PATH_DECODE (1 <= T <= 16;
+ * T == 0 is a no-op), but its scratch lives in a fixed array of
+ * DVSSQ_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *   - Shapes whose decode workspace (dvssq_forward_workspace_size with
+ *     DVSSQ_PATH_DECODE) exceeds DVSSQ_STATIC_SCRATCH_BYTES are rejected with
+ *     DVSSQ_ERR_WORKSPACE before any launch; dvssq_last_error() then states
+ *     the bytes needed and the limit.  T > 16 returns UNSUPPORTED_SHAPE.
+ *   - The first call on a device looks up the array's device address
+ *     (once per device, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (the kernels clear what must start at zero).  Calls that may overlap
+ *     on the GPU -- concurrent streams, other host threads -- race on it
+ *     and must be serialised by the caller.
+ * Other arguments and errors as dvssq_linear_forward.                        */
+#define DVSSQ_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+DVSSQ_API dvssq_status dvssq_linear_forward_static(const dvssq_shape *shape,
+                                                   const dvssq_weights *w, const void *x,
+                                                   int64_t T, const void *bias, void *y,
+                                                   int32_t y_dtype, void *stream);
+
 /* Reads (and clears when `clear` != 0) the device error word of the current
  * device; synchronises the device.  0 means no kernel gave up a wait.     */
 DVSSQ_API dvssq_status dvssq_device_error(uint32_t *word, int32_t clear);

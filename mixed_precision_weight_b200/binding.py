@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
     "dvssq_fwht", "dvssq_encode_workspace_size", "dvssq_encode",
-    "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_device_error",
+    "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
+    "dvssq_device_error", "STATIC_SCRATCH_BYTES",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
     "dvssq_profile_reset", "Y_F32", "Y_BF16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
     "EXPORTED_SYMBOLS",
@@ -45,7 +46,8 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 EXPORTED_SYMBOLS = (
     "dvssq_abi_version", "dvssq_status_string", "dvssq_last_error", "dvssq_fwht",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
-    "dvssq_linear_forward", "dvssq_device_error", "dvssq_profile_enable",
+    "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_device_error",
+    "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
     "dvssq_profile_reset",
 )
@@ -90,6 +92,8 @@ _sig = {
     "dvssq_linear_forward": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights), _P,
                                             ctypes.c_int64, _P, _P, ctypes.c_int32, ctypes.c_int32,
                                             _P, ctypes.c_size_t, _P]),
+    "dvssq_linear_forward_static": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights),
+                                                   _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "dvssq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "dvssq_profile_enable": (ctypes.c_int, [ctypes.c_int32]),
     "dvssq_profile_collect": (ctypes.c_int, []),
@@ -110,7 +114,7 @@ class DvssqError(RuntimeError):
         self.status = status
         msg = lib.dvssq_status_string(status).decode()
         detail = lib.dvssq_last_error().decode()
-        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail and status == 5 else ""))
+        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail and status in (4, 5) else ""))
 
 
 def _check(status: int, where: str):
@@ -231,6 +235,28 @@ def dvssq_linear_forward(shape: Shape, w: PackedWeights, x: torch.Tensor,
                                     _ptr(y), y_dtype, path, _ptr(workspace), workspace.numel(),
                                     _stream(stream)), "dvssq_linear_forward")
     return y
+
+
+def dvssq_linear_forward_static(shape: Shape, w: PackedWeights, x: torch.Tensor,
+                                bias: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                                y_dtype: int = Y_F32, stream=None):
+    """The decode forward (T <= 16) using the library's fixed internal scratch.
+
+    For callers that cannot allocate a workspace; see dvssq.h for the size
+    limit and the rule that overlapping calls must be serialised.
+    """
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, shape.M), dtype=torch.float32 if y_dtype == Y_F32 else torch.bfloat16,
+                        device=x.device)
+    wc = w._c(shape)
+    _check(lib.dvssq_linear_forward_static(ctypes.byref(shape), ctypes.byref(wc), _ptr(x), T,
+                                           _ptr(bias), _ptr(y), y_dtype, _stream(stream)),
+           "dvssq_linear_forward_static")
+    return y
+
+
+STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 def dvssq_device_error(clear: bool = True) -> int:

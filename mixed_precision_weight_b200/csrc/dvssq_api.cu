@@ -104,6 +104,8 @@ EncodeTiledFn tiled_encoder() {
 
 }  // namespace
 
+void set_last_error(const std::string &msg) { t_last_error = msg; }
+
 CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                         uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {

@@ -57,6 +57,7 @@ class Launcher {
 };
 
 Launcher &launcher();
+void set_last_error(const std::string &msg);
 
 // --------------------------------------------------------------- encoder ---
 struct EncodeArgs {

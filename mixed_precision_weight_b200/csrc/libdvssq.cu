@@ -5,3 +5,4 @@
 #include "encode.cu"
 #include "decode.cu"
 #include "prefill.cu"
+#include "static_scratch.cu"
