@@ -30,9 +30,10 @@ R2  W_rot[i, kb+j] = RN64(c_b * RN64(sum_l S_b[j,l] W[i, kb+l])): the +-1 sum
     is taken exactly and the scale is applied once, after the sum.
 R3  Salience follows the task's fixed choice: the L2 norm of each *rotated*
     column times a per-channel activation scale a_j (indexed by rotated
-    column).  The column sum of squares uses a fixed order: rows in chunks of
-    SSQ_CHUNK, within a chunk acc = acc + w*w (product and sum each rounded),
-    chunk partials added in ascending chunk order.
+    column).  The column sum of squares uses a fixed summation tree: rows in
+    chunks of SSQ_CHUNK, within a chunk acc = acc + w*w (product and sum each
+    rounded); chunk sums added in order within groups of SSQ_GROUP chunks;
+    group sums added in ascending order.
 R4  Top-k: n_sal largest scores, ties broken toward the lower column index;
     returned ascending.
 R5  INT4 groups are 64 contiguous rotated columns over the full K ("dense"
@@ -56,7 +57,8 @@ from fractions import Fraction
 
 import numpy as np
 
-SSQ_CHUNK = 64          # R3: rows per fixed-order partial of the column sum of squares
+SSQ_CHUNK = 16          # R3: rows per fixed-order partial of the column sum of squares
+SSQ_GROUP = 8           # R3: chunk sums per second-level partial
 GROUP = 64              # Tier B / §2: group size G = 64
 SAL_DEN = 8             # Tier A: top 12.5 % = 1/8 of the input channels
 
@@ -137,8 +139,12 @@ def hadamard(b: int) -> np.ndarray:
 
 
 def _bf16_exponent_lsb(v: np.ndarray):
-    """(floor(log2|v|), log2 of the last significand bit) for nonzero BF16 values."""
-    e = np.floor(np.log2(np.abs(v))).astype(np.int64)
+    """(exponent, log2 of the last significand bit) of nonzero BF16 values.
+
+    The exponent is floor(log2|v|) for normal values and -127 for subnormal
+    ones (an upper bound, so the exactness test stays sufficient).
+    """
+    e = np.maximum(np.floor(np.log2(np.abs(v))).astype(np.int64), -127)
     lsb = np.maximum(e - 7, -133)
     return e, lsb
 
@@ -213,16 +219,22 @@ def fwht(x: np.ndarray, b: int) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
-def column_ssq(W_rot: np.ndarray, chunk: int = SSQ_CHUNK) -> np.ndarray:
-    """R3: per-column sum of squares in the fixed chunked order."""
+def column_ssq(W_rot: np.ndarray, chunk: int = SSQ_CHUNK, group: int = SSQ_GROUP) -> np.ndarray:
+    """R3: per-column sum of squares in the fixed three-level order."""
     M, K = W_rot.shape
-    total = np.zeros(K, dtype=np.float64)
+    chunk_sums = []
     for c0 in range(0, M, chunk):
         part = np.zeros(K, dtype=np.float64)
         for i in range(c0, min(c0 + chunk, M)):
             w = W_rot[i]
             part = part + w * w
-        total = total + part
+        chunk_sums.append(part)
+    total = np.zeros(K, dtype=np.float64)
+    for g0 in range(0, len(chunk_sums), group):
+        gsum = np.zeros(K, dtype=np.float64)
+        for part in chunk_sums[g0:g0 + group]:
+            gsum = gsum + part
+        total = total + gsum
     return total
 
 
