@@ -252,6 +252,161 @@ class SparkDownStep:
         return step
 
 
+class DecodeStep(SparkDownStep):
+    """forward(T=1) + forward(T=16) only, on rotating pre-encoded copies."""
+
+    name = "spark_down_proj_2560x10240_r16_fwd_T1+T16"
+
+    def step(self):
+        dv = self.dv
+        fwd = self.copies[self.i % N_COPIES][2]
+        dv.dvssq_linear_forward(self.shape, fwd, self.x1, y=self.y1, workspace=self.ws1)
+        dv.dvssq_linear_forward(self.shape, fwd, self.x16, y=self.y16, workspace=self.ws16)
+        self.i += 1
+
+    def bytes_per_step(self):
+        return 2 * packed_bytes(self.M, self.K, self.r, self.n)
+
+    def launches_per_step(self):
+        return 4
+
+    def config(self):
+        c = super().config()
+        c.update(workload=self.name,
+                 step="dvssq_linear_forward(T=1) + dvssq_linear_forward(T=16)",
+                 l2=f"{N_COPIES} rotating encoded layers (~{N_COPIES * 18} MB) > 126 MB L2")
+        return c
+
+    def e2e_step(self):
+        # tokens in from pinned host memory, outputs back to the host
+        layer = self.dv.DvssqLinear(self.shape, self.copies[self.i % N_COPIES][2])
+        self.hy1.copy_(layer(self.hx1), non_blocking=True)
+        self.hy16.copy_(layer(self.hx16), non_blocking=True)
+        self.i += 1
+
+    def e2e_bytes(self):
+        return ((self.hx1.numel() + self.hx16.numel()) * 2,
+                (self.hy1.numel() + self.hy16.numel()) * 4)
+
+    def oracle_sample(self, O, synth):
+        wl = self.wl
+        enc = O.encode(O.torch_bf16_to_f64(wl.weight(seed_offset=555)),
+                       wl.act_scale(seed_offset=555).numpy(), wl.block, self.r, with_svd=False)
+        U, V = synth.lowrank_factors(self.M, self.K, self.r, seed=55)
+        Uf, Vf = O.torch_bf16_to_f64(U), O.torch_bf16_to_f64(V)
+        x1 = O.torch_bf16_to_f64(wl.activations(1))
+        x16 = O.torch_bf16_to_f64(wl.activations(16))
+
+        def step():
+            O.forward(enc, x1, U=Uf, V=Vf)
+            O.forward(enc, x16, U=Uf, V=Vf)
+        return step
+
+
+class PrefillStep:
+    """forward of 4096 tokens through the Spark up_proj layer (tensor cores)."""
+
+    name = "spark_up_proj_10240x2560_r16_prefill_T4096"
+    unit = "TFLOP/s"
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv, self.torch = dv, torch
+        wl = synth.WORKLOADS["spark_up_prefill"]
+        self.wl = wl
+        self.M, self.K, self.r, self.n, self.T = wl.M, wl.K, wl.rank, wl.n_sal, 4096
+        self.shape = dv.Shape.make(wl.M, wl.K, wl.block, wl.rank)
+        U, V = synth.lowrank_factors(wl.M, wl.K, wl.rank, seed=wl.seed + rank_id)
+        self.packed = dv.PackedWeights.empty(self.shape, device, U=U.to(device), V=V.to(device))
+        dv.dvssq_encode(self.shape, wl.weight(seed_offset=rank_id).to(device),
+                        wl.act_scale(seed_offset=rank_id).to(device), self.packed)
+        self.x = wl.activations(self.T, seed_offset=rank_id).to(device)
+        self.ws = torch.empty(dv.dvssq_forward_workspace_size(self.shape, self.T), dtype=torch.uint8,
+                              device=device)
+        self.y = torch.empty((self.T, self.M), dtype=torch.float32, device=device)
+
+    def step(self):
+        self.dv.dvssq_linear_forward(self.shape, self.packed, self.x, y=self.y, workspace=self.ws)
+
+    def work_per_step(self):
+        return 2.0 * self.T * self.M * self.K + 2.0 * self.T * self.r * (self.K + self.M)
+
+    def kernel_work(self, name):
+        if name == "pre_gemm":
+            return self.work_per_step()
+        if name == "pre_act":
+            salp = (self.n + 63) // 64 * 64
+            return self.T * self.K * 2 + self.T * (self.K + salp + 64) * 2
+        return None
+
+    def launches_per_step(self):
+        return 2
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "K": self.K, "block": 256, "rank": self.r,
+                "n_sal": self.n, "tokens": self.T,
+                "step": "dvssq_linear_forward(T=4096) on tcgen05",
+                "flops": "2*T*M*K + 2*T*r*(K+M) (algorithmic; the kernel also multiplies the "
+                         "dense-layout zeros and the salient tier)",
+                "l2": "x (21 MB) + packed layer (17.6 MB); each step reruns the same layer",
+                "parallelism": "replica per GPU"}
+
+
+class BulkEncodeStep:
+    """encode of all 108 MLP matrices of the 36-layer Spark shape (one pass)."""
+
+    name = "spark_mlp_36x3_bulk_encode"
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv, self.torch = dv, torch
+        H, I = 2560, 10240
+        # four BF16 sources per shape (4 x 3 x 52 MB > L2), used in rotation so
+        # that every encode reads its matrix from HBM
+        gen_cache = {}
+        for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
+            for c in range(4):
+                W = synth.weight(M, K, seed=10 + which + 7 * c + 100 * rank_id,
+                                 n_outlier_cols=max(1, K // 1000), outlier_scale=15.0).to(device)
+                act = synth.act_scale(K, seed=20 + which + 7 * c).to(device)
+                gen_cache[(which, c)] = (W, act)
+        self.shapes = {w: dv.Shape.make(M, K, 256, 16) for w, (M, K) in
+                       enumerate(((I, H), (I, H), (H, I)))}
+        self.packed = {w: dv.PackedWeights.empty(self.shapes[w], device) for w in range(3)}
+        self.src = gen_cache
+        ws = max(dv.dvssq_encode_workspace_size(sh) for sh in self.shapes.values())
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.H, self.I = H, I
+
+    def step(self):
+        for layer in range(36):
+            for w in range(3):
+                W, act = self.src[(w, layer % 4)]
+                self.dv.dvssq_encode(self.shapes[w], W, act, self.packed[w], workspace=self.ws)
+
+    def bytes_per_step(self):
+        H, I = self.H, self.I
+        return 36 * (2 * encode_bytes(I, H, H // 8) + encode_bytes(H, I, I // 8))
+
+    def launches_per_step(self):
+        return 108 * 5
+
+    def kernel_work(self, name):
+        H, I = self.H, self.I
+        per = {"enc_pass1": (2 * I * H * 2 + H * I * 2) / 3,
+               "enc_pass2": (2 * encode_bytes(I, H, H // 8) + encode_bytes(H, I, I // 8)) / 3}
+        return per.get(name)
+
+    def config(self):
+        return {"workload": self.name, "matrices": 108, "weights": 108 * 2560 * 10240,
+                "step": "dvssq_encode of 36 x (gate, up, down)",
+                "l2": "each matrix's BF16 source (52 MB) is read from HBM by pass 1; "
+                      "pass 2 re-reads it, partly from L2",
+                "parallelism": "replica per GPU"}
+
+
+WORKLOADS = {"spark_down": SparkDownStep, "decode": DecodeStep, "prefill": PrefillStep,
+             "bulk_encode": BulkEncodeStep}
+
+
 # -------------------------------------------------------------------- main --
 
 def threads_used():
@@ -304,7 +459,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device(device))
-    work = SparkDownStep(dv, synth, torch, rank, device)
+    work = WORKLOADS[args.workload](dv, synth, torch, rank, device)
+    unit = getattr(work, "unit", "GB/s")
     W = max(3, args.warmup)
     for _ in range(W):
         work.step()
@@ -332,8 +488,12 @@ def main():
         ms = float(t.item())
     err = dv.dvssq_device_error(clear=True)
     ms_step = ms / args.steps
-    bytes_step = work.bytes_per_step()
-    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    if unit == "TFLOP/s":
+        bytes_step = None
+        value = world * work.work_per_step() / (ms_step * 1e-3) / 1e12
+    else:
+        bytes_step = work.bytes_per_step()
+        value = world * bytes_step / (ms_step * 1e-3) / 1e9
 
     # per-kernel device times: the same K steps again with events around each launch
     dv.dvssq_profile_reset()
@@ -346,34 +506,47 @@ def main():
     prof = dv.dvssq_profile_read()
     pk, pk_kind = peaks()
     kernels = {}
-    M, K, r, n = work.M, work.K, work.r, work.n
     tot_ms = sum(v[1] for v in prof.values())
+    kb_fn = getattr(work, "kernel_work", None) or (
+        lambda name: kernel_bytes(name, work.M, work.K, work.r, work.n, 16))
     for name, (cnt, kms) in prof.items():
         avg = kms / cnt
         ent = {"launches": cnt, "avg_us": round(avg * 1e3, 3), "share": round(kms / tot_ms, 4)}
-        calls_T = 16 if name == "dec_prologue" else 1
-        b = kernel_bytes(name, M, K, r, n, calls_T)
+        b = kb_fn(name)
         if b is not None:
-            gbs = b / (avg * 1e-3) / 1e9
-            ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
+            if name == "pre_gemm":
+                tfs = b / (avg * 1e-3) / 1e12
+                ent.update(flops=b, tflops=round(tfs, 1),
+                           frac=round(tfs / pk["bf16_tflops_sustained"], 4))
+            else:
+                gbs = b / (avg * 1e-3) / 1e9
+                ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
         kernels[name] = ent
-    # dominant kernel among those with an algorithmic byte count
-    dom = max((kv for kv in prof.items() if kernel_bytes(kv[0], M, K, r, n, 16) is not None),
-              key=lambda kv: kv[1][1])[0]
-    db = kernel_bytes(dom, M, K, r, n, 16)
+    # dominant kernel among those with an algorithmic work count
+    dom = max((kv for kv in prof.items() if kb_fn(kv[0]) is not None), key=lambda kv: kv[1][1])[0]
+    db = kb_fn(dom)
     dom_avg_ms = prof[dom][1] / prof[dom][0]
-    achieved = db / (dom_avg_ms * 1e-3) / 1e9
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": pk["hbm_gbs"], "peak_source": pk_kind, "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4),
-                "traffic": dram_traffic(dom, args.workload),
-                "algorithmic_bytes_per_launch": db}
+    if dom == "pre_gemm":
+        achieved = db / (dom_avg_ms * 1e-3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": pk["bf16_tflops_sustained"],
+                    "peak_source": pk_kind + " (bf16 sustained; f16 has the same dense rate)",
+                    "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
+                    "traffic": dram_traffic(dom, args.workload),
+                    "algorithmic_flops_per_launch": db}
+    else:
+        achieved = db / (dom_avg_ms * 1e-3) / 1e9
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": pk["hbm_gbs"], "peak_source": pk_kind, "unit": "GB/s",
+                    "frac": round(achieved / pk["hbm_gbs"], 4),
+                    "traffic": dram_traffic(dom, args.workload),
+                    "algorithmic_bytes_per_launch": db}
     # the decode GEMV's own roofline (the headline HBM-bound kernel)
     dm = kernels.get("dec_main")
 
     # end-to-end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and hasattr(work, "e2e_step"):
         work.e2e_setup(synth)
         for _ in range(2):
             work.e2e_step()
@@ -396,7 +569,7 @@ def main():
                "ms_per_step": round(ems, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(work, "oracle_sample"):
         from oracle import dvssq_oracle as O
         nst, dt = run_oracle(work, O, synth)
         cpu = {"value": round(bytes_step * nst / dt / 1e9, 4), "unit": "GB/s",
@@ -404,7 +577,7 @@ def main():
                "sample": f"{nst} full step(s) of the same workload (encode without SVD + "
                          f"2 forwards) on the host, {dt:.1f} s"}
 
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+    line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": W, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp16",
             "data": "synthetic (seeded N(0,0.02) weights with outlier columns, N(0,1) tokens)",

@@ -177,7 +177,7 @@ dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes
   dvssq_status s = check_shape(shape);
   if (s != DVSSQ_OK) return s;
   if (bytes == nullptr) return DVSSQ_ERR_INVALID_ARG;
-  *bytes = encode_workspace_bytes(shape->M, shape->K);
+  *bytes = encode_workspace_bytes(shape->M, shape->K, shape->n_sal);
   return DVSSQ_OK;
 }
 
@@ -195,7 +195,7 @@ dvssq_status dvssq_encode(const dvssq_shape *shape, const void *W, const float *
   for (const void *b : bufs)
     if (b != nullptr && !aligned16(b)) return DVSSQ_ERR_MISALIGNED;
   if (!aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
-  if (workspace_bytes < encode_workspace_bytes(shape->M, shape->K)) return DVSSQ_ERR_WORKSPACE;
+  if (workspace_bytes < encode_workspace_bytes(shape->M, shape->K, shape->n_sal)) return DVSSQ_ERR_WORKSPACE;
   if ((s = ensure_device()) != DVSSQ_OK) return s;
   EncodeArgs a;
   a.M = shape->M; a.K = shape->K; a.block = shape->block; a.n_sal = shape->n_sal;

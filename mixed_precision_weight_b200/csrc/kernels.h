@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 #include <vector>
 
 namespace dvssq {
@@ -26,21 +27,31 @@ class Launcher {
   bool profiling = false;
   std::vector<ProfileRecord> pending;
 
+  // cluster_y > 0 launches thread-block clusters of (1, cluster_y, 1).
   template <typename... KArgs, typename... Args>
-  cudaError_t launch(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
-                     size_t smem, cudaStream_t st, bool pdl, Args &&...args) {
+  cudaError_t launch_ex(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                        size_t smem, cudaStream_t st, bool pdl, int cluster_y, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if (pdl && !profiling) {
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
+      attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[na].val.programmaticStreamSerializationAllowed = 1;
+      ++na;
     }
+    if (cluster_y > 0) {
+      attr[na].id = cudaLaunchAttributeClusterDimension;
+      attr[na].val.clusterDim.x = 1;
+      attr[na].val.clusterDim.y = (unsigned)cluster_y;
+      attr[na].val.clusterDim.z = 1;
+      ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
     ProfileRecord rec{name, nullptr, nullptr};
     if (profiling) {
       cudaEventCreate(&rec.start);
@@ -53,6 +64,12 @@ class Launcher {
       pending.push_back(rec);
     }
     return e;
+  }
+
+  template <typename... KArgs, typename... Args>
+  cudaError_t launch(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                     size_t smem, cudaStream_t st, bool pdl, Args &&...args) {
+    return launch_ex(name, kernel, grid, block, smem, st, pdl, 0, std::forward<Args>(args)...);
   }
 };
 
@@ -73,8 +90,7 @@ struct EncodeArgs {
   int64_t *info_host;  // 3 counters or nullptr
   void *workspace;
 };
-size_t encode_workspace_bytes(int M, int K);
-int pass2_rows_per_cta(int block, int n_sal);
+size_t encode_workspace_bytes(int M, int K, int n_sal);
 cudaError_t prepare_encode_kernels();
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L);
 

@@ -428,6 +428,10 @@ cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
 
 cudaError_t prepare_prefill_kernels() {
   cudaError_t e;
+  for (const void *f : {(const void *)pre_act_kernel<256>, (const void *)pre_act_kernel<128>})
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
   e = cudaFuncSetAttribute(pre_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)pre_smem_bytes(256));
   if (e != cudaSuccess) return e;
