@@ -2,45 +2,68 @@
 // equation of the MiniCPM5-2B-Hadamard-GSQ card (§2, Y = X What^T + (X B^T)
 // A^T) with the Spark card's INT8 salient tier, on the packed form.
 //
-// Two launches, chained by programmatic dependent launch:
-//   dec_prologue  one CTA per Hadamard block: xr = H_b x in fp32 (16-thread
-//                 Kronecker FWHT), written as FP16 in the GEMV's k-order; the
-//                 salient entries xs = xr[sal_idx]; the block's partial of
-//                 t = V xr; zeroes the split-K arrival counters.
-//   dec_main      CTA tile = 64 rows x (1024 * NR) columns.  TMA brings the
-//                 CTA's whole q8 slice (64B swizzle) and q4 tile (128B
-//                 swizzle) into shared memory at once, before the kernel
-//                 waits on the prologue, so the weight stream overlaps it.
-//                 Each warp owns 128-column slices of all 64 rows.  The
-//                 salient tier runs first: exact FP16 INT8 codes x xs on
-//                 mma.sync, scaled by s8 in FP32.  Then per 64-column group:
-//                 nibbles -> exact FP16 codes in registers -> mma.sync
-//                 m16n8k16 with FP32 accumulation -> acc += s4 * group sum.
-//                 Warps reduce in shared memory and the CTA adds U (its own
-//                 slice of t), so split-K partials sum to the whole layer.
-//                 One k-split writes y directly; otherwise the last CTA of a
-//                 row block sums the partials in k order (deterministic).
+// The layer is cut into work units of 16 rows x one 256-column slab (128
+// bytes of nibbles per row).  Units are numbered slab-major and split into
+// one contiguous, equal share per CTA (one CTA per SM), so every SM streams
+// the same number of weight bytes.
+//
+// dec_main (programmatic dependent launch):
+//   before the dependency wait - reads only the packed weights: TMA brings
+//     every unit's q4 box (16 x 128 B, 128B swizzle) and s4 box into shared
+//     memory; a two-round parallel search of sal_idx finds each slab's
+//     salient entries, whose INT8 columns then follow by TMA in 16-entry
+//     chunks; s8 is staged.
+//   after the wait - the CTA rotates x for its (at most kDecMaxSlabs) slabs
+//     itself (16-thread Kronecker FWHT, fp32), stores it as FP16 in the
+//     GEMV's k-order, scatters the salient entries, and forms per-group
+//     bias terms.  Warps then take units round-robin: nibbles become FP16
+//     1024+u (even columns) or 1024+16u (odd columns, whose activations are
+//     stored pre-divided by 16) with one LOP3 each; the MMA chain of a
+//     64-column group starts from minus the group's bias term, so its sum is
+//     the exact-code dot product; acc += s4 * group sum.  The salient chunks
+//     run the same way (1152 + q) and are scaled by s8.  Each unit writes its
+//     16 x T partial for its slab; the CTA that holds a slab's first unit
+//     also writes that slab's share of t = V x_rot.
+// dec_tail: y = sum over slabs of the partials (slab order, deterministic)
+//   + U t + bias, in FP32, optionally rounded to BF16.
 #include "common.cuh"
 #include "fwht_group.cuh"
 #include "kernels.h"
 
-#include <stdlib.h>
+#include <algorithm>
+#include <mutex>
+#include <vector>
 
 namespace dvssq {
 
-constexpr int kDecBM = 64;
-constexpr int kDecRound = 1024;          // columns of one round (8 warps x 128)
-constexpr int kDecThreads = 256;
-constexpr int kDecQ4Box = 64 * 128;      // bytes of one q4 box (64 rows x 256 cols)
-constexpr int kDecQ8Box = 64 * 64;       // bytes of one q8 box (64 rows x 64 entries)
-constexpr int kDecMaxNR = 4;
+constexpr int kSlab = 256;                   // rotated columns per slab
+constexpr int kUnitRows = 16;                // rows per work unit
+constexpr int kDecWarps = 16;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecMaxUnits = 48;             // units per CTA staged at once
+constexpr int kDecMaxSlabs = 4;              // distinct slabs per CTA
+constexpr int kQ4Unit = kUnitRows * 128;     // one q4 box: 16 rows x 128 B
+constexpr int kS4Unit = kUnitRows * 16;      // one s4 box: 16 rows x 8 scales
+constexpr int kQ8Chunk = kUnitRows * 16;     // one q8 box: 16 rows x 16 entries
+constexpr int kXRow = kSlab + 8;             // FP16 per token row of x_rot (padded)
+constexpr int kXsRow = 17 * 16 + 8;          // FP16 per token row of the salient x
+constexpr int kSamples = 512;                // sal_idx samples of the search
+constexpr int kTailThreads = 256;
+constexpr int kSmemLimit = 232448;           // opt-in shared memory per CTA (227 KB)
+
+// Shared-memory layout of dec_main: byte offsets from the 1024-aligned base.
+struct DecLayout {
+  int q4, s4, q8, xq, xs, corr, c8, s8, colpos, samp, scr, meta, bars, total;
+};
 
 struct DecodeParams {
-  int M, K, T, n_sal, rank, block, nkb, NR, BK, KT, RB, SE, nq8box;
-  int s4_tma, u_tma;          // 1 when the scale / U tables come by TMA
+  int M, K, T, n_sal, rank, block;
+  int nslab, ntile, units, grid, upc_max, ns_max, ntok, nscr;
+  int q8_budget, s4_tma;
   float c;
   const uint16_t *s4;
   const int32_t *sal_idx;
+  const int8_t *q8;
   const uint16_t *s8;
   const uint16_t *U;
   const uint16_t *V;
@@ -48,631 +71,755 @@ struct DecodeParams {
   const uint16_t *bias;
   void *y;
   int y_bf16;
-  __half *xr16;
-  __half *xs16;
-  float *tp;
-  float *part;
-  unsigned int *counters;
+  float *part;    // [slice][T][M]
+  float *tpart;   // [nslab][rank][T]
+  // partial slices summed by dec_tail: all nslab slices (slab-major
+  // kernel), or, per 16-row tile, the CTAs of a tile-major grid of row_grid
+  // CTAs over row_units units of row_ut units per tile
+  int tail_mode, row_grid, row_units, row_ut;
+  DecLayout L;
 };
 
-// Position i of each 16-column segment of xr16 holds column perm16(i): the
-// order in which nibble pairs come out of the dequantiser (see dequant_q4),
+// CTA of a grid of G CTAs over U units (CTA c holds [c U / G, (c + 1) U / G))
+// that holds unit u.
+__host__ __device__ inline int cta_of_unit(long long u, int G, long long U) {
+  return (int)(((u + 1) * G - 1) / U);
+}
+
+// Position i of each 16-column segment of the FP16 x_rot holds column
+// perm16(i): the order in which nibble pairs come out of dequant_q4_biased,
 // i.e. {0,4,1,5, 2,6,3,7, 8,12,9,13, 10,14,11,15}.
 __host__ __device__ constexpr int perm16(int i) {
   return (i & 8) | ((i & 1) << 2) | ((i >> 1) & 3);
 }
-
-// ------------------------------------------------------------- prologue ---
-// Dynamic shared memory: V block [rank][B + 8] FP16 (converted from BF16).
-template <int B>
-__global__ void __launch_bounds__(B) dec_prologue_kernel(DecodeParams p) {
-  pdl_launch_dependents();
-  constexpr int P = B / 16;
-  __shared__ float scratch[16][GroupScratch<B>::kElems];
-  __shared__ float xr[16][B + 1];
-  __shared__ __align__(16) __half xh[16][B + 8];
-  __shared__ int s_cnt[2];
-  extern __shared__ __align__(16) uint8_t vs_raw[];
-  __half(*vh)[B + 8] = reinterpret_cast<__half(*)[B + 8]>(vs_raw);
-
-  const int kb = blockIdx.x, tid = threadIdx.x;
-  const int tok = tid / P, t = tid % P;
-  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
-  const bool live = tok < p.T;
-  if (tid < 2) s_cnt[tid] = 0;
-
-  // issue every global load first: x, V, sal_idx
-  uint16_t xin[16];
-#pragma unroll
-  for (int a = 0; a < 16; ++a)
-    xin[a] = live ? p.x[(size_t)tok * p.K + (size_t)kb * B + P * a + t] : (uint16_t)0;
-  constexpr int VPT = 64 * B / 8 / B;            // uint4 per thread for rank <= 64
-  uint4 vreg[VPT];
-#pragma unroll
-  for (int u = 0; u < VPT; ++u) {
-    const int i = tid + u * B;
-    const int rr = i / (B / 8), cc = i % (B / 8);
-    vreg[u] = rr < p.rank ? *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K +
-                                                             (size_t)kb * B + cc * 8)
-                          : make_uint4(0, 0, 0, 0);
-  }
-  int lo = 0, hi = 0;
-  for (int e = tid; e < p.n_sal; e += B) {
-    const int s = p.sal_idx[e];
-    lo += s < kb * B;
-    hi += s < (kb + 1) * B;
-  }
-  if (kb == 0)
-    for (int i = tid; i < p.RB; i += B) p.counters[i] = 0u;
-
-  float v[16];
-#pragma unroll
-  for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f32(xin[a]);
-  // whole warps whose tokens are all beyond T skip the transform
-  const bool warp_live = (tid & ~31) / P < p.T;
-  if (warp_live) {
-    fwht_group<B>(v, scratch[tok], t);
-    uint32_t hn[8];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      v[j] *= p.c;
-      xr[tok][16 * t + j] = v[j];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      hn[i] = pack_half2(__float2half_rn(v[2 * i]), __float2half_rn(v[2 * i + 1]));
-    *reinterpret_cast<uint4 *>(&xh[tok][16 * t]) = make_uint4(hn[0], hn[1], hn[2], hn[3]);
-    *reinterpret_cast<uint4 *>(&xh[tok][16 * t + 8]) = make_uint4(hn[4], hn[5], hn[6], hn[7]);
-    if (live) {
-      uint32_t h[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        h[i] = pack_half2(__float2half_rn(v[perm16(2 * i)]), __float2half_rn(v[perm16(2 * i + 1)]));
-      uint4 *dst = reinterpret_cast<uint4 *>(p.xr16 + (size_t)tok * p.K + (size_t)kb * B + 16 * t);
-      dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-      dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-    }
-  } else {
-    *reinterpret_cast<uint4 *>(&xh[tok][16 * t]) = make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4 *>(&xh[tok][16 * t + 8]) = make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int u = 0; u < VPT; ++u) {
-    const int i = tid + u * B;
-    const int rr = i / (B / 8), cc = i % (B / 8);
-    if (rr < p.rank) {
-      const uint32_t w[4] = {vreg[u].x, vreg[u].y, vreg[u].z, vreg[u].w};
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        o[q] = pack_half2(__float2half_rn(bf16_bits_to_f32(w[q] & 0xFFFFu)),
-                          __float2half_rn(bf16_bits_to_f32(w[q] >> 16)));
-      *reinterpret_cast<uint4 *>(&vh[rr][cc * 8]) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-  __syncthreads();
-  if (lo) atomicAdd(&s_cnt[0], lo);
-  if (hi) atomicAdd(&s_cnt[1], hi);
-  // this block's partial of t = V xr (tokens x ranks) on mma.sync, one n-tile
-  // of 8 ranks per warp
-  for (int nt = warp; nt < (p.rank + 7) / 8; nt += B / 32) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int n = 8 * nt + g;
-#pragma unroll 4
-    for (int k0 = 0; k0 < B; k0 += 16) {
-      uint32_t a[4];
-      a[0] = *reinterpret_cast<const uint32_t *>(&xh[g][k0 + 2 * tig]);
-      a[1] = *reinterpret_cast<const uint32_t *>(&xh[g + 8][k0 + 2 * tig]);
-      a[2] = *reinterpret_cast<const uint32_t *>(&xh[g][k0 + 2 * tig + 8]);
-      a[3] = *reinterpret_cast<const uint32_t *>(&xh[g + 8][k0 + 2 * tig + 8]);
-      const uint32_t b0 = n < p.rank ? *reinterpret_cast<const uint32_t *>(&vh[n][k0 + 2 * tig]) : 0u;
-      const uint32_t b1 = n < p.rank ? *reinterpret_cast<const uint32_t *>(&vh[n][k0 + 2 * tig + 8]) : 0u;
-      mma_16816(acc, a, b0, b1, acc);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int q = g + 8 * (i >> 1), rr = 8 * nt + 2 * tig + (i & 1);
-      if (q < p.T && rr < p.rank) p.tp[((size_t)kb * p.rank + rr) * p.T + q] = acc[i];
-    }
-  }
-  __syncthreads();
-  // salient entries whose rotated column falls in this block
-  const int e_lo = s_cnt[0], e_hi = s_cnt[1];
-  for (int e = e_lo + tid; e < e_hi; e += B) {
-    const int col = p.sal_idx[e] - kb * B;
-    if (col < 0 || col >= B) continue;   // sal_idx must be sorted; ignore otherwise
-    for (int q = 0; q < p.T; ++q)
-      p.xs16[(size_t)q * p.n_sal + e] = __float2half_rn(xr[q][col]);
-  }
+__host__ __device__ constexpr int inv_perm16(int j) {
+  return (j & 8) | ((j & 3) << 1) | ((j >> 2) & 1);
 }
 
-// ----------------------------------------------------------------- main ---
-// 8 nibbles of a 32-bit word (biased by XOR 8, i.e. u = q + 8) -> four FP16
-// pairs holding the exact codes q: (n0,n4), (n1,n5), (n2,n6), (n3,n7).
-__device__ __forceinline__ void dequant_q4(uint32_t w, uint32_t out[4]) {
-  const uint32_t u = w ^ 0x88888888u;
-  const uint32_t magic = 0x64006400u;               // FP16 1024 in both halves
-  const __half2 sub_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
-  const __half2 mul_hi = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
-  const __half2 sub_hi = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));  // -72
-  uint32_t l0 = (u & 0x000F000Fu) | magic;
-  uint32_t h0 = (u & 0x00F000F0u) | magic;
-  uint32_t l1 = ((u >> 8) & 0x000F000Fu) | magic;
-  uint32_t h1 = ((u >> 8) & 0x00F000F0u) | magic;
-  __half2 r0 = __hsub2(*reinterpret_cast<__half2 *>(&l0), sub_lo);
-  __half2 r1 = __hfma2(*reinterpret_cast<__half2 *>(&h0), mul_hi, sub_hi);
-  __half2 r2 = __hsub2(*reinterpret_cast<__half2 *>(&l1), sub_lo);
-  __half2 r3 = __hfma2(*reinterpret_cast<__half2 *>(&h1), mul_hi, sub_hi);
-  out[0] = *reinterpret_cast<uint32_t *>(&r0);
-  out[1] = *reinterpret_cast<uint32_t *>(&r1);
-  out[2] = *reinterpret_cast<uint32_t *>(&r2);
-  out[3] = *reinterpret_cast<uint32_t *>(&r3);
+// Per bit: b ? (c ? ~a : a) : c.  With b a nibble mask and c holding the
+// bias bit (inside the mask) and the FP16 exponent pattern (outside it), one
+// instruction flips the sign bit of each selected nibble and splices it into
+// the mantissa of an FP16 1024.
+__device__ __forceinline__ uint32_t lop3_splice(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// 4 int8 codes -> two FP16 pairs (e0,e1), (e2,e3), exact.
-__device__ __forceinline__ void dequant_q8(uint32_t w, uint32_t &p01, uint32_t &p23) {
-  const uint32_t u = w ^ 0x80808080u;               // q + 128 in [0, 255]
-  uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
-  uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
-  const __half2 sub = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152
-  __half2 ra = __hsub2(*reinterpret_cast<__half2 *>(&a), sub);
-  __half2 rb = __hsub2(*reinterpret_cast<__half2 *>(&b), sub);
-  p01 = *reinterpret_cast<uint32_t *>(&ra);
-  p23 = *reinterpret_cast<uint32_t *>(&rb);
+// 8 two's-complement nibbles (columns c0..c7) -> FP16 pairs (c0,c4), (c1,c5),
+// (c2,c6), (c3,c7) holding 1024 + u for even columns and 1024 + 16u for odd
+// ones, u = q + 8 in [0, 15].  Exact.
+__device__ __forceinline__ void dequant_q4_biased(uint32_t w, uint32_t out[4]) {
+  const uint32_t w8 = w >> 8;
+  out[0] = lop3_splice(w, 0x000F000Fu, 0x64086408u);
+  out[1] = lop3_splice(w, 0x00F000F0u, 0x64806480u);
+  out[2] = lop3_splice(w8, 0x000F000Fu, 0x64086408u);
+  out[3] = lop3_splice(w8, 0x00F000F0u, 0x64806480u);
 }
 
-// B fragments (activations, FP16, GEMV k-order) of one 128-column slice for
-// n-tiles 0..NT-1: [group][ntile][8 registers].
-template <int NT>
-__device__ __forceinline__ void load_x_frags(const DecodeParams &p, int kw, int g, int tig,
-                                             uint32_t bq[2][NT][8]) {
-#pragma unroll
-  for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int tok = g + 8 * nt;
-      const int kc = kw + 64 * gi + 16 * tig;
-      if (tok < p.T && kc < p.K) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.xr16 + (size_t)tok * p.K + kc);
-        const uint4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
-        bq[gi][nt][0] = x0.x; bq[gi][nt][1] = x0.y; bq[gi][nt][2] = x0.z; bq[gi][nt][3] = x0.w;
-        bq[gi][nt][4] = x1.x; bq[gi][nt][5] = x1.y; bq[gi][nt][6] = x1.z; bq[gi][nt][7] = x1.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) bq[gi][nt][i] = 0u;
-      }
-    }
+// 4 int8 codes -> FP16 pairs (e0,e1), (e2,e3) holding 1152 + q.  Exact.
+__device__ __forceinline__ void dequant_q8_biased(uint32_t w, uint32_t &p01, uint32_t &p23) {
+  const uint32_t u = w ^ 0x80808080u;
+  p01 = __byte_perm(u, 0x64646464u, 0x4140);
+  p23 = __byte_perm(u, 0x64646464u, 0x4342);
 }
 
-// One 128-column slice (two 64-column groups) of the INT4 tier for the four
-// 16-row tiles: acc += s4 * (codes x activations).
-template <int NT>
-__device__ __forceinline__ void int4_slice(const uint8_t *bx, const uint16_t *ss4, int GPC,
-                                           int sgrp0, int half, int g, int tig,
-                                           const uint32_t bq[2][NT][8], float acc[4][NT][4]) {
-  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int gi = 0; gi < 2; ++gi) {
-    const int chunk = 4 * half + 2 * gi + (tig >> 1);
-    const int sgrp = sgrp0 + gi;
-#pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-      const int rlo = 16 * rt + g;
-      const uint32_t off = (uint32_t)(((chunk ^ (rlo & 7)) << 4) + 8 * (tig & 1));
-      const uint2 wl = *reinterpret_cast<const uint2 *>(bx + rlo * 128 + off);
-      const uint2 wh = *reinterpret_cast<const uint2 *>(bx + (rlo + 8) * 128 + off);
-      uint32_t fl[8], fh[8];
-      dequant_q4(wl.x, fl);
-      dequant_q4(wl.y, fl + 4);
-      dequant_q4(wh.x, fh);
-      dequant_q4(wh.y, fh + 4);
-      const float slo = bf16_bits_to_f32(ss4[rlo * GPC + sgrp]);
-      const float shi = bf16_bits_to_f32(ss4[(rlo + 8) * GPC + sgrp]);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float d[4];
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint32_t a[4] = {fl[2 * s], fh[2 * s], fl[2 * s + 1], fh[2 * s + 1]};
-          mma_16816(d, a, bq[gi][nt][2 * s], bq[gi][nt][2 * s + 1], s == 0 ? zero4 : d);
-        }
-        acc[rt][nt][0] = fmaf(slo, d[0], acc[rt][nt][0]);
-        acc[rt][nt][1] = fmaf(slo, d[1], acc[rt][nt][1]);
-        acc[rt][nt][2] = fmaf(shi, d[2], acc[rt][nt][2]);
-        acc[rt][nt][3] = fmaf(shi, d[3], acc[rt][nt][3]);
-      }
-    }
-  }
-}
-
-template <int NT>
-__global__ void __launch_bounds__(kDecThreads, NT == 1 ? 3 : 2) dec_main_kernel(
-    const __grid_constant__ CUtensorMap mq4, const __grid_constant__ CUtensorMap mq8,
-    const __grid_constant__ CUtensorMap ms4, const __grid_constant__ CUtensorMap mu,
-    DecodeParams p) {
+// --------------------------------------------------------------- dec_main --
+template <int B, int NT>
+__global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
+    const __grid_constant__ CUtensorMap mq4, const __grid_constant__ CUtensorMap ms4,
+    const __grid_constant__ CUtensorMap mq8, DecodeParams p) {
+  constexpr int NTOK = 8 * NT;
+  constexpr int P = B / 16;                 // threads per Hadamard block-row
+  constexpr int NBLK = kSlab / B;           // Hadamard blocks per slab
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  const int nbox = 4 * p.NR;
-  const int GPC = 16 * p.NR;
-  uint8_t *sq4 = base;                                                  // nbox boxes
-  uint8_t *sq8 = base + nbox * kDecQ4Box;                               // nq8box boxes
-  uint16_t *ss4 = reinterpret_cast<uint16_t *>(sq8 + p.nq8box * kDecQ8Box);   // [64][GPC]
-  uint16_t *su = ss4 + kDecBM * GPC;                                    // [64][rank]
-  float *tps = reinterpret_cast<float *>(su + kDecBM * 64);             // [rank][T]
-  float *s8s = tps + 64 * 16;                                           // [64]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(s8s + kDecBM);          // nbox + 2
-  __shared__ int s_last;
+  uint8_t *q4s = base + p.L.q4;
+  uint16_t *s4s = reinterpret_cast<uint16_t *>(base + p.L.s4);
+  uint8_t *q8s = base + p.L.q8;
+  __half *xq = reinterpret_cast<__half *>(base + p.L.xq);     // [ns][NTOK][kXRow]
+  __half *xs = reinterpret_cast<__half *>(base + p.L.xs);     // [ns][NTOK][kXsRow]
+  float *corr = reinterpret_cast<float *>(base + p.L.corr);   // [ns][4][NTOK]
+  float *c8 = reinterpret_cast<float *>(base + p.L.c8);       // [ns][NTOK]
+  float *s8s = reinterpret_cast<float *>(base + p.L.s8);      // [upc][16]
+  int16_t *colpos = reinterpret_cast<int16_t *>(base + p.L.colpos);   // [ns][256]
+  int *samp = reinterpret_cast<int *>(base + p.L.samp);       // [kSamples]
+  float *scr = reinterpret_cast<float *>(base + p.L.scr);
+  int *meta = reinterpret_cast<int *>(base + p.L.meta);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + p.L.bars);
+  int *lo = meta;                                   // [kDecMaxSlabs + 1]
+  int *lo16 = meta + 8;                             // [kDecMaxSlabs]
+  int *nch = meta + 16;                             // [kDecMaxSlabs]
+  int *q8off = meta + 24;                           // [kDecMaxUnits]
+  int *flags = meta + 24 + kDecMaxUnits;            // [0]: q8 staged
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
-  const int rb = blockIdx.x, kt = blockIdx.y;
-  const int m0 = rb * kDecBM, k0 = kt * p.BK, e0 = kt * p.SE;
-  const int nsal_cta = max(0, min(p.SE, p.n_sal - e0));
-  const bool s4_tma = p.s4_tma != 0, u_tma = p.u_tma != 0 && p.rank > 0;
+  const int u0 = (int)(((long long)blockIdx.x * p.units) / p.grid);
+  const int u1 = (int)(((long long)(blockIdx.x + 1) * p.units) / p.grid);
+  const int nu = u1 - u0;
+  if (nu <= 0) {
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
+  const int s_first = u0 / p.ntile;
+  const int ns = (u1 - 1) / p.ntile - s_first + 1;
+  if (ns > p.ns_max || nu > p.upc_max) {           // the host plan rules this out
+    if (tid == 0) set_error(kErrBadShape);
+    pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
 
-  if (tid == 0) {
-    for (int i = 0; i < nbox + 2; ++i) mbar_init(&bars[i], 1);
+  // ------------- before the dependency wait: packed weights only -------------
+  // warp 0: one lane per unit initialises its barrier and issues its boxes
+  if (warp == 0) {
+    for (int k = lane; k < nu; k += 32) mbar_init(&bars[k], 2);
     fence_mbarrier_init();
+    __syncwarp();
+    if (lane == 0) prefetch_tensormap(&mq4);
+    const uint32_t bytes = kQ4Unit + (p.s4_tma ? kS4Unit : 0);
+    for (int k = lane; k < nu; k += 32) {
+      const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
+      mbar_arrive_expect_tx(&bars[k], bytes);
+      tma_load_2d(q4s + k * kQ4Unit, &mq4, s * 128, tile * kUnitRows, &bars[k]);
+      if (p.s4_tma)
+        tma_load_2d(s4s + k * (kS4Unit / 2), &ms4, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
+    }
+  }
+  const int KG = p.K / 64;
+  const int step = (p.n_sal + kSamples - 1) / kSamples;
+  if (p.n_sal > 0)
+    for (int i = tid; i < kSamples; i += kDecThreads)
+      samp[i] = __ldg(p.sal_idx + min(i * step, p.n_sal - 1));
+  for (int i = tid; i < nu * kUnitRows; i += kDecThreads) {
+    const int k = i >> 4, r = i & 15;
+    const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
+    const int m = tile * kUnitRows + r;
+    s8s[i] = (m < p.M && p.n_sal > 0) ? bf16_bits_to_f32(p.s8[m]) : 0.0f;
+  }
+  if (!p.s4_tma) {
+    // scale rows whose stride a tensor map cannot carry: plain loads
+    for (int i = tid; i < nu * kUnitRows * 8; i += kDecThreads) {
+      const int k = i >> 7, r = (i >> 3) & 15, j = i & 7;
+      const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
+      const int m = tile * kUnitRows + r, gcol = 8 * (s >> 1) + j;
+      s4s[i] = (m < p.M && gcol < KG) ? p.s4[(size_t)m * KG + gcol] : (uint16_t)0;
+    }
+  }
+  for (int i = tid; i < ns * kSlab; i += kDecThreads) colpos[i] = -1;
+  for (int i = tid; i < ns * NTOK * kXsRow / 2; i += kDecThreads)
+    reinterpret_cast<uint32_t *>(xs)[i] = 0u;
+  // rows of V for the slabs whose first unit this CTA holds: warm L2
+  if (p.rank > 0)
+    for (int si = 0; si < ns; ++si) {
+      const int s = s_first + si;
+      if (s * p.ntile < u0) continue;
+      for (int i = tid; i < p.rank * 4; i += kDecThreads) {
+        const int rr = i >> 2, col = kSlab * s + 64 * (i & 3);
+        if (col < p.K)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(p.V + (size_t)rr * p.K + col));
+      }
+    }
+  __syncthreads();
+
+  // salient entries of each slab: lo[b] = #{e : sal_idx[e] < 256 (s_first + b)}
+  if (warp <= ns) {
+    int l = 0;
+    if (p.n_sal > 0) {
+      const int v = kSlab * (s_first + warp);
+      int j = 0;
+      for (int i0 = 0; i0 < kSamples; i0 += 32) {
+        const int i = i0 + lane;
+        j += __popc(__ballot_sync(0xffffffffu, i * step < p.n_sal && samp[i] < v));
+      }
+      // entries below v: all of [0, (j-1) step] plus some of ((j-1) step, j step)
+      const int lb = j > 0 ? (j - 1) * step + 1 : 0;
+      const int le = min(j * step, p.n_sal);
+      int cnt = 0;
+      for (int e = lb + lane; e < le; e += 32) cnt += __ldg(p.sal_idx + e) < v;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      l = lb + cnt;
+    }
+    if (lane == 0) lo[warp] = l;
   }
   __syncthreads();
-  if (tid == 0) {
-    // small per-CTA tables first, then the salient slice, then the INT4 tile
-    uint32_t small = (s4_tma ? kDecBM * GPC * 2 : 0) + (u_tma ? kDecBM * p.rank * 2 : 0);
-    if (small) {
-      mbar_arrive_expect_tx(&bars[nbox + 1], small);
-      if (s4_tma) tma_load_2d(ss4, &ms4, k0 / 64, m0, &bars[nbox + 1]);
-      if (u_tma) tma_load_2d(su, &mu, 0, m0, &bars[nbox + 1]);
+  if (tid < ns) {
+    const int a = lo[tid], b = lo[tid + 1];
+    lo16[tid] = a & ~15;
+    nch[tid] = b > a ? (b - (a & ~15) + 15) >> 4 : 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // q8 staging offsets: exclusive scan of the units' chunk bytes
+    int run = 0;
+    for (int k0 = 0; k0 < nu; k0 += 32) {
+      const int k = k0 + lane;
+      const int b = k < nu ? nch[(u0 + k) / p.ntile - s_first] * kQ8Chunk : 0;
+      int inc = b;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      if (k < nu) q8off[k] = run + inc - b;
+      run += __shfl_sync(0xffffffffu, inc, 31);
     }
-    if (nsal_cta > 0) {
-      const int nb = (nsal_cta + 63) / 64;
-      mbar_arrive_expect_tx(&bars[nbox], nb * kDecQ8Box);
-      for (int i = 0; i < nb; ++i)
-        tma_load_2d(sq8 + i * kDecQ8Box, &mq8, e0 + 64 * i, m0, &bars[nbox]);
+    const int staged = run <= p.q8_budget;
+    if (lane == 0) flags[0] = staged;
+    for (int k = lane; k < nu; k += 32) {
+      const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
+      const int n = staged ? nch[si] : 0;
+      mbar_arrive_expect_tx(&bars[k], (uint32_t)(n * kQ8Chunk));
+      for (int c = 0; c < n; ++c)
+        tma_load_2d(q8s + q8off[k] + c * kQ8Chunk, &mq8, lo16[si] + 16 * c, tile * kUnitRows,
+                    &bars[k]);
     }
-    for (int box = 0; box < nbox; ++box) {
-      if (k0 + 256 * box < p.K) {
-        mbar_arrive_expect_tx(&bars[box], kDecQ4Box);
-        tma_load_2d(sq4 + box * kDecQ4Box, &mq4, (k0 + 256 * box) / 2, m0, &bars[box]);
+  } else {
+    // column -> position of each salient entry in its slab's chunk range
+    for (int si = 0; si < ns; ++si) {
+      const int a = lo[si], b = lo[si + 1], s = s_first + si;
+      for (int e = a + tid - 32; e < b; e += kDecThreads - 32) {
+        const int col = __ldg(p.sal_idx + e) - kSlab * s;
+        if (col >= 0 && col < kSlab) colpos[si * kSlab + col] = (int16_t)(e - (a & ~15));
       }
     }
   }
-  // tables the tensor maps cannot carry (unaligned row strides), and s8
-  const int KG = p.K / 64;
-  for (int r = warp; r < kDecBM; r += 8) {
-    const int row = m0 + r;
-    if (!s4_tma)
-      for (int gi = lane; gi < GPC; gi += 32) {
-        const int gcol = k0 / 64 + gi;
-        ss4[r * GPC + gi] = (row < p.M && gcol < KG) ? p.s4[(size_t)row * KG + gcol] : (uint16_t)0;
-      }
-    if (!u_tma)
-      for (int rr = lane; rr < p.rank; rr += 32)
-        su[r * p.rank + rr] = row < p.M ? p.U[(size_t)row * p.rank + rr] : (uint16_t)0;
-    if (lane == 0) s8s[r] = (row < p.M && p.n_sal > 0) ? bf16_bits_to_f32(p.s8[row]) : 0.0f;
+  __syncthreads();
+
+  // ------------------------- after the wait: activations -------------------------
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // V rows of the first owned slab, into registers (consumed after the FWHT)
+  int own_si = -1;
+  for (int si = 0; si < ns; ++si)
+    if ((s_first + si) * p.ntile >= u0) { own_si = si; break; }
+  uint4 vreg[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    vreg[i] = make_uint4(0u, 0u, 0u, 0u);
+    const int rr = warp + kDecWarps * i, col = kSlab * (s_first + own_si) + 8 * lane;
+    if (own_si >= 0 && rr < p.rank && col < p.K)
+      vreg[i] = *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + col);
   }
 
-  pdl_wait();   // xr16, xs16, tp and the counters come from the prologue
-
-  // every remaining global load of the warp, issued together
-  const int kw0 = k0 + 128 * warp;
-  uint32_t bq[2][NT][8];
-  load_x_frags<NT>(p, kw0, g, tig, bq);
-  const int nsteps = nsal_cta / 16;
-  uint32_t sb01[2][NT], sb23[2][NT];     // up to two salient steps per warp
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int st = warp + 8 * j;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int tok = g + 8 * nt;
-      if (st < nsteps && tok < p.T) {
-        const uint2 xv = __ldcg(reinterpret_cast<const uint2 *>(
-            p.xs16 + (size_t)tok * p.n_sal + e0 + 16 * st + 4 * tig));
-        sb01[j][nt] = xv.x;
-        sb23[j][nt] = xv.y;
-      } else {
-        sb01[j][nt] = 0u;
-        sb23[j][nt] = 0u;
-      }
-    }
-  }
+  // rotate x for the CTA's slabs: block-row br = (si * NBLK + blk) * T + tok
   {
-    // the CTA's slice of t: sum of the prologue partials of its Hadamard blocks
-    const int kb0 = k0 / p.block, kb1 = min(p.nkb, (k0 + p.BK) / p.block);
-    const int nkbc = kb1 - kb0;
-    for (int i = tid; i < p.rank * p.T; i += kDecThreads) {
-      float pv[16];
+    const int nbr = ns * NBLK * p.T;
+    const int grp = tid / P, t = tid % P;
+    const int wgrp = (warp * 32) / P;            // first group of this warp
+    for (int br0 = 0; br0 < nbr; br0 += p.nscr) {
+      if (wgrp >= p.nscr || br0 + wgrp >= nbr) continue;   // whole warp idle
+      const int br = br0 + grp;
+      const bool live = br < nbr;                  // grp < nscr: nscr is whole warps
+      const int tok = live ? br % p.T : 0;
+      const int blk = live ? (br / p.T) % NBLK : 0;
+      const int si = live ? br / (p.T * NBLK) : 0;
+      const int col0 = kSlab * (s_first + si) + B * blk;
+      float v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        pv[u] = u < nkbc ? __ldcg(&p.tp[(size_t)(kb0 + u) * p.rank * p.T + i]) : 0.0f;
-      float sum = 0.0f;
+      for (int a = 0; a < 16; ++a) {
+        const int col = col0 + P * a + t;
+        v[a] = (live && col < p.K) ? bf16_bits_to_f32(p.x[(size_t)tok * p.K + col]) : 0.0f;
+      }
+      fwht_group<B>(v, scr + grp * GroupScratch<B>::kElems, t);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) sum += pv[u];
-      for (int u = 16; u < nkbc; ++u) sum += __ldcg(&p.tp[(size_t)(kb0 + u) * p.rank * p.T + i]);
-      tps[i] = sum;
+      for (int j = 0; j < 16; ++j) v[j] *= p.c;
+      const int cs = B * blk + 16 * t;            // slab column of v[0]
+      uint32_t h[8];
+      float se = 0.0f, so = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j0 = perm16(2 * i), j1 = perm16(2 * i + 1);
+        const __half a0 = __float2half_rn((j0 & 1) ? v[j0] * 0.0625f : v[j0]);
+        const __half a1 = __float2half_rn((j1 & 1) ? v[j1] * 0.0625f : v[j1]);
+        h[i] = pack_half2(a0, a1);
+        if (j0 & 1) so += __half2float(a0); else se += __half2float(a0);
+        if (j1 & 1) so += __half2float(a1); else se += __half2float(a1);
+      }
+      // bias term of the 64-column group: its four threads are adjacent lanes
+      float cp = 1032.0f * se + 1152.0f * so;
+      cp += __shfl_xor_sync(0xffffffffu, cp, 1);
+      cp += __shfl_xor_sync(0xffffffffu, cp, 2);
+      if (live) {
+        uint4 *dst = reinterpret_cast<uint4 *>(xq + (size_t)(si * NTOK + tok) * kXRow + cs);
+        dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+        if ((t & 3) == 0) corr[(si * 4 + cs / 64) * NTOK + tok] = cp;
+        const int16_t *cpos = colpos + si * kSlab + cs;
+        __half *xrow = xs + (size_t)(si * NTOK + tok) * kXsRow;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int pos = cpos[j];
+          if (pos >= 0) xrow[pos] = __float2half_rn(v[j]);
+        }
+      }
     }
   }
-  __syncthreads();   // s8s, fallback tables, tps complete
+  __syncthreads();
 
-  float acc[4][NT][4];
+  // salient bias terms: c8[si][tok] = 1152 * sum of the slab's salient x
+  for (int q = warp; q < ns * p.T; q += kDecWarps) {
+    const int si = q / p.T, tok = q % p.T;
+    const __half *xrow = xs + (size_t)(si * NTOK + tok) * kXsRow;
+    float sum = 0.0f;
+    for (int i = lane; i < 16 * nch[si]; i += 32) sum += __half2float(xrow[i]);
 #pragma unroll
-  for (int rt = 0; rt < 4; ++rt)
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) c8[si * NTOK + tok] = 1152.0f * sum;
+  }
+
+  // t share of each owned slab: tpart[s][rr][tok] = sum_j V[rr][j] x_rot[j]
+  if (p.rank > 0)
+    for (int si = own_si; si >= 0 && si < ns; ++si) {
+      const int s = s_first + si;
+      if (s * p.ntile < u0) continue;
+      if (si != own_si) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          vreg[i] = make_uint4(0u, 0u, 0u, 0u);
+          const int rr = warp + kDecWarps * i, col = kSlab * s + 8 * lane;
+          if (rr < p.rank && col < p.K)
+            vreg[i] = *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + col);
+        }
+      }
+      for (int tok = 0; tok < p.T; ++tok) {
+        float xv[8];
+        const __half *xrow = xq + (size_t)(si * NTOK + tok) * kXRow;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int cn = 8 * lane + j;
+          const float hv = __half2float(xrow[(cn & ~15) + inv_perm16(cn & 15)]);
+          xv[j] = (cn & 1) ? hv * 16.0f : hv;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = warp + kDecWarps * i;
+          if (rr >= p.rank) break;
+          const uint32_t w[4] = {vreg[i].x, vreg[i].y, vreg[i].z, vreg[i].w};
+          float d = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            d = fmaf(bf16_bits_to_f32(w[q] & 0xFFFFu), xv[2 * q], d);
+            d = fmaf(bf16_bits_to_f32(w[q] >> 16), xv[2 * q + 1], d);
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+          if (lane == 0) p.tpart[((size_t)s * p.rank + rr) * p.T + tok] = d;
+        }
+      }
+    }
+  __syncthreads();
+
+  // ----------------------------------- units -----------------------------------
+  const bool staged = flags[0] != 0;
+  uint32_t bq[NT == 1 ? 4 : 1][8];
+  int cur = -1;
+  for (int k = warp; k < nu; k += kDecWarps) {
+    const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
+    if constexpr (NT == 1) {
+      if (si != cur) {
+        const __half *xrow = xq + (size_t)(si * NTOK + g) * kXRow + 16 * tig;
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          const uint4 x0 = *reinterpret_cast<const uint4 *>(xrow + 64 * gi);
+          const uint4 x1 = *reinterpret_cast<const uint4 *>(xrow + 64 * gi + 8);
+          bq[gi][0] = x0.x; bq[gi][1] = x0.y; bq[gi][2] = x0.z; bq[gi][3] = x0.w;
+          bq[gi][4] = x1.x; bq[gi][5] = x1.y; bq[gi][6] = x1.z; bq[gi][7] = x1.w;
+        }
+        cur = si;
+      }
+    }
+    if (!mbar_wait(&bars[k], 0)) break;
+    const uint8_t *bx = q4s + k * kQ4Unit;
+    const uint16_t *sb = s4s + k * (kS4Unit / 2) + 4 * (s & 1);
+    const uint2 sl = *reinterpret_cast<const uint2 *>(sb + g * 8);
+    const uint2 sh = *reinterpret_cast<const uint2 *>(sb + (g + 8) * 8);
+    const uint32_t slw[4] = {sl.x & 0xFFFFu, sl.x >> 16, sl.y & 0xFFFFu, sl.y >> 16};
+    const uint32_t shw[4] = {sh.x & 0xFFFFu, sh.x >> 16, sh.y & 0xFFFFu, sh.y >> 16};
+    float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[rt][nt][i] = 0.0f;
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
 
-  // ---- salient INT8 tier first, into acc, then scaled by s8 ----
-  if (warp < nsteps && mbar_wait(&bars[nbox], 0)) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int st = warp + 8 * j;
-      if (st >= nsteps) break;
-      const uint8_t *bx = sq8 + (st >> 2) * kDecQ8Box;
-      const int chunk = st & 3;
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        const int rlo = 16 * rt + g;
-        const uint32_t off = (uint32_t)(((chunk ^ ((rlo >> 1) & 3)) << 4) + 4 * tig);
-        const uint32_t wl = *reinterpret_cast<const uint32_t *>(bx + rlo * 64 + off);
-        const uint32_t wh = *reinterpret_cast<const uint32_t *>(bx + (rlo + 8) * 64 + off);
-        uint32_t l01, l23, h01, h23;
-        dequant_q8(wl, l01, l23);
-        dequant_q8(wh, h01, h23);
-        const uint32_t a[4] = {l01, h01, l23, h23};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[rt][nt], a, sb01[j][nt], sb23[j][nt], acc[rt][nt]);
-      }
-    }
-    for (int st = warp + 16; st < nsteps; st += 8) {     // rare: more than two steps
-      const uint8_t *bx = sq8 + (st >> 2) * kDecQ8Box;
-      const int chunk = st & 3;
-      uint32_t b01[NT], b23[NT];
+    for (int gi = 0; gi < 4; ++gi) {
+      const int chunk = 2 * gi + (tig >> 1);
+      const uint32_t off = (uint32_t)(((chunk ^ g) << 4) + 8 * (tig & 1));
+      const uint2 wl = *reinterpret_cast<const uint2 *>(bx + g * 128 + off);
+      const uint2 wh = *reinterpret_cast<const uint2 *>(bx + (g + 8) * 128 + off);
+      uint32_t fl[8], fh[8];
+      dequant_q4_biased(wl.x, fl);
+      dequant_q4_biased(wl.y, fl + 4);
+      dequant_q4_biased(wh.x, fh);
+      dequant_q4_biased(wh.y, fh + 4);
+      const float slo = bf16_bits_to_f32(slw[gi]), shi = bf16_bits_to_f32(shw[gi]);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int tok = g + 8 * nt;
-        b01[nt] = b23[nt] = 0u;
-        if (tok < p.T) {
-          const uint2 xv = __ldcg(reinterpret_cast<const uint2 *>(
-              p.xs16 + (size_t)tok * p.n_sal + e0 + 16 * st + 4 * tig));
-          b01[nt] = xv.x;
-          b23[nt] = xv.y;
+        uint32_t b[8];
+        if constexpr (NT == 1) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) b[i] = bq[gi][i];
+        } else {
+          const __half *xrow =
+              xq + (size_t)(si * NTOK + g + 8 * nt) * kXRow + 64 * gi + 16 * tig;
+          const uint4 x0 = *reinterpret_cast<const uint4 *>(xrow);
+          const uint4 x1 = *reinterpret_cast<const uint4 *>(xrow + 8);
+          b[0] = x0.x; b[1] = x0.y; b[2] = x0.z; b[3] = x0.w;
+          b[4] = x1.x; b[5] = x1.y; b[6] = x1.z; b[7] = x1.w;
+        }
+        const float2 cc =
+            *reinterpret_cast<const float2 *>(corr + (si * 4 + gi) * NTOK + 8 * nt + 2 * tig);
+        float d[4] = {-cc.x, -cc.y, -cc.x, -cc.y};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t a[4] = {fl[2 * q], fh[2 * q], fl[2 * q + 1], fh[2 * q + 1]};
+          mma_16816(d, a, b[2 * q], b[2 * q + 1], d);
+        }
+        acc[nt][0] = fmaf(slo, d[0], acc[nt][0]);
+        acc[nt][1] = fmaf(slo, d[1], acc[nt][1]);
+        acc[nt][2] = fmaf(shi, d[2], acc[nt][2]);
+        acc[nt][3] = fmaf(shi, d[3], acc[nt][3]);
+      }
+    }
+
+    // salient INT8 chunks of this slab
+    const int nc = nch[si];
+    if (nc > 0) {
+      float d8[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float2 cc = *reinterpret_cast<const float2 *>(c8 + si * NTOK + 8 * nt + 2 * tig);
+        d8[nt][0] = -cc.x; d8[nt][1] = -cc.y; d8[nt][2] = -cc.x; d8[nt][3] = -cc.y;
+      }
+      const int mlo = tile * kUnitRows + g;
+      for (int c = 0; c < nc; ++c) {
+        uint32_t wl = 0u, wh = 0u;
+        if (staged) {
+          const uint8_t *cb = q8s + q8off[k] + c * kQ8Chunk;
+          wl = *reinterpret_cast<const uint32_t *>(cb + g * 16 + 4 * tig);
+          wh = *reinterpret_cast<const uint32_t *>(cb + (g + 8) * 16 + 4 * tig);
+        } else {
+          const size_t e = (size_t)lo16[si] + 16 * c + 4 * tig;
+          if (mlo < p.M)
+            wl = __ldg(reinterpret_cast<const uint32_t *>(p.q8 + (size_t)mlo * p.n_sal + e));
+          if (mlo + 8 < p.M)
+            wh = __ldg(reinterpret_cast<const uint32_t *>(p.q8 + (size_t)(mlo + 8) * p.n_sal + e));
+        }
+        uint32_t l01, l23, h01, h23;
+        dequant_q8_biased(wl, l01, l23);
+        dequant_q8_biased(wh, h01, h23);
+        const uint32_t a[4] = {l01, h01, l23, h23};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 xv = *reinterpret_cast<const uint2 *>(
+              xs + (size_t)(si * NTOK + g + 8 * nt) * kXsRow + 16 * c + 4 * tig);
+          mma_16816(d8[nt], a, xv.x, xv.y, d8[nt]);
         }
       }
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        const int rlo = 16 * rt + g;
-        const uint32_t off = (uint32_t)(((chunk ^ ((rlo >> 1) & 3)) << 4) + 4 * tig);
-        const uint32_t wl = *reinterpret_cast<const uint32_t *>(bx + rlo * 64 + off);
-        const uint32_t wh = *reinterpret_cast<const uint32_t *>(bx + (rlo + 8) * 64 + off);
-        uint32_t l01, l23, h01, h23;
-        dequant_q8(wl, l01, l23);
-        dequant_q8(wh, h01, h23);
-        const uint32_t a[4] = {l01, h01, l23, h23};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[rt][nt], a, b01[nt], b23[nt], acc[rt][nt]);
-      }
-    }
-#pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
-      const float s8lo = s8s[16 * rt + g], s8hi = s8s[16 * rt + g + 8];
+      const float s8lo = s8s[k * 16 + g], s8hi = s8s[k * 16 + g + 8];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        acc[rt][nt][0] *= s8lo;
-        acc[rt][nt][1] *= s8lo;
-        acc[rt][nt][2] *= s8hi;
-        acc[rt][nt][3] *= s8hi;
+        acc[nt][0] = fmaf(s8lo, d8[nt][0], acc[nt][0]);
+        acc[nt][1] = fmaf(s8lo, d8[nt][1], acc[nt][1]);
+        acc[nt][2] = fmaf(s8hi, d8[nt][2], acc[nt][2]);
+        acc[nt][3] = fmaf(s8hi, d8[nt][3], acc[nt][3]);
+      }
+    }
+
+    // this unit's partial of slab s
+    const int m = tile * kUnitRows + g;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int tok = 8 * nt + 2 * tig;
+      float *dst = p.part + ((size_t)s * p.T + tok) * p.M;
+      if (tok < p.T) {
+        if (m < p.M) dst[m] = acc[nt][0];
+        if (m + 8 < p.M) dst[m + 8] = acc[nt][2];
+      }
+      if (tok + 1 < p.T) {
+        if (m < p.M) dst[p.M + m] = acc[nt][1];
+        if (m + 8 < p.M) dst[p.M + m + 8] = acc[nt][3];
       }
     }
   }
+}
 
-  // ---- INT4 tier, one round of 1024 columns at a time ----
-  const bool small_ok = !(s4_tma || u_tma) || mbar_wait(&bars[nbox + 1], 0);
-  for (int round = 0; round < p.NR && small_ok; ++round) {
-    const int kw = kw0 + kDecRound * round;
-    if (kw >= p.K) break;
-    if (round > 0) load_x_frags<NT>(p, kw, g, tig, bq);
-    const int box = 4 * round + (warp >> 1);
-    if (!mbar_wait(&bars[box], 0)) break;
-    int4_slice<NT>(sq4 + box * kDecQ4Box, ss4, GPC, 16 * round + 2 * warp, warp & 1, g, tig, bq,
-                   acc);
-  }
-
-  // ---- reduce the 8 warps' k slices in shared memory (reusing the q4 boxes) ----
-  __syncthreads();
-  float *red = reinterpret_cast<float *>(base);      // [8][64][16]
-#pragma unroll
-  for (int rt = 0; rt < 4; ++rt)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int rlo = 16 * rt + g, tok = 2 * tig + 8 * nt;
-      red[(warp * 64 + rlo) * 16 + tok] = acc[rt][nt][0];
-      red[(warp * 64 + rlo) * 16 + tok + 1] = acc[rt][nt][1];
-      red[(warp * 64 + rlo + 8) * 16 + tok] = acc[rt][nt][2];
-      red[(warp * 64 + rlo + 8) * 16 + tok + 1] = acc[rt][nt][3];
+// --------------------------------------------------------------- dec_tail --
+// CTA = 64 rows of one token; thread (q, r) sums the q-th quarter of the
+// slabs for row r, and the quarters are added in order.
+__global__ void __launch_bounds__(kTailThreads) dec_tail_kernel(DecodeParams p) {
+  constexpr int R = kTailThreads / 4;
+  __shared__ float ts[64];
+  __shared__ float tq[4][64];
+  __shared__ float pq[4][R];
+  const int q = threadIdx.x / R, r = threadIdx.x % R;
+  const int m = blockIdx.x * R + r, tok = blockIdx.y;
+  const bool live = m < p.M;
+  // packed inputs first: they are not produced upstream
+  uint4 ur[2];
+  ur[0] = ur[1] = make_uint4(0u, 0u, 0u, 0u);
+  if (live)
+    for (int i = 0; i < 2; ++i) {
+      const int rr = 8 * (2 * q + i);
+      if (rr < p.rank) ur[i] = *reinterpret_cast<const uint4 *>(p.U + (size_t)m * p.rank + rr);
     }
-  __syncthreads();
-  for (int i = tid; i < kDecBM * p.T; i += kDecThreads) {
-    const int tok = i >> 6, r = i & 63, m = m0 + r;
-    if (m >= p.M) continue;
-    float v = 0.0f;
+  const float bv = (live && p.bias && q == 0) ? bf16_bits_to_f32(p.bias[m]) : 0.0f;
+  pdl_wait();
+  pdl_launch_dependents();
+  int nsl = p.nslab;
+  if (p.tail_mode == 1 && live) {
+    const long long t = m / 16;
+    nsl = cta_of_unit((t + 1) * p.row_ut - 1, p.row_grid, p.row_units) -
+          cta_of_unit(t * p.row_ut, p.row_grid, p.row_units) + 1;
+  }
+  // t = V x_rot: slab quarter q of rank index r
+  if (r < p.rank) {
+    const int s0 = (q * p.nslab) / 4, s1 = ((q + 1) * p.nslab) / 4;
+    float t = 0.0f;
+    int s = s0;
+    for (; s + 8 <= s1; s += 8) {
+      float tv[8];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[(w * 64 + r) * 16 + tok];
-    for (int rr = 0; rr < p.rank; ++rr)
-      v = fmaf(bf16_bits_to_f32(su[r * p.rank + rr]), tps[rr * p.T + tok], v);
-    if (p.KT == 1) {
-      if (p.bias) v += bf16_bits_to_f32(p.bias[m]);
-      if (p.y_bf16)
-        reinterpret_cast<uint16_t *>(p.y)[(size_t)tok * p.M + m] = f32_to_bf16_rn_bits(v);
-      else
-        reinterpret_cast<float *>(p.y)[(size_t)tok * p.M + m] = v;
-    } else {
-      p.part[((size_t)kt * p.T + tok) * p.M + m] = v;
+      for (int i = 0; i < 8; ++i) tv[i] = __ldcg(&p.tpart[((size_t)(s + i) * p.rank + r) * p.T + tok]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t += tv[i];
+    }
+    for (; s < s1; ++s) t += __ldcg(&p.tpart[((size_t)s * p.rank + r) * p.T + tok]);
+    tq[q][r] = t;
+  }
+  float v = 0.0f;
+  if (live) {
+    const int s0 = (q * nsl) / 4, s1 = ((q + 1) * nsl) / 4;
+    const float *src = p.part + (size_t)tok * p.M + m;
+    const size_t stride = (size_t)p.T * p.M;
+    int s = s0;
+    for (; s + 16 <= s1; s += 16) {
+      float pv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pv[i] = __ldcg(src + (size_t)(s + i) * stride);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v += pv[i];
+    }
+    float pv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pv[i] = s + i < s1 ? __ldcg(src + (size_t)(s + i) * stride) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v += pv[i];
+  }
+  pq[q][r] = v;
+  __syncthreads();
+  if (threadIdx.x < p.rank)
+    ts[threadIdx.x] = ((tq[0][threadIdx.x] + tq[1][threadIdx.x]) + tq[2][threadIdx.x]) + tq[3][threadIdx.x];
+  __syncthreads();
+  // U t: quarter q takes rank indices [16q, 16q + 16)
+  float ut = 0.0f;
+  for (int i = 0; i < 2; ++i) {
+    const int rr = 8 * (2 * q + i);
+    if (rr >= p.rank) break;
+    const uint32_t w[4] = {ur[i].x, ur[i].y, ur[i].z, ur[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ut = fmaf(bf16_bits_to_f32(w[j] & 0xFFFFu), ts[rr + 2 * j], ut);
+      ut = fmaf(bf16_bits_to_f32(w[j] >> 16), ts[rr + 2 * j + 1], ut);
     }
   }
-  if (p.KT == 1) return;
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&p.counters[rb], 1u) == (unsigned)(p.KT - 1));
+  tq[q][r] = ut;
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // last CTA of this row block: sum the partials in k order
-  for (int i = tid; i < kDecBM * p.T; i += kDecThreads) {
-    const int tok = i >> 6, r = i & 63, m = m0 + r;
-    if (m >= p.M) continue;
-    float v = 0.0f;
-    int k = 0;
-    for (; k + 8 <= p.KT; k += 8) {
-      float pv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) pv[u] = __ldcg(&p.part[((size_t)(k + u) * p.T + tok) * p.M + m]);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v += pv[u];
-    }
-    for (; k < p.KT; ++k) v += __ldcg(&p.part[((size_t)k * p.T + tok) * p.M + m]);
-    if (p.bias) v += bf16_bits_to_f32(p.bias[m]);
-    if (p.y_bf16)
-      reinterpret_cast<uint16_t *>(p.y)[(size_t)tok * p.M + m] = f32_to_bf16_rn_bits(v);
-    else
-      reinterpret_cast<float *>(p.y)[(size_t)tok * p.M + m] = v;
-  }
+  if (q != 0 || !live) return;
+  float y = ((pq[0][r] + pq[1][r]) + pq[2][r]) + pq[3][r];
+  y += ((tq[0][r] + tq[1][r]) + tq[2][r]) + tq[3][r];
+  y += bv;
+  if (p.y_bf16)
+    reinterpret_cast<uint16_t *>(p.y)[(size_t)tok * p.M + m] = f32_to_bf16_rn_bits(y);
+  else
+    reinterpret_cast<float *>(p.y)[(size_t)tok * p.M + m] = y;
 }
 
 // ---------------------------------------------------------------- host ---
 namespace {
 
-struct DecTile {
-  int NR, BK, KT, RB, SE, nq8box;
-};
+std::mutex g_sm_mu;
+std::vector<int> g_sm_count;
 
-// Columns per CTA: one round (1024) by default; two rounds when the grid
-// would not fit the resident CTA slots.  DVSSQ_DECODE_ROUNDS overrides it
-// (tuning only).
-DecTile dec_tile(int M, int K, int n_sal, int T) {
-  DecTile d;
-  const int RB = (M + kDecBM - 1) / kDecBM;
-  // two rounds when the grid would overfill the resident CTA slots, and for
-  // T <= 8, where longer k-slices amortise the per-CTA work
-  int NR = 1;
-  const int slots = 148 * (T <= 8 ? 3 : 2);
-  if (K > kDecRound &&
-      ((long long)RB * ((K + kDecRound - 1) / kDecRound) > slots || T <= 8))
-    NR = 2;
-  if (const char *env = getenv("DVSSQ_DECODE_ROUNDS")) {
-    const int v = atoi(env);
-    if (v >= 1 && v <= kDecMaxNR) NR = v;
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(g_sm_mu);
+  if ((int)g_sm_count.size() <= dev) g_sm_count.resize(dev + 1, 0);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
   }
-  d.NR = NR;
-  d.BK = kDecRound * NR;
-  d.KT = (K + d.BK - 1) / d.BK;
-  d.RB = RB;
-  const int boxes = (n_sal + 63) / 64;
-  d.SE = n_sal > 0 ? 64 * ((boxes + d.KT - 1) / d.KT) : 0;
-  d.nq8box = d.SE / 64;
-  return d;
+  return g_sm_count[dev];
 }
 
-size_t dec_smem_bytes(const DecTile &d) {
-  return 1024 + (size_t)4 * d.NR * kDecQ4Box + (size_t)d.nq8box * kDecQ8Box +
-         (size_t)kDecBM * 16 * d.NR * 2 + (size_t)kDecBM * 64 * 2 + 64 * 16 * 4 + kDecBM * 4 +
-         (size_t)(4 * d.NR + 2) * 8;
+struct DecPlan {
+  int nslab, ntile, units, grid, upc_max, ns_max, NT, ntok, nscr, q8_budget;
+  DecLayout L;
+  bool ok;
+};
+
+int slabs_spanned(long long units, int grid, int ntile, int c) {
+  const int u0 = (int)((c * units) / grid), u1 = (int)(((c + 1) * units) / grid);
+  if (u1 <= u0) return 0;
+  return (u1 - 1) / ntile - u0 / ntile + 1;
+}
+
+// Grid, per-CTA maxima and the shared-memory layout of one decode call.
+DecPlan dec_plan(int M, int K, int block, int T, int nsm) {
+  DecPlan d{};
+  d.nslab = (K + kSlab - 1) / kSlab;
+  d.ntile = (M + kUnitRows - 1) / kUnitRows;
+  d.units = d.nslab * d.ntile;
+  d.NT = T <= 8 ? 1 : 2;
+  d.ntok = 8 * d.NT;
+  int grid = std::min(d.units, nsm);
+  for (;;) {
+    const int upc = (d.units + grid - 1) / grid;
+    int ns = 0;
+    for (int c = 0; c < grid; ++c) ns = std::max(ns, slabs_spanned(d.units, grid, d.ntile, c));
+    if ((upc <= kDecMaxUnits && ns <= kDecMaxSlabs) || grid >= d.units) {
+      d.grid = grid;
+      d.upc_max = upc;
+      d.ns_max = ns;
+      break;
+    }
+    grid = std::min(d.units, grid + std::max(1, grid / 4));
+  }
+  const int P = block / 16;
+  const int gpw = 32 / P;                          // Hadamard groups per warp
+  const int nbr = d.ns_max * (kSlab / block) * T;
+  int nscr = std::min(nbr, block == 256 ? 16 : 32);
+  nscr = (nscr + gpw - 1) / gpw * gpw;             // whole warps
+  d.nscr = nscr;
+  const int scr_elems = 16 * (P + 1) + 1;
+  auto al = [](int v, int a) { return (v + a - 1) / a * a; };
+  DecLayout &L = d.L;
+  int off = 0;
+  L.q4 = off;     off += d.upc_max * kQ4Unit;
+  L.s4 = off;     off += d.upc_max * kS4Unit;
+  L.xq = off;     off += al(d.ns_max * d.ntok * kXRow * 2, 128);
+  L.xs = off;     off += al(d.ns_max * d.ntok * kXsRow * 2, 128);
+  L.corr = off;   off += al(d.ns_max * 4 * d.ntok * 4, 128);
+  L.c8 = off;     off += al(d.ns_max * d.ntok * 4, 128);
+  L.s8 = off;     off += al(d.upc_max * kUnitRows * 4, 128);
+  L.colpos = off; off += al(d.ns_max * kSlab * 2, 128);
+  L.samp = off;   off += kSamples * 4;
+  L.scr = off;    off += al(d.nscr * scr_elems * 4, 128);
+  L.meta = off;   off += 512;
+  L.bars = off;   off += al(d.upc_max * 8, 128);
+  L.q8 = off;
+  const int room = kSmemLimit - 1024 - off;
+  d.q8_budget = std::max(0, std::min(room, d.upc_max * 4 * kQ8Chunk)) / kQ8Chunk * kQ8Chunk;
+  off += d.q8_budget;
+  L.total = off + 1024;
+  d.ok = room >= 0 && d.upc_max <= kDecMaxUnits && d.ns_max <= kDecMaxSlabs;
+  return d;
 }
 
 }  // namespace
 
+size_t decode_row_slices(int K, int n_sal);
+
 size_t decode_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T) {
-  const DecTile d = dec_tile(M, K, n_sal, T);
+  (void)block;
+  const size_t nslab = (size_t)(K + kSlab - 1) / kSlab;
+  const size_t slices = T <= 2 ? std::max(nslab, decode_row_slices(K, n_sal)) : nslab;
   size_t off = 0;
   auto take = [&](size_t b) { off += (b + 255) & ~(size_t)255; };
-  take((size_t)T * K * 2);                       // xr16
-  take((size_t)T * n_sal * 2 + 16);              // xs16
-  take((size_t)(K / block) * rank * T * 4);      // tp
-  take((size_t)d.KT * T * M * 4);                // split-K partials
-  take((size_t)d.RB * 4);                        // counters
+  take(slices * T * M * 4);            // partials (per slab, or per CTA of a tile)
+  take(nslab * rank * T * 4 + 16);     // per-slab shares of t = V x_rot
   return off;
 }
 
+cudaError_t launch_decode_row(const ForwardArgs &a, cudaStream_t st, Launcher &L);
+cudaError_t prepare_decode_row_kernels();
+
 cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
-  const DecTile d = dec_tile(a.M, a.K, a.n_sal, a.T);
+  if (a.T <= 2) {
+    const cudaError_t e = launch_decode_row(a, st, L);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  const DecPlan d = dec_plan(a.M, a.K, a.block, a.T, sm_count());
+  if (!d.ok) {
+    set_last_error("decode: no shared-memory plan fits this shape");
+    return cudaErrorInvalidConfiguration;
+  }
   DecodeParams p;
   p.M = a.M; p.K = a.K; p.T = a.T; p.n_sal = a.n_sal; p.rank = a.rank; p.block = a.block;
-  p.nkb = a.K / a.block;
-  p.NR = d.NR; p.BK = d.BK; p.KT = d.KT; p.RB = d.RB; p.SE = d.SE; p.nq8box = d.nq8box;
+  p.nslab = d.nslab; p.ntile = d.ntile; p.units = d.units; p.grid = d.grid;
+  p.upc_max = d.upc_max; p.ns_max = d.ns_max; p.ntok = d.ntok; p.nscr = d.nscr;
+  p.q8_budget = d.q8_budget;
   p.c = (float)sqrt(1.0 / (double)a.block);
-  p.s4 = a.s4; p.sal_idx = a.sal_idx; p.s8 = a.s8; p.U = a.U; p.V = a.V;
+  p.s4 = a.s4; p.sal_idx = a.sal_idx; p.q8 = a.q8; p.s8 = a.s8; p.U = a.U; p.V = a.V;
   p.x = a.x; p.bias = a.bias; p.y = a.y; p.y_bf16 = a.y_bf16;
+  p.L = d.L;
+  p.tail_mode = 0; p.row_grid = 1; p.row_units = 1; p.row_ut = 1;
   char *ws = static_cast<char *>(a.workspace);
   size_t off = 0;
   auto take = [&](size_t b) { char *q = ws + off; off += (b + 255) & ~(size_t)255; return q; };
-  p.xr16 = reinterpret_cast<__half *>(take((size_t)a.T * a.K * 2));
-  p.xs16 = reinterpret_cast<__half *>(take((size_t)a.T * a.n_sal * 2 + 16));
-  p.tp = reinterpret_cast<float *>(take((size_t)p.nkb * a.rank * a.T * 4));
-  p.part = reinterpret_cast<float *>(take((size_t)p.KT * a.T * a.M * 4));
-  p.counters = reinterpret_cast<unsigned int *>(take((size_t)p.RB * 4));
+  p.part = reinterpret_cast<float *>(take((size_t)d.nslab * a.T * a.M * 4));
+  p.tpart = reinterpret_cast<float *>(take((size_t)d.nslab * a.rank * a.T * 4 + 16));
 
-  CUtensorMap mq4, mq8, ms4, mu;
+  CUtensorMap mq4, ms4, mq8;
   if (encode_tmap_2d(&mq4, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q4, (uint64_t)a.K / 2, (uint64_t)a.M,
-                     (uint64_t)a.K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                     (uint64_t)a.K / 2, 128, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B) !=
+      CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // scale rows are K/32 bytes: a tensor map needs a multiple of 16, and the
-  // box start (k0/64 elements) is aligned because k0 is a multiple of 1024
+  // s4 rows are K/32 bytes: a tensor map needs a multiple of 16
   p.s4_tma = (a.K % 512 == 0) && ((uintptr_t)a.s4 % 16 == 0);
   ms4 = mq4;
-  if (p.s4_tma &&
-      encode_tmap_2d(&ms4, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s4, (uint64_t)a.K / 64,
-                     (uint64_t)a.M, (uint64_t)a.K / 32, 16 * d.NR, 64,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+  if (p.s4_tma && encode_tmap_2d(&ms4, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s4, (uint64_t)a.K / 64,
+                                 (uint64_t)a.M, (uint64_t)a.K / 32, 8, kUnitRows,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
     p.s4_tma = 0;
-  p.u_tma = a.rank > 0 && (a.rank % 8 == 0) && ((uintptr_t)a.U % 16 == 0);
-  mu = mq4;
-  if (p.u_tma &&
-      encode_tmap_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.U, (uint64_t)a.rank, (uint64_t)a.M,
-                     (uint64_t)a.rank * 2, a.rank, 64, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
-    p.u_tma = 0;
-  if (a.n_sal > 0) {
-    if (encode_tmap_2d(&mq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q8, (uint64_t)a.n_sal,
-                       (uint64_t)a.M, (uint64_t)a.n_sal, 64, 64,
-                       CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  } else {
-    mq8 = mq4;   // never used
-  }
+  mq8 = mq4;   // never read when there are no salient columns
+  if (a.n_sal > 0 &&
+      encode_tmap_2d(&mq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q8, (uint64_t)a.n_sal, (uint64_t)a.M,
+                     (uint64_t)a.n_sal, 16, kUnitRows, CU_TENSOR_MAP_SWIZZLE_NONE) !=
+          CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
   cudaError_t e;
-  const size_t vsm = (size_t)a.rank * (a.block + 8) * 2;
+  const dim3 grid(d.grid), block(kDecThreads);
+  const size_t smem = d.L.total;
   if (a.block == 256)
-    e = L.launch("dec_prologue", dec_prologue_kernel<256>, dim3(p.nkb), dim3(256), vsm, st, false, p);
+    e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<256, 1>, grid, block, smem, st, true,
+                             mq4, ms4, mq8, p)
+                  : L.launch("dec_main", dec_main_kernel<256, 2>, grid, block, smem, st, true,
+                             mq4, ms4, mq8, p);
   else
-    e = L.launch("dec_prologue", dec_prologue_kernel<128>, dim3(p.nkb), dim3(128), vsm, st, false, p);
+    e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<128, 1>, grid, block, smem, st, true,
+                             mq4, ms4, mq8, p)
+                  : L.launch("dec_main", dec_main_kernel<128, 2>, grid, block, smem, st, true,
+                             mq4, ms4, mq8, p);
   if (e != cudaSuccess) return e;
-  const size_t smem = dec_smem_bytes(d);
-  if (a.T <= 8)
-    return L.launch("dec_main", dec_main_kernel<1>, dim3(p.RB, p.KT), dim3(kDecThreads), smem, st,
-                    true, mq4, mq8, ms4, mu, p);
-  return L.launch("dec_main", dec_main_kernel<2>, dim3(p.RB, p.KT), dim3(kDecThreads), smem, st,
-                  true, mq4, mq8, ms4, mu, p);
+  return L.launch("dec_tail", dec_tail_kernel, dim3((a.M + kTailThreads / 4 - 1) / (kTailThreads / 4), a.T),
+                  dim3(kTailThreads), 0, st, true, p);
 }
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-  for (const void *f : {(const void *)dec_main_kernel<1>, (const void *)dec_main_kernel<2>,
-                        (const void *)dec_prologue_kernel<256>, (const void *)dec_prologue_kernel<128>})
+  for (const void *f :
+       {(const void *)dec_main_kernel<256, 1>, (const void *)dec_main_kernel<256, 2>,
+        (const void *)dec_main_kernel<128, 1>, (const void *)dec_main_kernel<128, 2>}) {
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
-  if ((e = cudaFuncSetAttribute(dec_main_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                200 * 1024)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(dec_main_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                200 * 1024)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(dec_prologue_kernel<256>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 264 * 2)) !=
-      cudaSuccess)
-    return e;
-  return cudaFuncSetAttribute(dec_prologue_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              64 * 136 * 2);
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kSmemLimit)) != cudaSuccess)
+      return e;
+  }
+  (void)sm_count();
+  return prepare_decode_row_kernels();
 }
 
 }  // namespace dvssq

@@ -4,5 +4,6 @@
 #include "fwht.cu"
 #include "encode.cu"
 #include "decode.cu"
+#include "decode_row.cu"
 #include "prefill.cu"
 #include "static_scratch.cu"
