@@ -73,18 +73,9 @@ struct DecodeParams {
   int y_bf16;
   float *part;    // [slice][T][M]
   float *tpart;   // [nslab][rank][T]
-  // partial slices summed by dec_tail: all nslab slices (slab-major
-  // kernel), or, per 16-row tile, the CTAs of a tile-major grid of row_grid
-  // CTAs over row_units units of row_ut units per tile
-  int tail_mode, row_grid, row_units, row_ut;
+  int nslices;    // partial slices dec_tail sums for every output
   DecLayout L;
 };
-
-// CTA of a grid of G CTAs over U units (CTA c holds [c U / G, (c + 1) U / G))
-// that holds unit u.
-__host__ __device__ inline int cta_of_unit(long long u, int G, long long U) {
-  return (int)(((u + 1) * G - 1) / U);
-}
 
 // Position i of each 16-column segment of the FP16 x_rot holds column
 // perm16(i): the order in which nibble pairs come out of dequant_q4_biased,
@@ -571,12 +562,7 @@ __global__ void __launch_bounds__(kTailThreads) dec_tail_kernel(DecodeParams p) 
   const float bv = (live && p.bias && q == 0) ? bf16_bits_to_f32(p.bias[m]) : 0.0f;
   pdl_wait();
   pdl_launch_dependents();
-  int nsl = p.nslab;
-  if (p.tail_mode == 1 && live) {
-    const long long t = m / 16;
-    nsl = cta_of_unit((t + 1) * p.row_ut - 1, p.row_grid, p.row_units) -
-          cta_of_unit(t * p.row_ut, p.row_grid, p.row_units) + 1;
-  }
+  const int nsl = p.nslices;
   // t = V x_rot: slab quarter q of rank index r
   if (r < p.rank) {
     const int s0 = (q * p.nslab) / 4, s1 = ((q + 1) * p.nslab) / 4;
@@ -762,7 +748,7 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   p.s4 = a.s4; p.sal_idx = a.sal_idx; p.q8 = a.q8; p.s8 = a.s8; p.U = a.U; p.V = a.V;
   p.x = a.x; p.bias = a.bias; p.y = a.y; p.y_bf16 = a.y_bf16;
   p.L = d.L;
-  p.tail_mode = 0; p.row_grid = 1; p.row_units = 1; p.row_ut = 1;
+  p.nslices = d.nslab;
   char *ws = static_cast<char *>(a.workspace);
   size_t off = 0;
   auto take = [&](size_t b) { char *q = ws + off; off += (b + 255) & ~(size_t)255; return q; };
