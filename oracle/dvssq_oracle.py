@@ -49,6 +49,11 @@ R8  Forward: y = sum_j (q_ij s4_ig) xr_j + s8_i sum_k q8_ik xr_{sal_k}
     not rounded.
 R9  Nibble packing: two's-complement 4-bit codes, two per byte, the even
     rotated column in the low nibble.
+R10 MLP block of the Spark shape ("Myric/Spark-X2.5-4B-GGUF", "The model":
+    GELU FFN, 36 layers; "Spark-X2.5-4B-ASHQ1-GGUF", "Architecture":
+    ffn_gate / ffn_up / ffn_down): x_next = down(GELU(gate x) * up x) with
+    the exact erf GELU, no norm or residual, and hidden states rounded to
+    BF16 after every projection and after the gated product.
 """
 from __future__ import annotations
 
@@ -448,5 +453,23 @@ def spark_model_footprint(hubs=(3, 7, 11, 15, 19, 23, 27, 31, 35), layers=36,
 
 
 def gelu(v: np.ndarray) -> np.ndarray:
+    """Exact (erf) GELU, v * Phi(v), in fp64."""
     from scipy.special import erf
     return 0.5 * v * (1.0 + erf(v / math.sqrt(2.0)))
+
+
+def gelu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """R10: h = RN_bf16(gelu(g) * u) for BF16 g, u held as fp64."""
+    return rn_bf16(gelu(np.asarray(g, np.float64)) * np.asarray(u, np.float64))
+
+
+def mlp_block(enc_gate: dict, enc_up: dict, enc_down: dict, x: np.ndarray) -> np.ndarray:
+    """R10: one Spark-shaped MLP block on the packed form, BF16 between steps.
+
+    g = RN_bf16(gate x), u = RN_bf16(up x), h = RN_bf16(gelu(g) u),
+    x_next = RN_bf16(down h); every projection is forward() in fp64.
+    """
+    g = rn_bf16(forward(enc_gate, x))
+    u = rn_bf16(forward(enc_up, x))
+    h = gelu_mul(g, u)
+    return rn_bf16(forward(enc_down, h))

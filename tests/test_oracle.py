@@ -403,3 +403,51 @@ def test_oracle_is_independent_of_library():
     import oracle.dvssq_oracle as mod
     src = open(mod.__file__).read()
     assert "mixed_precision_weight_b200" not in src and "ctypes" not in src
+
+
+# ------------------------------------------------------------- R10 MLP block --
+
+def test_gelu_closed_forms():
+    # gelu(v) = v * Phi(v): Phi(0) = 1/2, Phi(1) and Phi(-2) from the normal table
+    assert O.gelu(np.array([0.0]))[0] == 0.0
+    assert abs(O.gelu(np.array([1.0]))[0] - 0.8413447460685429) < 1e-15
+    assert abs(O.gelu(np.array([-2.0]))[0] - (-2.0 * 0.022750131948179195)) < 1e-15
+    v = np.linspace(-6, 6, 97)
+    # Phi(v) + Phi(-v) = 1  =>  gelu(v) - gelu(-v) = v
+    assert np.allclose(O.gelu(v) - O.gelu(-v), v, rtol=0, atol=1e-14)
+    assert np.all(O.gelu(np.array([40.0])) == 40.0)
+
+
+def test_gelu_mul_rounds_once_to_bf16():
+    rng = np.random.default_rng(4)
+    g = O.rn_bf16(rng.normal(size=257))
+    u = O.rn_bf16(rng.normal(size=257))
+    h = O.gelu_mul(g, u)
+    assert np.array_equal(h, O.rn_bf16(h))                  # already BF16
+    exact = O.gelu(g) * u
+    # BF16 spacing at |v| in [2^e, 2^(e+1)) is 2^(e-7); RN errs by at most half
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))) - 7)
+    assert np.all(np.abs(h - exact) <= 0.5 * ulp)
+
+
+def test_mlp_block_matches_dense_composition():
+    # the block on the packed form equals the composition written with each
+    # layer's effective dense weight, with the same BF16 rounding points
+    rng = np.random.default_rng(5)
+    H, I = 256, 512
+    encs = []
+    for (M, K), seed in (((I, H), 1), ((I, H), 2), ((H, I), 3)):
+        W = O.rn_bf16(rng.normal(scale=0.05, size=(M, K)))
+        act = np.abs(rng.normal(size=K)) + 0.1
+        encs.append(O.encode(W, act, 256, 4))
+    x = O.rn_bf16(rng.normal(size=(2, H)))
+    y = O.mlp_block(*encs, x)
+    Wg, Wu, Wd = (O.dense_effective_weight(e) for e in encs)
+    g = O.rn_bf16(x @ Wg.T)
+    u = O.rn_bf16(x @ Wu.T)
+    h = O.rn_bf16(O.gelu(g) * u)
+    ref = O.rn_bf16(h @ Wd.T)
+    # identical up to fp64 rounding of the two summation orders: BF16 values
+    # may differ only where a sum lands within ~1e-12 of a rounding boundary
+    assert np.mean(y == ref) > 0.99
+    assert np.max(np.abs(y - ref)) <= 2.0 ** -7 * np.max(np.abs(ref))
