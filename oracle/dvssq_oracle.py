@@ -453,9 +453,15 @@ def spark_model_footprint(hubs=(3, 7, 11, 15, 19, 23, 27, 31, 35), layers=36,
 
 
 def gelu(v: np.ndarray) -> np.ndarray:
-    """Exact (erf) GELU, v * Phi(v), in fp64."""
-    from scipy.special import erf
-    return 0.5 * v * (1.0 + erf(v / math.sqrt(2.0)))
+    """Exact (erf) GELU, v * Phi(v), in fp64.
+
+    Phi(v) = erfc(-v / sqrt 2) / 2 -- the same function as (1 + erf(v/sqrt 2))/2,
+    written so that it keeps its relative accuracy for negative v (1 + erf
+    cancels to 0 in fp64 below v ~ -8).
+    """
+    from scipy.special import erfc
+    v = np.asarray(v, dtype=np.float64)
+    return 0.5 * v * erfc(-v / math.sqrt(2.0))
 
 
 def gelu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:

@@ -416,6 +416,8 @@ def test_gelu_closed_forms():
     # Phi(v) + Phi(-v) = 1  =>  gelu(v) - gelu(-v) = v
     assert np.allclose(O.gelu(v) - O.gelu(-v), v, rtol=0, atol=1e-14)
     assert np.all(O.gelu(np.array([40.0])) == 40.0)
+    # deep negative tail: Phi(-10) = 7.619853024160527e-24 (normal table)
+    assert abs(O.gelu(np.array([-10.0]))[0] / (-10.0 * 7.619853024160527e-24) - 1) < 1e-12
 
 
 def test_gelu_mul_rounds_once_to_bf16():
