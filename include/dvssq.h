@@ -145,6 +145,21 @@ DVSSQ_API const char *dvssq_last_error(void);
 DVSSQ_API dvssq_status dvssq_fwht(const void *x, float *y, int64_t rows, int32_t cols,
                         int32_t block, void *stream);
 
+/* Gated GELU of a Spark-shaped MLP block, the step between the up and down
+ * projections ("Myric/Spark-X2.5-4B-GGUF", "The model": GELU FFN;
+ * "Spark-X2.5-4B-ASHQ1-GGUF", "Architecture": ffn_gate / ffn_up /
+ * ffn_down).  The pages name the activation only; the gated erf form is this
+ * library's reading:
+ *   h[i] = RN_bf16( gelu(gate[i]) * up[i] ),  gelu(v) = v/2 (1 + erf(v/sqrt 2))
+ * evaluated in FP32.
+ *   gate, up  bf16 [n]  (device, caller-owned)
+ *   h         bf16 [n]  (device; may alias gate or up)
+ *   n         >= 0 (0 is a no-op); all three pointers 16-byte aligned
+ * Stream-ordered and asynchronous.
+ * Errors: INVALID_ARG, MISALIGNED, DEVICE, CUDA.                            */
+DVSSQ_API dvssq_status dvssq_gelu_mul(const void *gate, const void *up, void *h, int64_t n,
+                                      void *stream);
+
 /* Bytes of workspace dvssq_encode needs for `shape` (host only; no CUDA). */
 DVSSQ_API dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes);
 

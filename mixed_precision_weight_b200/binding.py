@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
-    "dvssq_fwht", "dvssq_encode_workspace_size", "dvssq_encode",
+    "dvssq_fwht", "dvssq_gelu_mul", "dvssq_encode_workspace_size", "dvssq_encode",
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
     "dvssq_device_error", "STATIC_SCRATCH_BYTES",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
@@ -45,6 +45,7 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 EXPORTED_SYMBOLS = (
     "dvssq_abi_version", "dvssq_status_string", "dvssq_last_error", "dvssq_fwht",
+    "dvssq_gelu_mul",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
     "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_device_error",
     "dvssq_profile_enable",
@@ -84,6 +85,7 @@ _sig = {
     "dvssq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dvssq_last_error": (ctypes.c_char_p, []),
     "dvssq_fwht": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P]),
+    "dvssq_gelu_mul": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P]),
     "dvssq_encode_workspace_size": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)]),
     "dvssq_encode": (ctypes.c_int, [ctypes.POINTER(Shape), _P, _P, ctypes.POINTER(_Weights), _P,
                                     ctypes.POINTER(_EncodeInfo), _P, ctypes.c_size_t, _P]),
@@ -172,6 +174,18 @@ class PackedWeights:
                         self.q8.data_ptr() if has_sal else None, self.s8.data_ptr(),
                         self.U.data_ptr() if self.U is not None and shape.rank > 0 else None,
                         self.V.data_ptr() if self.V is not None and shape.rank > 0 else None)
+
+
+def dvssq_gelu_mul(gate: torch.Tensor, up: torch.Tensor, h: torch.Tensor | None = None,
+                   stream=None):
+    """h = RN_bf16(gelu(gate) * up) elementwise, BF16 in and out."""
+    if gate.dtype != torch.bfloat16 or up.dtype != torch.bfloat16 or gate.shape != up.shape:
+        raise TypeError("gate and up must be bfloat16 tensors of one shape")
+    if h is None:
+        h = torch.empty_like(gate)
+    _check(lib.dvssq_gelu_mul(_ptr(gate), _ptr(up), _ptr(h), gate.numel(), _stream(stream)),
+           "dvssq_gelu_mul")
+    return h
 
 
 def dvssq_fwht(x: torch.Tensor, block: int, y: torch.Tensor | None = None, stream=None):

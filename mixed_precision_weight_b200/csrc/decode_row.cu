@@ -406,10 +406,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
       if (uf < u0 || uf >= u1) continue;
       uint4 vreg[NV];
       const int c0 = kSlab * s + 8 * lane;          // 8 columns = one DP2A segment
-#pragma unroll
       // the first owned slab came by TMA with the weights; a further one
       // (only for very wide layers) is read from global memory
       const bool staged = s == s_own && mbar_wait(vbar, 0);
+#pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int rr = cw + kCons * i;
         if (staged) {

@@ -173,6 +173,19 @@ dvssq_status dvssq_fwht(const void *x, float *y, int64_t rows, int32_t cols, int
   return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
 }
 
+dvssq_status dvssq_gelu_mul(const void *gate, const void *up, void *h, int64_t n, void *stream) {
+  if (n < 0 || n > ((int64_t)1 << 40)) return DVSSQ_ERR_INVALID_ARG;
+  if (n == 0) return DVSSQ_OK;
+  if (gate == nullptr || up == nullptr || h == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(h)) return DVSSQ_ERR_MISALIGNED;
+  dvssq_status s = ensure_device();
+  if (s != DVSSQ_OK) return s;
+  cudaError_t e = launch_gelu_mul(static_cast<const uint16_t *>(gate),
+                                  static_cast<const uint16_t *>(up), static_cast<uint16_t *>(h),
+                                  n, static_cast<cudaStream_t>(stream), launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
 dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes) {
   dvssq_status s = check_shape(shape);
   if (s != DVSSQ_OK) return s;

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <string>
 #include <utility>
 #include <vector>
@@ -95,6 +96,8 @@ cudaError_t prepare_encode_kernels();
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L);
 
 // ------------------------------------------------------------ activations -
+cudaError_t launch_gelu_mul(const uint16_t *g, const uint16_t *u, uint16_t *h, long long n,
+                            cudaStream_t st, Launcher &L);
 cudaError_t launch_fwht(const uint16_t *x, float *y, int64_t rows, int cols, int block,
                         cudaStream_t st, Launcher &L);
 

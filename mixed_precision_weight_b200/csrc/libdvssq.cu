@@ -2,6 +2,7 @@
 // error word) and helpers without relocatable device code.
 #include "dvssq_api.cu"
 #include "fwht.cu"
+#include "glue.cu"
 #include "encode.cu"
 #include "decode.cu"
 #include "decode_row.cu"
