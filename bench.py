@@ -1,20 +1,25 @@
 """Benchmark of the DV-SSQ layer on B200: one JSON line on rank 0.
 
-A step is one pass of the whole path on the Spark-shaped down_proj layer
-(W 2560 x 10240 BF16, H_256 blocks, 1280 salient columns, rank 16):
-    encode W  ->  forward of 1 token  ->  forward of 16 tokens.
-The metric's unit is GB/s of algorithmic bytes: the encoder reads W once and
-writes the packed form; each forward reads the packed layer once (x and y
-are not counted).  Eight independent copies of the layer (about 1.1 GB) are
-used in rotation so that no step finds its inputs in the 126 MB L2, and the
-forwards of a step read a copy that was encoded four steps earlier.
+Default step (the Spark-shaped down_proj: W 2560 x 10240 BF16, H_256 blocks,
+1280 salient columns, rank 16): encode W -> forward of 1 token -> forward of
+16 tokens.  The unit is GB/s of algorithmic bytes: the encoder reads W once
+and writes the packed form; each forward reads the packed layer once (x and y
+are not counted).  Eight independent copies of the layer are used in
+rotation so that no step finds its inputs in the 126 MB L2, and the forwards
+of a step read a copy that was encoded four steps earlier.
+
+Other workloads (--workload): decode (the two forwards only), prefill (4096
+tokens through the up_proj, TFLOP/s), bulk_encode (all 108 matrices of the
+36-layer Spark MLP stack) and stack (one token through the 36 x (gate, up,
+GELU, down) stack, 1.9 GB of packed weights per token).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload spark_down|spark_up_prefill|bulk_encode]
+                    [--workload spark_down|decode|prefill|bulk_encode|stack]
 
-With --gpus N > 1 (under torchrun, one process per GPU) every rank runs the
-same step on its own layers: the path has no data-path exchange, so scaling
-is weak and the timing is the max over ranks.
+The timed region replays one CUDA graph per rotation slot (--no-graphs
+launches eagerly instead).  With --gpus N > 1 (under torchrun, one process
+per GPU) every rank runs the same step on its own layers: the path has no
+data-path exchange, so scaling is weak and the timing is the max over ranks.
 """
 from __future__ import annotations
 
@@ -58,15 +63,19 @@ def encode_bytes(M, K, n_sal):
 
 
 def kernel_bytes(name, M, K, rank, n_sal, T):
-    """Algorithmic bytes of one launch of each kernel (see the design notes)."""
+    """Algorithmic bytes of one launch of each kernel (see the design notes).
+
+    The decode GEMV (dec_row for one or two tokens, dec_main above) reads the
+    packed layer except U; dec_tail reads U.  x, y and the partial sums are
+    not counted."""
     if name == "enc_pass1":
         return M * K * 2
     if name == "enc_pass2":
         return encode_bytes(M, K, n_sal)
-    if name == "dec_main":
-        return M * K // 2 + M * (K // 64) * 2 + M * n_sal + M * 2 + M * rank * 2
-    if name == "dec_prologue":
-        return rank * K * 2 + n_sal * 4 + T * K * 2
+    if name in ("dec_row", "dec_main"):
+        return packed_bytes(M, K, rank, n_sal) - M * rank * 2
+    if name == "dec_tail":
+        return M * rank * 2
     return None
 
 
@@ -186,13 +195,18 @@ class SparkDownStep:
             dv.dvssq_encode(self.shape, W, act, packed, workspace=self.ws_enc)
         self.i = 0
 
-    def step(self):
+    graph_slots = N_COPIES
+
+    def step_slot(self, i):
         dv = self.dv
-        W, act, packed = self.copies[self.i % N_COPIES]
+        W, act, packed = self.copies[i % N_COPIES]
         dv.dvssq_encode(self.shape, W, act, packed, workspace=self.ws_enc)
-        fwd = self.copies[(self.i + N_COPIES // 2) % N_COPIES][2]
+        fwd = self.copies[(i + N_COPIES // 2) % N_COPIES][2]
         dv.dvssq_linear_forward(self.shape, fwd, self.x1, y=self.y1, workspace=self.ws1)
         dv.dvssq_linear_forward(self.shape, fwd, self.x16, y=self.y16, workspace=self.ws16)
+
+    def step(self):
+        self.step_slot(self.i)
         self.i += 1
 
     def bytes_per_step(self):
@@ -257,12 +271,11 @@ class DecodeStep(SparkDownStep):
 
     name = "spark_down_proj_2560x10240_r16_fwd_T1+T16"
 
-    def step(self):
+    def step_slot(self, i):
         dv = self.dv
-        fwd = self.copies[self.i % N_COPIES][2]
+        fwd = self.copies[i % N_COPIES][2]
         dv.dvssq_linear_forward(self.shape, fwd, self.x1, y=self.y1, workspace=self.ws1)
         dv.dvssq_linear_forward(self.shape, fwd, self.x16, y=self.y16, workspace=self.ws16)
-        self.i += 1
 
     def bytes_per_step(self):
         return 2 * packed_bytes(self.M, self.K, self.r, self.n)
@@ -324,8 +337,13 @@ class PrefillStep:
                               device=device)
         self.y = torch.empty((self.T, self.M), dtype=torch.float32, device=device)
 
-    def step(self):
+    graph_slots = 1
+
+    def step_slot(self, i):
         self.dv.dvssq_linear_forward(self.shape, self.packed, self.x, y=self.y, workspace=self.ws)
+
+    def step(self):
+        self.step_slot(0)
 
     def work_per_step(self):
         return 2.0 * self.T * self.M * self.K + 2.0 * self.T * self.r * (self.K + self.M)
@@ -403,8 +421,131 @@ class BulkEncodeStep:
                 "parallelism": "replica per GPU"}
 
 
+class StackStep:
+    """One token through the 36-layer Spark MLP stack (decode, T = 1).
+
+    Per layer: g = gate(x), u = up(x) (BF16 outputs), h = RN_bf16(gelu(g) u),
+    x = down(h) (BF16); gate/up are 10240 x 2560 and down 2560 x 10240, rank
+    16 (layers 0..13 and 29..35) or 24 (14..28).  The 108 packed matrices
+    (1.9 GB) far exceed L2, so every token streams them all from HBM."""
+
+    name = "spark_mlp_stack_36x(gate,up,down)_T1"
+    graph_slots = 1
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv, self.torch, self.device = dv, torch, device
+        H, I = 2560, 10240
+        self.H, self.I = H, I
+        self.layers = []
+        ws = 0
+        for l in range(36):
+            r = synth.stack_rank(l)
+            mats = []
+            for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
+                seed = synth.layer_seed(1 + rank_id, l, which)
+                shape = dv.Shape.make(M, K, 256, r)
+                W = synth.weight_device(M, K, seed, device, n_outlier_cols=max(1, K // 1000),
+                                        outlier_scale=15.0)
+                act = synth.act_scale(K, seed).to(device)
+                U, V = synth.lowrank_factors(M, K, r, seed=seed + 17)
+                packed = dv.PackedWeights.empty(shape, device, U=U.to(device), V=V.to(device))
+                need = dv.dvssq_encode_workspace_size(shape)
+                if need > ws:
+                    self.ws_enc = torch.empty(need, dtype=torch.uint8, device=device)
+                    ws = need
+                dv.dvssq_encode(shape, W, act, packed, workspace=self.ws_enc)
+                del W
+                mats.append((shape, packed))
+            self.layers.append(mats)
+        del self.ws_enc
+        fw = max(dv.dvssq_forward_workspace_size(sh, 1) for mats in self.layers for sh, _ in mats)
+        self.ws = torch.empty(fw, dtype=torch.uint8, device=device)
+        self.x0 = synth.activations(1, H, seed=3 + rank_id, n_outlier=13,
+                                    outlier_scale=25.0).to(device)
+        self.x = torch.empty((1, H), dtype=torch.bfloat16, device=device)
+        self.g = torch.empty((1, I), dtype=torch.bfloat16, device=device)
+        self.u = torch.empty((1, I), dtype=torch.bfloat16, device=device)
+        self.h = torch.empty((1, I), dtype=torch.bfloat16, device=device)
+
+    def run(self, x, out):
+        dv = self.dv
+        cur = x
+        for l, ((sg, pg), (su, pu), (sd, pd)) in enumerate(self.layers):
+            dv.dvssq_linear_forward(sg, pg, cur, y=self.g, y_dtype=dv.Y_BF16, workspace=self.ws)
+            dv.dvssq_linear_forward(su, pu, cur, y=self.u, y_dtype=dv.Y_BF16, workspace=self.ws)
+            dv.dvssq_gelu_mul(self.g, self.u, self.h)
+            dv.dvssq_linear_forward(sd, pd, self.h, y=out, y_dtype=dv.Y_BF16, workspace=self.ws)
+            cur = out
+
+    def step_slot(self, i):
+        self.run(self.x0, self.x)
+
+    def step(self):
+        self.step_slot(0)
+
+    def bytes_per_step(self):
+        return sum(packed_bytes(sh.M, sh.K, sh.rank, sh.n_sal) for mats in self.layers
+                   for sh, _ in mats)
+
+    def launches_per_step(self):
+        return 36 * (3 * 2 + 1)
+
+    def kernel_work(self, name):
+        # average algorithmic bytes per launch over the stack's launches
+        shapes = [sh for mats in self.layers for sh, _ in mats]
+        per = [kernel_bytes(name, sh.M, sh.K, sh.rank, sh.n_sal, 1) for sh in shapes]
+        if name == "gelu_mul":
+            return 3 * self.I * 2
+        if any(v is None for v in per):
+            return None
+        return sum(per) / len(per)
+
+    def config(self):
+        return {"workload": self.name, "layers": 36, "hidden": self.H, "intermediate": self.I,
+                "block": 256, "rank": "16 (layers 0-13, 29-35), 24 (14-28)",
+                "n_sal": "K/8 per matrix", "tokens": 1,
+                "step": "36 x (dvssq_linear_forward gate, up -> dvssq_gelu_mul -> down), "
+                        "BF16 hidden states, one CUDA graph per token",
+                "packed_bytes_per_token": self.bytes_per_step(),
+                "l2": "1.9 GB of packed weights per token > 126 MB L2",
+                "lowrank_factors": "seeded synthetic U, V (values do not change the work)",
+                "parallelism": "replica per GPU"}
+
+    # ---- end-to-end: token in from pinned host memory, hidden state back ----
+    def e2e_setup(self, synth):
+        torch = self.torch
+        self.hx = synth.activations(1, self.H, seed=9, n_outlier=13,
+                                    outlier_scale=25.0).pin_memory()
+        self.hy = torch.empty((1, self.H), dtype=torch.bfloat16).pin_memory()
+        self.dx = torch.empty((1, self.H), dtype=torch.bfloat16, device=self.device)
+
+    def e2e_step(self):
+        self.dx.copy_(self.hx, non_blocking=True)
+        self.run(self.dx, self.x)
+        self.hy.copy_(self.x, non_blocking=True)
+
+    def e2e_bytes(self):
+        return self.H * 2, self.H * 2
+
+    # ---- the oracle on the host cores: forwards of one gate matrix ----
+    def oracle_sample(self, O, synth):
+        H, I = self.H, self.I
+        W = synth.weight(I, H, seed=77, n_outlier_cols=2, outlier_scale=15.0)
+        enc = O.encode(O.torch_bf16_to_f64(W), synth.act_scale(H, seed=77).numpy(), 256, 0,
+                       with_svd=False)
+        U, V = synth.lowrank_factors(I, H, 16, seed=78)
+        Uf, Vf = O.torch_bf16_to_f64(U), O.torch_bf16_to_f64(V)
+        x = O.torch_bf16_to_f64(synth.activations(1, H, seed=79))
+        self._oracle_bytes = packed_bytes(I, H, 16, H // 8)
+        self.oracle_what = "forward(s) of one 10240 x 2560 gate matrix (packed bytes per forward)"
+
+        def step():
+            O.forward(enc, x, U=Uf, V=Vf)
+        return step
+
+
 WORKLOADS = {"spark_down": SparkDownStep, "decode": DecodeStep, "prefill": PrefillStep,
-             "bulk_encode": BulkEncodeStep}
+             "bulk_encode": BulkEncodeStep, "stack": StackStep}
 
 
 # -------------------------------------------------------------------- main --
@@ -438,6 +579,7 @@ def main():
     ap.add_argument("--workload", default="spark_down")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graphs", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -467,6 +609,30 @@ def main():
     torch.cuda.synchronize()
     dv.dvssq_device_error(clear=True)
 
+    # one CUDA graph per rotation slot: the timed region replays the same
+    # launches without the host in the loop
+    graphs = []
+    n_slots = getattr(work, "graph_slots", 0)
+    if n_slots and not args.no_graphs:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for slot in range(n_slots):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    work.step_slot(slot)
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(side)
+        for i in range(W):
+            graphs[i % n_slots].replay()
+        torch.cuda.synchronize()
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % n_slots].replay()
+        else:
+            work.step()
+
     def barrier():
         if world > 1:
             dist.barrier()
@@ -477,8 +643,8 @@ def main():
     barrier()
     with ClockSampler(local) as clk:
         start.record(stream)
-        for _ in range(args.steps):
-            work.step()
+        for i in range(args.steps):
+            timed_step(i)
         stop.record(stream)
         barrier()
     ms = start.elapsed_time(stop)
@@ -504,6 +670,7 @@ def main():
     dv.dvssq_profile_collect()
     dv.dvssq_profile_enable(False)
     prof = dv.dvssq_profile_read()
+    launches_measured = sum(c for c, _ in prof.values())
     pk, pk_kind = peaks()
     kernels = {}
     tot_ms = sum(v[1] for v in prof.values())
@@ -542,7 +709,7 @@ def main():
                     "traffic": dram_traffic(dom, args.workload),
                     "algorithmic_bytes_per_launch": db}
     # the decode GEMV's own roofline (the headline HBM-bound kernel)
-    dm = kernels.get("dec_main")
+    dm = kernels.get("dec_row") or kernels.get("dec_main")
 
     # end-to-end through the public API with pinned host buffers
     e2e = None
@@ -572,17 +739,19 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(work, "oracle_sample"):
         from oracle import dvssq_oracle as O
         nst, dt = run_oracle(work, O, synth)
-        cpu = {"value": round(bytes_step * nst / dt / 1e9, 4), "unit": "GB/s",
+        sample_bytes = getattr(work, "_oracle_bytes", None) or bytes_step
+        what = getattr(work, "oracle_what", "full step(s) of the same workload "
+                                            "(encode without SVD + 2 forwards)")
+        cpu = {"value": round(sample_bytes * nst / dt / 1e9, 4), "unit": "GB/s",
                "cores": threads_used(), "kind": "oracle",
-               "sample": f"{nst} full step(s) of the same workload (encode without SVD + "
-                         f"2 forwards) on the host, {dt:.1f} s"}
+               "sample": f"{nst} {what} on the host, {dt:.1f} s"}
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": W, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp16",
             "data": "synthetic (seeded N(0,0.02) weights with outlier columns, N(0,1) tokens)",
             "config": work.config(), "roofline": roofline, "kernels": kernels,
-            "decode_gemv": dm, "gpu_launches": work.launches_per_step() * args.steps,
+            "decode_gemv": dm, "gpu_launches": launches_measured,
             "e2e": e2e, "cpu_baseline": cpu, "device_error_word": err,
             "clocks": clk.summary()}
     if rank == 0:

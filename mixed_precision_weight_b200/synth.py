@@ -21,8 +21,8 @@ import numpy as np
 import torch
 
 __all__ = [
-    "weight", "act_scale", "activations", "lowrank_factors", "Workload",
-    "WORKLOADS", "layer_seed",
+    "weight", "weight_device", "act_scale", "activations", "lowrank_factors", "Workload",
+    "WORKLOADS", "layer_seed", "stack_rank",
 ]
 
 
@@ -43,6 +43,22 @@ def weight(M: int, K: int, seed: int, std: float = 0.02,
         cols = g.choice(K, size=n_outlier_cols, replace=False)
         w[:, cols] *= np.float32(outlier_scale)
     return _to_bf16(w)
+
+
+def weight_device(M: int, K: int, seed: int, device, std: float = 0.02,
+                  n_outlier_cols: int = 0, outlier_scale: float = 1.0) -> torch.Tensor:
+    """Like ``weight`` but drawn on ``device`` by torch's seeded generator.
+
+    For workloads too large to draw on the host in reasonable time (the
+    36-layer stack); the values differ from ``weight``'s for the same seed.
+    """
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    w = torch.randn((M, K), generator=g, device=device, dtype=torch.float32) * std
+    if n_outlier_cols:
+        cols = torch.randperm(K, generator=g, device=device)[:n_outlier_cols]
+        w[:, cols] *= outlier_scale
+    return w.to(torch.bfloat16)
 
 
 def act_scale(K: int, seed: int) -> torch.Tensor:
@@ -73,6 +89,12 @@ def lowrank_factors(M: int, K: int, r: int, seed: int, std: float = 0.01):
     U = g.standard_normal((M, r), dtype=np.float32) * np.float32(std)
     V = g.standard_normal((r, K), dtype=np.float32) * np.float32(std)
     return _to_bf16(U), _to_bf16(V)
+
+
+def stack_rank(layer: int) -> int:
+    """Residual rank of a layer of the 36-layer Spark stack: 24 on layers
+    14..28, 16 elsewhere."""
+    return 24 if 14 <= layer <= 28 else 16
 
 
 def layer_seed(base: int, layer: int, which: int) -> int:
