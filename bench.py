@@ -351,9 +351,14 @@ class PrefillStep:
     def kernel_work(self, name):
         if name == "pre_gemm":
             return self.work_per_step()
+        salp = (self.n + 63) // 64 * 64
+        kc = self.K + salp + 64
         if name == "pre_act":
-            salp = (self.n + 63) // 64 * 64
-            return self.T * self.K * 2 + self.T * (self.K + salp + 64) * 2
+            # x read + Xc written
+            return self.T * self.K * 2 + self.T * kc * 2
+        if name == "pre_mat":
+            # packed layer read + materialised A written
+            return packed_bytes(self.M, self.K, self.r, self.n) + self.M * kc * 2
         return None
 
     def launches_per_step(self):

@@ -10,14 +10,15 @@
 // pre_act   one CTA per 16 tokens builds Xc in FP16: fp32 Kronecker FWHT of
 //           each Hadamard block, the salient gather, and t = V xr with
 //           mma.sync (fp32 accumulation over all blocks).
-// pre_gemm  CTA tile 128 rows x BN tokens.  Warp 0 streams Xc tiles by TMA
-//           (128B swizzle); warps 2-5 dequantise the packed weights of the
-//           stage straight into the UMMA K-major 128B-swizzled layout (q4 . s4
-//           is exact in FP16 for scales in [2^-17, 8188]; q8 . s8 and U are
-//           rounded once); warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into
-//           a TMEM accumulator and commits each stage back to its producers;
-//           warps 2-5 then read TMEM (tcgen05.ld) and write y.  No TMA
-//           multicast is used anywhere.
+// pre_mat   materialises A in FP16 once per call (the GPU counterpart of the
+//           Spark card's materialize_weights), alongside pre_act: q4 . s4 is
+//           exact in FP16 for scales in [2^-17, 8188]; q8 . s8 and U are
+//           rounded once.
+// pre_gemm  CTA tile 128 rows x BN tokens.  Warp 0 streams the A and Xc
+//           tiles of each K stage by TMA (128B swizzle, no multicast); warp 1
+//           issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator and
+//           commits each stage back to the producer; warps 2-5 read TMEM
+//           (tcgen05.ld) and write y.
 #include "common.cuh"
 #include "fwht_group.cuh"
 #include "kernels.h"
@@ -43,6 +44,7 @@ struct PrefillParams {
   void *y;
   int y_bf16;
   __half *xc;      // [T][Kc]
+  __half *a;       // [M][Kc]
 };
 
 // ------------------------------------------------------------------ pre_act
@@ -54,7 +56,7 @@ static size_t pre_act_smem_bytes(int B, int rank, int n_sal) {
 }
 
 template <int B>
-__global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
+__device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int blk) {
   constexpr int P = B / 16;
   constexpr int NW = B / 32;
   __shared__ float scratch[16][GroupScratch<B>::kElems];
@@ -67,7 +69,7 @@ __global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
                                       (size_t)p.rank * (B + 8) * 2);
 
   const int tid = threadIdx.x, tok = tid / P, t = tid % P;
-  const int t0 = blockIdx.x * 16, gt = t0 + tok;
+  const int t0 = blk * 16, gt = t0 + tok;
   const bool live = gt < p.T;
   const int nkb = p.K / B;
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
@@ -77,11 +79,46 @@ __global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
   float tacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
   const int ntiles = (p.rank + 7) / 8;
 
+  // the next block's x (registers) and V rows (registers, stored to vh at the
+  // top of its iteration) are loaded one block ahead, so that their latency
+  // overlaps the current block's work
+  constexpr int VPT = 64 * (B / 8) / B;          // uint4 of V per thread (rank <= 64)
+  uint16_t xn[16];
+  uint4 vn[VPT];
+  auto fetch = [&](int kb) {
+#pragma unroll
+    for (int a = 0; a < 16; ++a)
+      xn[a] = live ? p.x[(size_t)gt * p.K + (size_t)kb * B + P * a + t] : (uint16_t)0;
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int i = tid + u * B;
+      const int rr = i / (B / 8), cc = i % (B / 8);
+      vn[u] = rr < p.rank
+                  ? *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + (size_t)kb * B + cc * 8)
+                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  fetch(0);
   for (int kb = 0; kb < nkb; ++kb) {
     float v[16];
 #pragma unroll
-    for (int a = 0; a < 16; ++a)
-      v[a] = live ? bf16_bits_to_f32(p.x[(size_t)gt * p.K + (size_t)kb * B + P * a + t]) : 0.0f;
+    for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f32(xn[a]);
+    // V block as FP16 (vh is free: the previous iteration ended with a barrier)
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+      const int i = tid + u * B;
+      const int rr = i / (B / 8), cc = i % (B / 8);
+      if (rr < p.rank) {
+        const uint32_t wv[4] = {vn[u].x, vn[u].y, vn[u].z, vn[u].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = pack_half2(__float2half_rn(bf16_bits_to_f32(wv[q] & 0xFFFFu)),
+                            __float2half_rn(bf16_bits_to_f32(wv[q] >> 16)));
+        *reinterpret_cast<uint4 *>(&vh[rr][cc * 8]) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    if (kb + 1 < nkb) fetch(kb + 1);
     fwht_group<B>(v, scratch[tok], t);
     uint32_t h[8];
 #pragma unroll
@@ -97,19 +134,6 @@ __global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
       uint4 *dst = reinterpret_cast<uint4 *>(p.xc + (size_t)gt * p.Kc + (size_t)kb * B + 16 * t);
       dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
       dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-    }
-    // V block as FP16
-    for (int i = tid; i < p.rank * (B / 8); i += B) {
-      const int rr = i / (B / 8), cc = i % (B / 8);
-      const uint4 raw =
-          *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + (size_t)kb * B + cc * 8);
-      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        o[u] = pack_half2(__float2half_rn(bf16_bits_to_f32(wv[u] & 0xFFFFu)),
-                          __float2half_rn(bf16_bits_to_f32(wv[u] >> 16)));
-      *reinterpret_cast<uint4 *>(&vh[rr][cc * 8]) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     __syncthreads();
     // salient gather: entries whose column lies in this block (sal_idx sorted)
@@ -176,18 +200,7 @@ __global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
   }
 }
 
-// ----------------------------------------------------------------- pre_gemm
-// One producer thread per tile row writes the 64 FP16 operands of a stage as
-// eight 16-byte chunks in the 128B-swizzled K-major layout.
-__device__ __forceinline__ void store_row_sw128(uint8_t *stage, int row, const uint32_t h[32]) {
-  uint8_t *rp = stage + row * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 v = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
-    *reinterpret_cast<uint4 *>(rp + ((c ^ (row & 7)) << 4)) = v;
-  }
-}
-
+// ------------------------------------------------------------------ pre_mat
 // 8 nibbles (two's complement) of word w times scale s -> 4 FP16 pairs in
 // column order (n0,n1), (n2,n3), (n4,n5), (n6,n7); exact for FP16-safe s.
 __device__ __forceinline__ void dequant_q4_scaled(uint32_t w, __half2 s2, uint32_t out[4]) {
@@ -212,9 +225,73 @@ __device__ __forceinline__ void dequant_q4_scaled(uint32_t w, __half2 s2, uint32
   out[3] = __byte_perm(c, d, 0x7632);   // (n6, n7)
 }
 
+// A[m][8 c .. 8 c + 7] for one (row, 8-column chunk) per thread, so that a
+// warp writes 512 contiguous bytes: chunks of the first K/8 columns are
+// q4 . s4, then q8 . s8 (n_sal padded to 64), then U (padded to 64 columns).
+__device__ __forceinline__ void pre_mat_item(const PrefillParams &p, const long long item) {
+  const int nc = p.Kc / 8;
+  if (item >= (long long)p.M * nc) return;
+  const int m = (int)(item / nc), ci = (int)(item - (long long)m * nc);
+  const int kq = p.K / 8, ks = p.salp / 8;
+  uint32_t h[4];
+  if (ci < kq) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(p.q4 + (size_t)m * (p.K / 2)) + ci);
+    const __half sh = __float2half_rn(bf16_bits_to_f32(p.s4[(size_t)m * (p.K / 64) + ci / 8]));
+    dequant_q4_scaled(w, __halves2half2(sh, sh), h);
+  } else if (ci < kq + ks) {
+    const int e0 = 8 * (ci - kq);
+    const float s8f = bf16_bits_to_f32(p.s8[m]);
+    uint2 raw = make_uint2(0u, 0u);
+    if (e0 < p.n_sal)
+      raw = __ldg(reinterpret_cast<const uint2 *>(p.q8 + (size_t)m * p.n_sal + e0));
+    const uint32_t wv[2] = {raw.x, raw.y};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t w = wv[u];
+      const float f0 = (float)(int8_t)(w & 0xFF) * s8f, f1 = (float)(int8_t)((w >> 8) & 0xFF) * s8f;
+      const float f2 = (float)(int8_t)((w >> 16) & 0xFF) * s8f, f3 = (float)(int8_t)(w >> 24) * s8f;
+      h[2 * u] = pack_half2(__float2half_rn(f0), __float2half_rn(f1));
+      h[2 * u + 1] = pack_half2(__float2half_rn(f2), __float2half_rn(f3));
+    }
+  } else {
+    const int r0 = 8 * (ci - kq - ks);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ra = r0 + 2 * j, rb = ra + 1;
+      const float u0 = ra < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + ra]) : 0.0f;
+      const float u1 = rb < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + rb]) : 0.0f;
+      h[j] = pack_half2(__float2half_rn(u0), __float2half_rn(u1));
+    }
+  }
+  *reinterpret_cast<uint4 *>(p.a + (size_t)m * p.Kc + 8 * ci) = make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// pre_act (one CTA per 16 tokens) lets pre_mat launch at once (programmatic
+// dependent launch), so the bandwidth-bound materialisation fills the SMs the
+// latency-bound activation pass leaves idle.  pre_mat reads only the packed
+// weights; it waits for pre_act only before it exits, so that its completion
+// (which orders the GEMM) implies pre_act's.
+template <int B>
+__global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
+  pdl_launch_dependents();
+  pre_act_block<B>(p, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(256) pre_mat_kernel(PrefillParams p, long long items) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < items;
+       i += (long long)gridDim.x * blockDim.x)
+    pre_mat_item(p, i);
+  pdl_wait();
+}
+
+// ----------------------------------------------------------------- pre_gemm
+// Persistent: one CTA per SM walks output tiles (row tile fastest).  TMEM
+// holds two accumulators of BN columns: the MMA warp fills one while the
+// epilogue warps drain the other (acc_full / acc_empty barriers).
 template <int BN>
 __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
-    const __grid_constant__ CUtensorMap mxc, PrefillParams p) {
+    const __grid_constant__ CUtensorMap ma, const __grid_constant__ CUtensorMap mxc,
+    PrefillParams p, int nmt, int ntiles) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int A_STAGE = kPreBM * 128;
@@ -223,23 +300,26 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
   uint8_t *sb = base + kPreStages * A_STAGE;
   uint64_t *full = reinterpret_cast<uint64_t *>(sb + kPreStages * B_STAGE);
   uint64_t *empty = full + kPreStages;
-  uint64_t *accum = empty + kPreStages;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+  uint64_t *acc_full = empty + kPreStages;       // [2]
+  uint64_t *acc_empty = acc_full + 2;            // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * kPreBM, n0 = blockIdx.y * BN;
   const int S = p.nstages;
 
   if (tid == 0) {
     for (int s = 0; s < kPreStages; ++s) {
-      mbar_init(&full[s], 129);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -249,108 +329,64 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
   bool ok = true;
 
   if (warp == 0) {
-    // ---------------- activation operand producer (TMA) ----------------
+    // ---------------- operand producer (TMA: weights and activations) ----------------
     if (lane == 0) {
+      prefetch_tensormap(&ma);
       prefetch_tensormap(&mxc);
-      for (int s = 0; s < S && ok; ++s) {
-        const int slot = s % kPreStages, round = s / kPreStages;
-        if (!mbar_wait(&empty[slot], (round & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[slot], B_STAGE);
-        tma_load_2d(sb + slot * B_STAGE, &mxc, 64 * s, n0, &full[slot]);
+      long long gs = 0;                           // stage counter over all tiles
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % nmt) * kPreBM, n0 = (tile / nmt) * BN;
+        for (int s = 0; s < S && ok; ++s, ++gs) {
+          const int slot = (int)(gs % kPreStages);
+          const uint32_t round = (uint32_t)(gs / kPreStages);
+          if (!mbar_wait(&empty[slot], (round & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[slot], A_STAGE + B_STAGE);
+          tma_load_2d(sa + slot * A_STAGE, &ma, 64 * s, m0, &full[slot]);
+          tma_load_2d(sb + slot * B_STAGE, &mxc, 64 * s, n0, &full[slot]);
+        }
       }
     }
   } else if (warp == 1) {
     // ---------------------------- MMA issuer -----------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_f16(kPreBM, BN);
-      for (int s = 0; s < S && ok; ++s) {
-        const int slot = s % kPreStages, round = s / kPreStages;
-        if (!mbar_wait(&full[slot], round & 1)) { ok = false; break; }
+      long long gs = 0;
+      int li = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++li) {
+        const int ab = li & 1;
+        if (!mbar_wait(&acc_empty[ab], ((li >> 1) & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sa + slot * A_STAGE), b0 = smem_u32(sb + slot * B_STAGE);
+        const uint32_t acc = tmem + (uint32_t)(ab * BN);
+        for (int s = 0; s < S && ok; ++s, ++gs) {
+          const int slot = (int)(gs % kPreStages);
+          const uint32_t round = (uint32_t)(gs / kPreStages);
+          if (!mbar_wait(&full[slot], round & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sa + slot * A_STAGE), b0 = smem_u32(sb + slot * B_STAGE);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_f16(tmem, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k), idesc,
-                     (s > 0 || k > 0) ? 1u : 0u);
-        tc_commit(&empty[slot]);
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16(acc, umma_desc_sw128(a0 + 32 * k), umma_desc_sw128(b0 + 32 * k), idesc,
+                       (s > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&empty[slot]);
+        }
+        tc_commit(&acc_full[ab]);
       }
-      tc_commit(accum);
     }
   } else {
-    // ------------- weight operand producers, then the epilogue -------------
-    const int i = tid - 64;              // tile row 0..127
-    const int m = m0 + i;
-    const bool rowok = m < p.M;
-    const int KG = p.K / 64;
-    uint4 cur0 = make_uint4(0, 0, 0, 0), cur1 = cur0;
-    uint16_t cur_s = 0;
-    auto load_q4 = [&](int s, uint4 &w0, uint4 &w1, uint16_t &sc) {
-      if (rowok && s < p.nq4) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.q4 + (size_t)m * (p.K / 2) + 32 * s);
-        w0 = __ldg(src);
-        w1 = __ldg(src + 1);
-        sc = p.s4[(size_t)m * KG + s];
-      }
-    };
-    load_q4(0, cur0, cur1, cur_s);
-    const float s8f = rowok && p.n_sal > 0 ? bf16_bits_to_f32(p.s8[m]) : 0.0f;
-    for (int s = 0; s < S && ok; ++s) {
-      const int slot = s % kPreStages, round = s / kPreStages;
-      uint4 nx0 = make_uint4(0, 0, 0, 0), nx1 = nx0;
-      uint16_t nx_s = 0;
-      load_q4(s + 1, nx0, nx1, nx_s);
-      uint32_t h[32];
-      if (!rowok) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) h[j] = 0u;
-      } else if (s < p.nq4) {
-        const __half sh = __float2half_rn(bf16_bits_to_f32(cur_s));
-        const __half2 s2 = __halves2half2(sh, sh);
-        const uint32_t wv[8] = {cur0.x, cur0.y, cur0.z, cur0.w, cur1.x, cur1.y, cur1.z, cur1.w};
-#pragma unroll
-        for (int q = 0; q < 8; ++q) dequant_q4_scaled(wv[q], s2, h + 4 * q);
-      } else if (s < p.nq4 + p.nsal) {
-        const int e0 = 64 * (s - p.nq4);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 raw = make_uint4(0, 0, 0, 0);
-          if (e0 + 16 * q < p.n_sal)
-            raw = __ldg(reinterpret_cast<const uint4 *>(p.q8 + (size_t)m * p.n_sal + e0 + 16 * q));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t w = wv[u];
-            const float f0 = (float)(int8_t)(w & 0xFF) * s8f, f1 = (float)(int8_t)((w >> 8) & 0xFF) * s8f;
-            const float f2 = (float)(int8_t)((w >> 16) & 0xFF) * s8f, f3 = (float)(int8_t)(w >> 24) * s8f;
-            h[8 * q + 2 * u] = pack_half2(__float2half_rn(f0), __float2half_rn(f1));
-            h[8 * q + 2 * u + 1] = pack_half2(__float2half_rn(f2), __float2half_rn(f3));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r0 = 2 * j, r1 = 2 * j + 1;
-          const float u0 = r0 < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + r0]) : 0.0f;
-          const float u1 = r1 < p.rank ? bf16_bits_to_f32(p.U[(size_t)m * p.rank + r1]) : 0.0f;
-          h[j] = pack_half2(__float2half_rn(u0), __float2half_rn(u1));
-        }
-      }
-      if (!mbar_wait(&empty[slot], (round & 1) ^ 1)) { ok = false; break; }
-      store_row_sw128(sa + slot * A_STAGE, i, h);
-      fence_proxy_async_smem();
-      mbar_arrive(&full[slot]);
-      cur0 = nx0; cur1 = nx1; cur_s = nx_s;
-    }
     // ------------------------------ epilogue ------------------------------
-    if (ok && mbar_wait(accum, 0)) {
+    const int quarter = warp & 3;
+    int li = 0;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++li) {
+      const int ab = li & 1;
+      const int m0 = (tile % nmt) * kPreBM, n0 = (tile / nmt) * BN;
+      if (!mbar_wait(&acc_full[ab], (li >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      const int quarter = warp & 3;
       const int row = m0 + 32 * quarter + lane;
       const float bv = (p.bias != nullptr && row < p.M) ? bf16_bits_to_f32(p.bias[row]) : 0.0f;
 #pragma unroll 1
       for (int c = 0; c < BN / 16; ++c) {
         uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + 16 * c, r);
+        tmem_ld16(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(ab * BN) + 16 * c, r);
         tmem_ld_wait();
         if (row < p.M) {
 #pragma unroll
@@ -366,13 +402,16 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
           }
         }
       }
+      // this accumulator may be overwritten by the tile after next
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -380,14 +419,15 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
 static int pre_bn(int T) { return T > 128 ? 256 : (T > 64 ? 128 : 64); }
 
 static size_t pre_smem_bytes(int BN) {
-  return 1024 + (size_t)kPreStages * (kPreBM * 128 + BN * 128) + 256;
+  return 1024 + (size_t)kPreStages * (kPreBM * 128 + BN * 128) + 256;   // + barriers, TMEM slot
 }
 
 size_t prefill_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T) {
-  (void)M; (void)block; (void)rank;
+  (void)block; (void)rank;
   const int salp = (n_sal + 63) / 64 * 64;
   const size_t Kc = (size_t)K + salp + 64;
-  return ((size_t)T * Kc * 2 + 255) & ~(size_t)255;
+  // Xc [T][Kc] and the materialised A [M][Kc], FP16
+  return (((size_t)T * Kc * 2 + 255) & ~(size_t)255) + (((size_t)M * Kc * 2 + 255) & ~(size_t)255);
 }
 
 cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
@@ -402,28 +442,44 @@ cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   p.q4 = a.q4; p.s4 = a.s4; p.sal_idx = a.sal_idx; p.q8 = a.q8; p.s8 = a.s8;
   p.U = a.U; p.V = a.V; p.x = a.x; p.bias = a.bias; p.y = a.y; p.y_bf16 = a.y_bf16;
   p.xc = reinterpret_cast<__half *>(a.workspace);
+  p.a = reinterpret_cast<__half *>(static_cast<char *>(a.workspace) +
+                                   (((size_t)a.T * p.Kc * 2 + 255) & ~(size_t)255));
 
   const size_t act_smem = pre_act_smem_bytes(a.block, a.rank, a.n_sal);
   cudaError_t e;
-  dim3 ga((a.T + 15) / 16);
+  const dim3 ga((a.T + 15) / 16);
   if (a.block == 256)
     e = L.launch("pre_act", pre_act_kernel<256>, ga, dim3(256), act_smem, st, false, p);
   else
     e = L.launch("pre_act", pre_act_kernel<128>, ga, dim3(128), act_smem, st, false, p);
   if (e != cudaSuccess) return e;
+  const long long items = (long long)a.M * (p.Kc / 8);
+  const long long mat_blocks = std::min<long long>((items + 255) / 256, (long long)sm_count() * 8);
+  e = L.launch("pre_mat", pre_mat_kernel, dim3((unsigned)mat_blocks), dim3(256), 0, st, true, p,
+               items);
+  if (e != cudaSuccess) return e;
 
-  CUtensorMap mxc;
+
+  CUtensorMap mxc, ma;
   const int BN = pre_bn(a.T);
   if (encode_tmap_2d(&mxc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.xc, (uint64_t)p.Kc, (uint64_t)a.T,
                      (uint64_t)p.Kc * 2, 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  dim3 gg((a.M + kPreBM - 1) / kPreBM, (a.T + BN - 1) / BN);
+  if (encode_tmap_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.a, (uint64_t)p.Kc, (uint64_t)a.M,
+                     (uint64_t)p.Kc * 2, 64, kPreBM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int nmt = (a.M + kPreBM - 1) / kPreBM;
+  const int ntiles = nmt * ((a.T + BN - 1) / BN);
+  const dim3 gg((unsigned)std::min(ntiles, sm_count()));
   const size_t smem = pre_smem_bytes(BN);
   if (BN == 256)
-    return L.launch("pre_gemm", pre_gemm_kernel<256>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
+    return L.launch("pre_gemm", pre_gemm_kernel<256>, gg, dim3(kPreThreads), smem, st, false, ma,
+                    mxc, p, nmt, ntiles);
   if (BN == 128)
-    return L.launch("pre_gemm", pre_gemm_kernel<128>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
-  return L.launch("pre_gemm", pre_gemm_kernel<64>, gg, dim3(kPreThreads), smem, st, false, mxc, p);
+    return L.launch("pre_gemm", pre_gemm_kernel<128>, gg, dim3(kPreThreads), smem, st, false, ma,
+                    mxc, p, nmt, ntiles);
+  return L.launch("pre_gemm", pre_gemm_kernel<64>, gg, dim3(kPreThreads), smem, st, false, ma, mxc,
+                  p, nmt, ntiles);
 }
 
 cudaError_t prepare_prefill_kernels() {
