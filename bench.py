@@ -213,7 +213,7 @@ class SparkDownStep:
         return encode_bytes(self.M, self.K, self.n) + 2 * packed_bytes(self.M, self.K, self.r, self.n)
 
     def launches_per_step(self):
-        return 4 + 2 + 2
+        return 3 + 2 + 2
 
     def config(self):
         return {"workload": self.name, "M": self.M, "K": self.K, "block": 256, "rank": self.r,
@@ -410,7 +410,7 @@ class BulkEncodeStep:
         return 36 * (2 * encode_bytes(I, H, H // 8) + encode_bytes(H, I, I // 8))
 
     def launches_per_step(self):
-        return 108 * 5
+        return 108 * 3
 
     def kernel_work(self, name):
         H, I = self.H, self.I
@@ -436,6 +436,7 @@ class StackStep:
 
     name = "spark_mlp_stack_36x(gate,up,down)_T1"
     graph_slots = 1
+    fused = True      # one cooperative launch per token (dvssq_mlp_stack_forward)
 
     def __init__(self, dv, synth, torch, rank_id, device):
         self.dv, self.torch, self.device = dv, torch, device
@@ -465,6 +466,7 @@ class StackStep:
         del self.ws_enc
         fw = max(dv.dvssq_forward_workspace_size(sh, 1) for mats in self.layers for sh, _ in mats)
         self.ws = torch.empty(fw, dtype=torch.uint8, device=device)
+        self.mstack = dv.MlpStack(self.layers, device=device) if self.fused else None
         self.x0 = synth.activations(1, H, seed=3 + rank_id, n_outlier=13,
                                     outlier_scale=25.0).to(device)
         self.x = torch.empty((1, H), dtype=torch.bfloat16, device=device)
@@ -474,6 +476,9 @@ class StackStep:
 
     def run(self, x, out):
         dv = self.dv
+        if self.fused:
+            self.mstack.forward(x, y=out)
+            return
         cur = x
         for l, ((sg, pg), (su, pu), (sd, pd)) in enumerate(self.layers):
             dv.dvssq_linear_forward(sg, pg, cur, y=self.g, y_dtype=dv.Y_BF16, workspace=self.ws)
@@ -493,9 +498,11 @@ class StackStep:
                    for sh, _ in mats)
 
     def launches_per_step(self):
-        return 36 * (3 * 2 + 1)
+        return 1 if self.fused else 36 * (3 * 2 + 1)
 
     def kernel_work(self, name):
+        if name == "mlp_stack":
+            return self.bytes_per_step()
         # average algorithmic bytes per launch over the stack's launches
         shapes = [sh for mats in self.layers for sh, _ in mats]
         per = [kernel_bytes(name, sh.M, sh.K, sh.rank, sh.n_sal, 1) for sh in shapes]
@@ -509,8 +516,10 @@ class StackStep:
         return {"workload": self.name, "layers": 36, "hidden": self.H, "intermediate": self.I,
                 "block": 256, "rank": "16 (layers 0-13, 29-35), 24 (14-28)",
                 "n_sal": "K/8 per matrix", "tokens": 1,
-                "step": "36 x (dvssq_linear_forward gate, up -> dvssq_gelu_mul -> down), "
-                        "BF16 hidden states, one CUDA graph per token",
+                "step": ("dvssq_mlp_stack_forward: the 36 blocks in one cooperative launch"
+                         if self.fused else
+                         "36 x (dvssq_linear_forward gate, up -> dvssq_gelu_mul -> down)")
+                        + ", BF16 hidden states, one CUDA graph per token",
                 "packed_bytes_per_token": self.bytes_per_step(),
                 "l2": "1.9 GB of packed weights per token > 126 MB L2",
                 "lowrank_factors": "seeded synthetic U, V (values do not change the work)",
@@ -549,8 +558,14 @@ class StackStep:
         return step
 
 
+class StackChainStep(StackStep):
+    """The same stack as 108 single-layer forwards and 36 gelu_mul launches."""
+    name = "spark_mlp_stack_36x(gate,up,down)_T1_chain"
+    fused = False
+
+
 WORKLOADS = {"spark_down": SparkDownStep, "decode": DecodeStep, "prefill": PrefillStep,
-             "bulk_encode": BulkEncodeStep, "stack": StackStep}
+             "bulk_encode": BulkEncodeStep, "stack": StackStep, "stack_chain": StackChainStep}
 
 
 # -------------------------------------------------------------------- main --
@@ -714,7 +729,7 @@ def main():
                     "traffic": dram_traffic(dom, args.workload),
                     "algorithmic_bytes_per_launch": db}
     # the decode GEMV's own roofline (the headline HBM-bound kernel)
-    dm = kernels.get("dec_row") or kernels.get("dec_main")
+    dm = kernels.get("dec_row") or kernels.get("dec_main") or kernels.get("mlp_stack")
 
     # end-to-end through the public API with pinned host buffers
     e2e = None

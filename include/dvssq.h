@@ -167,8 +167,9 @@ DVSSQ_API dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, siz
  *   1. W_rot = W . H_K in fp64; each +-1 sum is exact whenever
  *      inexact_rotation_blocks is 0, the scale 1/sqrt(b) is applied once.
  *   2. score_j = act_scale_j * sqrt(sum_i W_rot[i,j]^2); the sum runs over
- *      rows in chunks of 64 (within a chunk acc = acc + w*w, each operation
- *      rounded), chunk partials added in ascending order.
+ *      rows in chunks of 16 (within a chunk acc = acc + w*w, each operation
+ *      rounded), the chunk sums in groups of 8 consecutive chunks (each group
+ *      summed from 0 in ascending order), the group sums in ascending order.
  *   3. sal_idx = the n_sal largest scores, ties to the lower index, sorted.
  *   4. INT8 tier per row: s8 = bf16_rn(max_{j in sal} |W_rot| / 127),
  *      q8 = clip(rint(w / s8), -128, 127)  (division as w * (1/s8)).
@@ -245,6 +246,52 @@ DVSSQ_API dvssq_status dvssq_linear_forward_static(const dvssq_shape *shape,
                                                    const dvssq_weights *w, const void *x,
                                                    int64_t T, const void *bias, void *y,
                                                    int32_t y_dtype, void *stream);
+
+/* One layer of a stack of gated-GELU MLP blocks ("Myric/Spark-X2.5-4B-GGUF",
+ * "The model": GELU FFN; "Spark-X2.5-4B-ASHQ1-GGUF", "Architecture":
+ * ffn_gate / ffn_up / ffn_down), each projection in packed DV-SSQ form:
+ * shape[0] / w[0] = gate (M = inter, K = hidden), shape[1] / w[1] = up (same
+ * shape), shape[2] / w[2] = down (M = hidden, K = inter).  Host struct of
+ * device pointers, read only.                                              */
+typedef struct {
+  dvssq_shape shape[3];
+  dvssq_weights w[3];
+} dvssq_mlp_layer;
+
+/* Bytes of workspace the MLP-stack calls need for these layers (host only).
+ * Supported stacks: every gate/up is inter x hidden and every down hidden x
+ * inter with one Hadamard block size; hidden and inter multiples of 512;
+ * n_sal a multiple of 32; rank a multiple of 8 and at most 32.  Others
+ * return UNSUPPORTED_SHAPE.                                                */
+DVSSQ_API dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers,
+                                                      int32_t n_layers, size_t *bytes);
+
+/* Prepares `workspace` for dvssq_mlp_stack_forward on these layers: writes
+ * the device table of the layers and, per matrix, (V H_K) in FP32 (the
+ * blockwise FWHT of each row of V; H is symmetric).  Synchronises `stream`.
+ * Call again whenever a layer's pointers or V change.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_mlp_stack_prepare(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                               void *workspace, size_t workspace_bytes,
+                                               void *stream);
+
+/* One token through the whole stack, in one cooperative launch:
+ *   for each layer:  g = RN_bf16(gate(x)), u = RN_bf16(up(x)),
+ *                    h = RN_bf16(gelu(g) u)  (as dvssq_gelu_mul),
+ *                    x = RN_bf16(down(h));
+ *   y = x after the last layer.
+ * Each projection is the dvssq_linear_forward equation without bias, with
+ * the rank-r input t = V (H x) formed as (V H) x.  Rows are computed as exact
+ * int32 dot products of the codes with int16 activations (one scale per 64
+ * rotated columns, one per 32 salient entries), scaled in FP32.
+ *   layers, n_layers  as given to dvssq_mlp_stack_prepare for `workspace`
+ *   x  bf16 [hidden] (device);  y  bf16 [hidden] (device; may alias x)
+ * Stream-ordered and asynchronous.  A wait that runs out sets the device
+ * error word (dvssq_device_error) and the call's output is then undefined.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_mlp_stack_forward(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                               const void *x, void *y, void *workspace,
+                                               size_t workspace_bytes, void *stream);
 
 /* Reads (and clears when `clear` != 0) the device error word of the current
  * device; synchronises the device.  0 means no kernel gave up a wait.     */

@@ -9,8 +9,10 @@ is no CPU or PyTorch fallback: if the library is missing this import fails.
 Functions keep the C names (see include/dvssq.h):
     dvssq_fwht, dvssq_encode_workspace_size, dvssq_encode,
     dvssq_forward_workspace_size, dvssq_linear_forward, dvssq_device_error,
-    dvssq_profile_* .
-``DvssqLinear`` bundles one encoded layer with its workspaces.
+    dvssq_mlp_stack_workspace_size, dvssq_mlp_stack_prepare,
+    dvssq_mlp_stack_forward, dvssq_profile_* .
+``DvssqLinear`` bundles one encoded layer with its workspaces; ``MlpStack``
+bundles a stack of gated-GELU MLP blocks with its prepared workspace.
 """
 from __future__ import annotations
 
@@ -24,7 +26,8 @@ __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
     "dvssq_fwht", "dvssq_gelu_mul", "dvssq_encode_workspace_size", "dvssq_encode",
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
-    "dvssq_device_error", "STATIC_SCRATCH_BYTES",
+    "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
+    "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
     "dvssq_profile_reset", "Y_F32", "Y_BF16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
     "EXPORTED_SYMBOLS",
@@ -48,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "dvssq_gelu_mul",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
     "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_device_error",
+    "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
     "dvssq_profile_reset",
@@ -71,6 +75,10 @@ class _Weights(ctypes.Structure):
     _fields_ = [("q4", ctypes.c_void_p), ("s4", ctypes.c_void_p), ("sal_idx", ctypes.c_void_p),
                 ("q8", ctypes.c_void_p), ("s8", ctypes.c_void_p), ("U", ctypes.c_void_p),
                 ("V", ctypes.c_void_p)]
+
+
+class _MlpLayer(ctypes.Structure):
+    _fields_ = [("shape", Shape * 3), ("w", _Weights * 3)]
 
 
 class _EncodeInfo(ctypes.Structure):
@@ -97,6 +105,12 @@ _sig = {
     "dvssq_linear_forward_static": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights),
                                                    _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "dvssq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
+    "dvssq_mlp_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32,
+                                                      ctypes.POINTER(ctypes.c_size_t)]),
+    "dvssq_mlp_stack_prepare": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32, _P,
+                                               ctypes.c_size_t, _P]),
+    "dvssq_mlp_stack_forward": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32, _P, _P,
+                                               _P, ctypes.c_size_t, _P]),
     "dvssq_profile_enable": (ctypes.c_int, [ctypes.c_int32]),
     "dvssq_profile_collect": (ctypes.c_int, []),
     "dvssq_profile_count": (ctypes.c_int32, []),
@@ -271,6 +285,59 @@ def dvssq_linear_forward_static(shape: Shape, w: PackedWeights, x: torch.Tensor,
 
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def _mlp_layers(layers) -> ctypes.Array:
+    """[(gate, up, down)] of (Shape, PackedWeights) -> the C array of dvssq_mlp_layer."""
+    arr = (_MlpLayer * len(layers))()
+    for l, mats in enumerate(layers):
+        if len(mats) != 3:
+            raise ValueError("each layer is (gate, up, down)")
+        for mi, (shape, packed) in enumerate(mats):
+            arr[l].shape[mi] = shape
+            arr[l].w[mi] = packed._c(shape)
+    return arr
+
+
+def dvssq_mlp_stack_workspace_size(layers) -> int:
+    arr = _mlp_layers(layers)
+    n = ctypes.c_size_t(0)
+    _check(lib.dvssq_mlp_stack_workspace_size(arr, len(layers), ctypes.byref(n)),
+           "dvssq_mlp_stack_workspace_size")
+    return n.value
+
+
+def dvssq_mlp_stack_prepare(layers, workspace: torch.Tensor, stream=None):
+    arr = _mlp_layers(layers)
+    _check(lib.dvssq_mlp_stack_prepare(arr, len(layers), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "dvssq_mlp_stack_prepare")
+
+
+def dvssq_mlp_stack_forward(layers, x: torch.Tensor, workspace: torch.Tensor,
+                            y: torch.Tensor | None = None, stream=None, _arr=None):
+    """y = one BF16 token [hidden] through the prepared stack."""
+    arr = _mlp_layers(layers) if _arr is None else _arr
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib.dvssq_mlp_stack_forward(arr, len(layers), _ptr(x), _ptr(y), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "dvssq_mlp_stack_forward")
+    return y
+
+
+class MlpStack:
+    """A stack of gated-GELU MLP blocks with its prepared workspace."""
+
+    def __init__(self, layers, device="cuda", stream=None):
+        self.layers = [tuple(m) for m in layers]
+        self._arr = _mlp_layers(self.layers)
+        self.workspace = torch.empty(dvssq_mlp_stack_workspace_size(self.layers),
+                                     dtype=torch.uint8, device=device)
+        dvssq_mlp_stack_prepare(self.layers, self.workspace, stream=stream)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
+        return dvssq_mlp_stack_forward(self.layers, x, self.workspace, y=y, stream=stream,
+                                       _arr=self._arr)
 
 
 def dvssq_device_error(clear: bool = True) -> int:

@@ -20,6 +20,7 @@ enum DeviceError : uint32_t {
   kErrWaitMbarrier = 1u << 0,   // an mbarrier wait ran out
   kErrWaitTmem = 1u << 1,       // a TMEM accumulator wait ran out
   kErrBadShape = 1u << 2,       // a kernel saw a shape it does not support
+  kErrWaitGrid = 1u << 3,       // a grid-wide barrier wait ran out
 };
 
 // Device error word of the library (one translation unit: see libdvssq.cu).
@@ -82,6 +83,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn_bits(float f) {
 // --------------------------------------------------------- smem addresses -
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// gelu(v) = v/2 (1 + erf(v / sqrt 2)) in FP32.  1 + erf(z) = erfc(-z): the
+// complementary form keeps its relative accuracy for negative v, where
+// 1 + erf would cancel.
+__device__ __forceinline__ float gelu_erf(float v) {
+  return 0.5f * v * erfcf(-v * 0.70710678118654752f);
 }
 
 // --------------------------------------------------------------- mbarrier -

@@ -79,6 +79,7 @@ dvssq_status ensure_device() {
   }
   if ((e = prepare_encode_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_forward_kernels()) != cudaSuccess) return cuda_fail(e);
+  if ((e = prepare_stack_kernels()) != cudaSuccess) return cuda_fail(e);
   ready[dev] = 1;
   return DVSSQ_OK;
 }
@@ -190,7 +191,7 @@ dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes
   dvssq_status s = check_shape(shape);
   if (s != DVSSQ_OK) return s;
   if (bytes == nullptr) return DVSSQ_ERR_INVALID_ARG;
-  *bytes = encode_workspace_bytes(shape->M, shape->K, shape->n_sal);
+  *bytes = encode_workspace_bytes(shape->M, shape->K, shape->block, shape->n_sal);
   return DVSSQ_OK;
 }
 
@@ -208,7 +209,8 @@ dvssq_status dvssq_encode(const dvssq_shape *shape, const void *W, const float *
   for (const void *b : bufs)
     if (b != nullptr && !aligned16(b)) return DVSSQ_ERR_MISALIGNED;
   if (!aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
-  if (workspace_bytes < encode_workspace_bytes(shape->M, shape->K, shape->n_sal)) return DVSSQ_ERR_WORKSPACE;
+  if (workspace_bytes < encode_workspace_bytes(shape->M, shape->K, shape->block, shape->n_sal))
+    return DVSSQ_ERR_WORKSPACE;
   if ((s = ensure_device()) != DVSSQ_OK) return s;
   EncodeArgs a;
   a.M = shape->M; a.K = shape->K; a.block = shape->block; a.n_sal = shape->n_sal;
@@ -282,6 +284,79 @@ dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvssq_weights 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = p == DVSSQ_PATH_DECODE ? launch_decode(a, st, launcher())
                                          : launch_prefill(a, st, launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------- MLP stack ---
+namespace {
+// Host-side checks of a stack and its flattening into matrix descriptors.
+dvssq_status stack_descs(const dvssq_mlp_layer *layers, int32_t n_layers,
+                         std::vector<StackMatDesc> &mats, StackShapeInfo &si) {
+  if (layers == nullptr || n_layers < 1 || n_layers > 4096) return DVSSQ_ERR_INVALID_ARG;
+  mats.assign((size_t)n_layers * 3, StackMatDesc{});
+  for (int l = 0; l < n_layers; ++l)
+    for (int mi = 0; mi < 3; ++mi) {
+      const dvssq_shape *sh = &layers[l].shape[mi];
+      const dvssq_weights *w = &layers[l].w[mi];
+      dvssq_status s = check_shape(sh);
+      if (s != DVSSQ_OK) return s;
+      if (w->q4 == nullptr || w->s4 == nullptr || w->s8 == nullptr) return DVSSQ_ERR_INVALID_ARG;
+      if (sh->n_sal > 0 && (w->sal_idx == nullptr || w->q8 == nullptr))
+        return DVSSQ_ERR_INVALID_ARG;
+      if (sh->rank > 0 && (w->U == nullptr || w->V == nullptr)) return DVSSQ_ERR_INVALID_ARG;
+      const void *bufs[] = {w->q4, w->s4, w->s8, w->sal_idx, w->q8, w->U, w->V};
+      for (const void *b : bufs)
+        if (b != nullptr && !aligned16(b)) return DVSSQ_ERR_MISALIGNED;
+      StackMatDesc &m = mats[(size_t)l * 3 + mi];
+      m.q4 = w->q4; m.s4 = w->s4; m.sal_idx = w->sal_idx; m.q8 = w->q8; m.s8 = w->s8;
+      m.U = w->U; m.V = w->V; m.vh = nullptr;
+      m.M = sh->M; m.K = sh->K; m.block = sh->block; m.n_sal = sh->n_sal; m.r = sh->rank;
+    }
+  if (!stack_shape_info(mats.data(), n_layers, si)) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  return DVSSQ_OK;
+}
+}  // namespace
+
+dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                            size_t *bytes) {
+  if (bytes == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  std::vector<StackMatDesc> mats;
+  StackShapeInfo si{};
+  dvssq_status s = stack_descs(layers, n_layers, mats, si);
+  if (s != DVSSQ_OK) return s;
+  *bytes = stack_workspace_bytes(si, n_layers);
+  return DVSSQ_OK;
+}
+
+dvssq_status dvssq_mlp_stack_prepare(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+  std::vector<StackMatDesc> mats;
+  StackShapeInfo si{};
+  dvssq_status s = stack_descs(layers, n_layers, mats, si);
+  if (s != DVSSQ_OK) return s;
+  if (workspace == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  if (!aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
+  if (workspace_bytes < stack_workspace_bytes(si, n_layers)) return DVSSQ_ERR_WORKSPACE;
+  cudaError_t e = stack_prepare(mats.data(), n_layers, si, workspace,
+                                static_cast<cudaStream_t>(stream), launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
+dvssq_status dvssq_mlp_stack_forward(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                     const void *x, void *y, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
+  std::vector<StackMatDesc> mats;
+  StackShapeInfo si{};
+  dvssq_status s = stack_descs(layers, n_layers, mats, si);
+  if (s != DVSSQ_OK) return s;
+  if (x == nullptr || y == nullptr || workspace == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
+  if (workspace_bytes < stack_workspace_bytes(si, n_layers)) return DVSSQ_ERR_WORKSPACE;
+  cudaError_t e = launch_mlp_stack(mats.data(), n_layers, si, x, y, workspace,
+                                   static_cast<cudaStream_t>(stream), launcher());
+  if (e == cudaErrorNotSupported) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
   return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
 }
 

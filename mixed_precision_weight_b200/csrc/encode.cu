@@ -3,16 +3,18 @@
 // Foundations §1-§2).
 //
 //   pass 1  W_rot = W . H_K row-block by row-block in fp64 (exact +-1 sums,
-//           one scale by 1/sqrt(b)); per-column sum of squares over fixed
-//           chunks of 16 rows; exactness check of every row-block.
-//   score   chunk partials summed in ascending order, score = a * sqrt(ssq).
+//           one scale by 1/sqrt(b)); per-column sums of squares over fixed
+//           chunks of 16 rows, summed by the CTA into groups of 8 chunks; the
+//           last CTA of each column block adds the groups in order and writes
+//           score = a * sqrt(ssq).  Exactness check of every row-block.
 //   select  the n_sal largest scores (ties -> lower index) by an MSB-first
-//           radix select in one CTA; outputs sorted indices, a column bit
-//           mask and per-32-column prefix counts.
-//   pass 2  rotation again, INT4 group RTN with BF16 scales, nibble packing,
-//           optional fp32 residual; salient values to an fp64 stash in the
-//           workspace and their per-row maxima by atomic max.
-//   pass 3  INT8 tier from the stash: one BF16 scale per row, codes.
+//           radix select in one CTA that stops as soon as the boundary digit
+//           is taken whole; outputs sorted indices and per-32-column prefix
+//           counts.
+//   pass 2  whole rows per CTA (dynamic tile order): rotation again, salient
+//           values moved to a shared-memory stash and zeroed in place, INT4
+//           group RTN with BF16 scales, nibble packing, optional fp32
+//           residual; then the INT8 tier of the CTA's rows from the stash.
 #include <algorithm>
 
 #include "common.cuh"
@@ -22,7 +24,10 @@
 namespace dvssq {
 
 constexpr int kSsqChunk = 16;     // rows per fixed-order partial (salience)
+constexpr int kSsqGroup = 8;      // chunk partials per group sum
 constexpr int kStages = 4;        // cp.async ring depth per group (row-blocks)
+constexpr int kTileRowsMax = 64;  // rows per pass-2 tile, upper bound
+constexpr int kStashSmemMax = 96 * 1024;
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
@@ -60,46 +65,70 @@ __device__ __forceinline__ uint16_t bf16_of_quotient(double a, double d, double 
   return f64_to_bf16_rn(q);
 }
 
-// Exponent statistics of one thread's 16 BF16 inputs: (max biased exponent,
-// min of max(biased exponent, 1)) over nonzero values.
-__device__ __forceinline__ void exp_stats(const uint16_t *x, int &emax, int &emin1) {
-#pragma unroll
-  for (int a = 0; a < 16; ++a) {
-    uint32_t m = x[a] & 0x7FFFu;
-    int eb = (int)(m >> 7);
-    if (m != 0) {
-      emax = max(emax, eb);
-      emin1 = min(emin1, max(eb, 1));
-    }
-  }
+// Per-halfword unsigned max / min of two pairs of 16-bit lanes.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Exponent statistics of BF16 pairs for the exact-sum test.  Per 16-bit lane:
+//   mx = max magnitude (the 15 bits below the sign),
+//   mn = min over nonzero values of (magnitude - 1); a zero maps to 0xFFFF.
+// Forcing the sign bits on makes every lane >= 0x8000, so subtracting one
+// from each lane never borrows across the halves.
+__device__ __forceinline__ void exp_pair_stats(uint32_t w, uint32_t &mx, uint32_t &mn) {
+  mx = vmax_u16x2(mx, w & 0x7FFF7FFFu);
+  mn = vmin_u16x2(mn, ((w | 0x80008000u) - 0x00010001u) ^ 0x80008000u);
+}
+
+// Spread test of one row-block from its (emax, emin1) over nonzero values,
+// biased BF16 exponents with subnormals counted as 1: every +-1 partial sum
+// of b terms is exact in fp64 when emax - emin1 <= 45 - log2(b).
+__device__ __forceinline__ bool spread_exceeds(int emax, int emin1, int lg) {
+  return emax >= 0 && emin1 <= 255 && (emax - emin1) > 45 - lg;
 }
 
 // ---------------------------------------------------------------- pass 1 --
-// One group of P threads per (row chunk, column block) pair; the group walks
-// the chunk's rows in ascending order so that each column's partial sum of
-// squares follows the fixed order acc = acc + w*w.
+// A CTA holds NG groups of P threads; group g owns the 16-row chunk
+// cg * NG + g of column block kb and walks it in ascending row order, so that
+// each column's chunk partial follows the fixed order acc = acc + w*w.  The
+// CTA then forms the 8-chunk group sums (ascending chunks, from 0.0) in shared
+// memory, and the CTA that finishes a column block last adds that block's
+// group sums in ascending order and writes the scores.
 template <int B>
-__global__ void __launch_bounds__(128) enc_pass1_kernel(const uint16_t *__restrict__ W, int M,
-                                                        int K, double c, double *__restrict__ part,
-                                                        unsigned long long *__restrict__ info) {
+__global__ void __launch_bounds__(128) enc_pass1_kernel(
+    const uint16_t *__restrict__ W, int M, int K, double c, const float *__restrict__ act_scale,
+    double *__restrict__ gpart, double *__restrict__ score, unsigned int *__restrict__ done,
+    unsigned long long *__restrict__ info) {
   constexpr int P = B / 16;
   constexpr int GPW = 32 / P;
   constexpr int NG = GPW * 4;
   constexpr int SCR = GroupScratch<B>::kElems;
+  static_assert(SCR >= B, "chunk partials reuse the transpose scratch");
+  static_assert(NG % kSsqGroup == 0, "whole chunk groups per CTA");
+  constexpr int SGC = NG / kSsqGroup;
   __shared__ double scratch[NG][SCR];
   __shared__ __align__(16) uint16_t ring[NG][kStages][B];
+  __shared__ unsigned int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = lane / P, t = lane % P;
   const int g = warp * GPW + gw;
   const int nkb = K / B;
   const int nchunk = (M + kSsqChunk - 1) / kSsqChunk;
-  const long long pair = (long long)blockIdx.x * NG + g;
-  const bool active = pair < (long long)nchunk * nkb;
-  const int chunk = active ? (int)(pair / nkb) : 0;
-  const int kb = active ? (int)(pair % nkb) : 0;
+  const int nsg = (nchunk + kSsqGroup - 1) / kSsqGroup;
+  const int ncg = (nchunk + NG - 1) / NG;
+  const int cg = blockIdx.x / nkb, kb = blockIdx.x - cg * nkb;
+  const int chunk = cg * NG + g;
   const int r0 = chunk * kSsqChunk;
-  const int nrows = active ? min(kSsqChunk, M - r0) : 0;
+  const int nrows = chunk < nchunk ? min(kSsqChunk, M - r0) : 0;
+  const int lg = (B == 256) ? 8 : 7;
 
   // Each row-block is B*2 bytes = 2B/16 16-byte pieces; P threads copy them.
   constexpr int PIECES = B * 2 / 16;
@@ -118,22 +147,25 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(const uint16_t *__restri
   double ssq[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) ssq[j] = 0.0;
-  unsigned long long inexact = 0;
-  const int lg = (B == 256) ? 8 : 7;
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;
 
   for (int i = 0; i < kSsqChunk; ++i) {   // uniform trip count keeps the warp converged
     issue(i + kStages - 1);
     cp_async_wait<kStages - 1>();
     __syncwarp();
-    uint16_t xin[16];
     const uint16_t *buf = ring[g][i % kStages];
-#pragma unroll
-    for (int a = 0; a < 16; ++a) xin[a] = buf[P * a + t];
-    int emax = -1, emin1 = 1 << 20;
-    exp_stats(xin, emax, emin1);
+    if (i < nrows) {
+      // this thread's 32 contiguous bytes of the row-block, for the exact-sum test
+      const uint4 *wq = reinterpret_cast<const uint4 *>(buf) + 2 * t;
+      const uint4 a = wq[0], b = wq[1];
+      exp_pair_stats(a.x, mx, mn); exp_pair_stats(a.y, mx, mn);
+      exp_pair_stats(a.z, mx, mn); exp_pair_stats(a.w, mx, mn);
+      exp_pair_stats(b.x, mx, mn); exp_pair_stats(b.y, mx, mn);
+      exp_pair_stats(b.z, mx, mn); exp_pair_stats(b.w, mx, mn);
+    }
     double v[16];
 #pragma unroll
-    for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(xin[a]);
+    for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
     fwht_group<B>(v, scratch[g], t);
     if (i < nrows) {
 #pragma unroll
@@ -143,74 +175,86 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(const uint16_t *__restri
         ssq[j] = __dadd_rn(ssq[j], __dmul_rn(w, w));
       }
     }
-    // exactness of this row-block: reduce over the P lanes of the group
-#pragma unroll
-    for (int o = 1; o < P; o <<= 1) {
-      emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
-      emin1 = min(emin1, __shfl_xor_sync(0xffffffffu, emin1, o));
-    }
-    if (t == 0 && i < nrows && emax >= 0 && (emax - emin1) > 45 - lg) ++inexact;
     __syncwarp();
   }
   cp_async_wait<0>();
-  if (active) {
-    double *dst = part + (size_t)chunk * K + (size_t)kb * B + 16 * t;
-    if (B == 256) {
-      const double c2 = c * c;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) ssq[j] = __dmul_rn(ssq[j], c2);
-    }
-#pragma unroll
-    for (int j = 0; j < 16; j += 2) {
-      double2 d = make_double2(ssq[j], ssq[j + 1]);
-      *reinterpret_cast<double2 *>(dst + j) = d;
-    }
-    if (t == 0 && inexact) atomicAdd(&info[0], inexact);
-  }
-}
 
-// ----------------------------------------------------------------- score --
-// ssq_j = sum over groups (ascending) of [sum over the group's 8 chunk
-// partials (ascending)]; score_j = a_j * sqrt(ssq_j).  A CTA owns 32 columns:
-// its 256 threads form group sums (8 independent loads each) into shared
-// memory, 64 groups at a time, and 32 threads add them in order.
-constexpr int kSsqGroup = 8;
-constexpr int kScoreCols = 32;
-constexpr int kScoreGroupsPerPass = 64;
-
-__global__ void __launch_bounds__(256) enc_score_kernel(
-    const double *__restrict__ part, int nchunk, int K, const float *__restrict__ act_scale,
-    double *__restrict__ score, unsigned long long *__restrict__ info) {
-  __shared__ double gs[kScoreGroupsPerPass][kScoreCols + 1];
-  const int tid = threadIdx.x, col = tid & 31, sub = tid >> 5;     // 8 sub-rows
-  const int j0 = blockIdx.x * kScoreCols;
-  const int j = j0 + col;
-  const int ngroups = (nchunk + kSsqGroup - 1) / kSsqGroup;
-  double tot = 0.0;
-  for (int g0 = 0; g0 < ngroups; g0 += kScoreGroupsPerPass) {
-    const int gn = min(kScoreGroupsPerPass, ngroups - g0);
-    for (int gi = sub; gi < gn; gi += 8) {
-      const int c0 = (g0 + gi) * kSsqGroup;
-      double v[kSsqGroup];
+  // Exact-sum test, first over the whole chunk: the chunk's spread bounds the
+  // spread of each of its row-blocks.  Only a chunk that fails it is checked
+  // row by row (from global memory).
+  {
+    const uint32_t mxh = max(mx & 0xFFFFu, mx >> 16), mnh = min(mn & 0xFFFFu, mn >> 16);
+    const int emax = (int)(mxh >> 7);
+    const int emin1 = mnh == 0xFFFFu ? 0xFFFF : max((int)((mnh + 1u) >> 7), 1);
+    // one u16x2 word reduced by max: (emax, 0xFFFF - emin1)
+    uint32_t pk = ((uint32_t)emax << 16) | (uint32_t)(0xFFFF - emin1);
 #pragma unroll
-      for (int u = 0; u < kSsqGroup; ++u)
-        v[u] = (j < K && c0 + u < nchunk) ? part[(size_t)(c0 + u) * K + j] : 0.0;
-      double sgrp = 0.0;
+    for (int o = 1; o < P; o <<= 1) pk = vmax_u16x2(pk, __shfl_xor_sync(0xffffffffu, pk, o));
+    const int gmax = (int)(pk >> 16), gmin1 = 0xFFFF - (int)(pk & 0xFFFFu);
+    const bool fail = nrows > 0 && spread_exceeds(gmax, gmin1, lg);
+    // the warp's groups may differ: the whole warp runs the row loop (its
+    // shuffles need every lane), each group counting only its own rows
+    if (__any_sync(0xffffffffu, fail)) {
+      unsigned long long inexact = 0;
+      for (int i = 0; i < kSsqChunk; ++i) {
+        const bool row = fail && i < nrows;
+        uint32_t rx = 0u, rn = 0xFFFFFFFFu;
+        if (row) {
+          const uint32_t *src =
+              reinterpret_cast<const uint32_t *>(W + (size_t)(r0 + i) * K + (size_t)kb * B);
+          for (int q = t; q < B / 2; q += P) exp_pair_stats(src[q], rx, rn);
+        }
+        const uint32_t rxh = max(rx & 0xFFFFu, rx >> 16), rnh = min(rn & 0xFFFFu, rn >> 16);
+        const int re = (int)(rxh >> 7);
+        const int rm = rnh == 0xFFFFu ? 0xFFFF : max((int)((rnh + 1u) >> 7), 1);
+        uint32_t rp = ((uint32_t)re << 16) | (uint32_t)(0xFFFF - rm);
 #pragma unroll
-      for (int u = 0; u < kSsqGroup; ++u)
-        if (c0 + u < nchunk) sgrp = __dadd_rn(sgrp, v[u]);
-      gs[gi][col] = sgrp;
+        for (int o = 1; o < P; o <<= 1) rp = vmax_u16x2(rp, __shfl_xor_sync(0xffffffffu, rp, o));
+        if (row) inexact += spread_exceeds((int)(rp >> 16), 0xFFFF - (int)(rp & 0xFFFFu), lg);
+      }
+      if (t == 0 && inexact) atomicAdd(&info[0], inexact);
     }
-    __syncthreads();
-    if (sub == 0)
-      for (int gi = 0; gi < gn; ++gi) tot = __dadd_rn(tot, gs[gi][col]);
-    __syncthreads();
   }
-  if (sub == 0 && j < K) {
+
+  // chunk partials -> shared memory (the transpose scratch is free now)
+  if (B == 256) {
+    const double c2 = c * c;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ssq[j] = __dmul_rn(ssq[j], c2);
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) scratch[g][16 * t + j] = ssq[j];
+  __syncthreads();
+  // group sums: SGC chunk groups x B columns, two per thread
+  for (int it = threadIdx.x; it < SGC * B; it += blockDim.x) {
+    const int sl = it / B, col = it - sl * B;
+    const int sg = cg * SGC + sl;
+    if (sg >= nsg) continue;
+    double s = 0.0;
+#pragma unroll
+    for (int u = 0; u < kSsqGroup; ++u) {
+      const int gg = sl * kSsqGroup + u;
+      if (cg * NG + gg < nchunk) s = __dadd_rn(s, scratch[gg][col]);
+    }
+    gpart[(size_t)sg * K + (size_t)kb * B + col] = s;
+  }
+  // the last CTA of this column block adds its group sums in order
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&done[kb], 1u) == (unsigned int)(ncg - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  unsigned long long bad = 0;
+  for (int col = threadIdx.x; col < B; col += blockDim.x) {
+    const int j = kb * B + col;
+    double tot = 0.0;
+    for (int sg = 0; sg < nsg; ++sg) tot = __dadd_rn(tot, __ldcg(gpart + (size_t)sg * K + j));
     const double s = __dmul_rn((double)act_scale[j], __dsqrt_rn(tot));
-    if (!isfinite(s)) atomicAdd(&info[2], 1ull);
+    bad += !isfinite(s);
     score[j] = s;
   }
+  if (bad) atomicAdd(&info[2], bad);
 }
 
 // ---------------------------------------------------------------- select --
@@ -253,22 +297,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp, int *s_t
   return r;
 }
 
+// MSB-first radix select over 8-bit digits.  After each digit the CTA knows
+// the prefix of the n_sal-th largest key and how many keys sharing that prefix
+// are still to be taken (krem).  When krem equals the number of keys with the
+// prefix, every one of them is taken and the lower digits no longer matter:
+// the loop stops there (typically after the exponent and two or three
+// significand digits) instead of running all eight digits.
 __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
-    const double *__restrict__ score, int K, int n_sal, int M, int32_t *__restrict__ sal_idx,
-    uint32_t *__restrict__ sal_mask, int32_t *__restrict__ sal_prefix,
-    unsigned long long *__restrict__ rowmax) {
+    const double *__restrict__ score, int K, int n_sal, int32_t *__restrict__ sal_idx,
+    int32_t *__restrict__ sal_prefix) {
   extern __shared__ unsigned long long skeys[];
   __shared__ unsigned int hist[256];
   __shared__ int s_warp[32];
   __shared__ int s_total;
   __shared__ unsigned long long s_prefix;
-  __shared__ unsigned int s_krem;
+  __shared__ unsigned int s_krem, s_whole;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool in_smem = K <= kSelSmemKeys;
 
-  for (int i = tid; i < M; i += kSelThreads) rowmax[i] = 0ull;    // for pass 2
-  for (int w = tid; w < (K + 31) / 32; w += kSelThreads) sal_mask[w] = 0u;
-  if (n_sal == 0) return;
+  if (n_sal == 0) {
+    for (int w = tid; w < (K + 31) / 32; w += kSelThreads) sal_prefix[w] = 0;
+    return;
+  }
   if (in_smem)
     for (int j = tid; j < K; j += kSelThreads) skeys[j] = order_key(score[j]);
   __syncthreads();
@@ -336,6 +386,7 @@ __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
           cum += hist[d];
         }
         s_krem = krem - cum;
+        s_whole = (krem - cum) == hist[d];
         s_prefix = prefix | ((unsigned long long)d << shift);
       }
     }
@@ -343,222 +394,319 @@ __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
     krem = s_krem;
     prefix = s_prefix;
     pmask |= 255ull << shift;
+    const bool whole = s_whole;
     __syncthreads();
+    if (whole) break;
   }
-  // prefix = key of the n_sal-th largest score; krem = how many keys equal to
-  // it are taken, lowest indices first.  Contiguous index ranges per thread.
+  // Selected: (key & pmask) > prefix, or == prefix among the first krem such
+  // keys in index order.  Contiguous index ranges per thread; sal_prefix[w] is
+// the number of selected columns below column 32 w.
   const int per = (K + kSelThreads - 1) / kSelThreads;
   const int j0 = min(K, tid * per), j1 = min(K, j0 + per);
   int n_eq = 0;
-  for (int j = j0; j < j1; ++j) n_eq += key(j) == prefix;
+  for (int j = j0; j < j1; ++j) n_eq += (key(j) & pmask) == prefix;
   const int eq_before = block_exclusive_scan(n_eq, s_warp, &s_total);
   int n_sel = 0;
   {
     int eqr = eq_before;
     for (int j = j0; j < j1; ++j) {
-      const unsigned long long k = key(j);
+      const unsigned long long k = key(j) & pmask;
       n_sel += k > prefix || (k == prefix && (unsigned)(eqr++) < krem);
     }
   }
   int pos = block_exclusive_scan(n_sel, s_warp, &s_total);
   int eqr = eq_before;
   for (int j = j0; j < j1; ++j) {
-    const unsigned long long k = key(j);
+    const unsigned long long k = key(j) & pmask;
     const bool sel = k > prefix || (k == prefix && (unsigned)(eqr++) < krem);
     if ((j & 31) == 0) sal_prefix[j >> 5] = pos;
-    if (sel && pos < n_sal) {
-      sal_idx[pos++] = j;
-      atomicOr(&sal_mask[j >> 5], 1u << (j & 31));
-    }
+    if (sel && pos < n_sal) sal_idx[pos++] = j;
   }
 }
 
 // ---------------------------------------------------------------- pass 2 --
-// One group of P threads per (8 rows, column block): rotate again, INT4 group
-// RTN with BF16 scales, nibble packing, optional fp32 residual.  Salient
-// values go to the fp64 stash sv[row][entry] and the row maxima of their
-// magnitudes to rowmax (atomic max on the bit patterns of non-negative
-// doubles).  For b = 256 the scale c = 1/16 is a power of two: the stash and
-// rowmax hold the unscaled sums and pass 3 applies c exactly, and the codes
-// use w * inv = v * (c * inv) exactly.
-constexpr int kP2Rows = 8;
+// A CTA takes tiles of R whole rows from a global counter.  Within a tile the
+// R * nkb row-blocks are ordered column-block-major and split into NG equal
+// runs of ipg >= kStages - 1 row-blocks, one run per group, so a group's
+// cp.async ring can run ahead into the next tile (whose index is fetched one
+// tile early).  Per row-block the group rotates again, stages its outputs in
+// shared memory, moves the block's salient values to the stash and zeroes
+// them in place (so the INT4 tier needs no column mask: a zero has code 0),
+// then quantises.  When the tile is done the CTA forms each row's INT8 scale
+// from the stash and writes the INT8 codes.  For b = 256 the scale c = 1/16 is
+// a power of two: the stash holds the unscaled sums and c is applied exactly
+// in the scales, and the codes use w * inv = v * (c * inv) exactly.
+struct Pass2Params {
+  const uint16_t *W;
+  int M, K, n_sal;
+  int R, rshift;      // rows per tile (a power of two) and its log2
+  int ipg;            // row-blocks per group and tile
+  int ntiles;
+  int stash_smem;     // 1: stash in dynamic shared memory [2][R][n_sal]; 0: in sv [M][n_sal]
+  double c;
+  const int32_t *sal_idx, *sal_prefix;
+  uint8_t *q4;
+  uint16_t *s4;
+  int8_t *q8;
+  uint16_t *s8;
+  float *resid;
+  double *sv;
+  unsigned int *tile_ctr;
+  unsigned long long *info;
+};
+
+constexpr int kStageStride = 18;   // doubles per thread's 16 staged outputs (+2: no bank conflicts)
+
+// Eight 4-bit codes (two's complement in the low bits of l[0..7]) into one
+// word, code 2m in the low nibble of byte m.
+__device__ __forceinline__ uint32_t pack_nibbles8(const uint32_t *l) {
+  const uint32_t e = __byte_perm(__byte_perm(l[0], l[2], 0x0040), __byte_perm(l[4], l[6], 0x4000),
+                                 0x7610);
+  const uint32_t o = __byte_perm(__byte_perm(l[1], l[3], 0x0040), __byte_perm(l[5], l[7], 0x4000),
+                                 0x7610);
+  return (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+}
 
 template <int B, bool RESID>
-__global__ void __launch_bounds__(128) enc_pass2_kernel(
-    const uint16_t *__restrict__ W, int M, int K, int n_sal, double c,
-    const uint32_t *__restrict__ sal_mask, const int32_t *__restrict__ sal_prefix,
-    uint8_t *__restrict__ q4, uint16_t *__restrict__ s4, double *__restrict__ sv,
-    unsigned long long *__restrict__ rowmax, float *__restrict__ resid,
-    unsigned long long *__restrict__ info) {
+__global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) {
   constexpr int P = B / 16;
   constexpr int GPW = 32 / P;
   constexpr int NG = GPW * 4;
-  constexpr int SCR = GroupScratch<B>::kElems;
+  constexpr int SCR0 = GroupScratch<B>::kElems;
+  constexpr int SCR1 = P * kStageStride;
+  constexpr int SCR = ((SCR0 > SCR1 ? SCR0 : SCR1) + 1) & ~1;   // even: 16-byte aligned rows
   constexpr bool kPow2 = B == 256;
-  __shared__ double scratch[NG][SCR];
+  constexpr int PIECES = B * 2 / 16;
+  __shared__ __align__(16) double scratch[NG][SCR];
   __shared__ __align__(16) uint16_t ring[NG][kStages][B];
+  __shared__ unsigned long long s_rmax[2][kTileRowsMax];
+  __shared__ int s_tile[4];
+  extern __shared__ __align__(16) double stash_s[];
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gw = lane / P, t = lane % P;
   const int g = warp * GPW + gw;
-  const int nkb = K / B;
-  const int nrc = (M + kP2Rows - 1) / kP2Rows;
-  const long long pair = (long long)blockIdx.x * NG + g;
-  const bool active = pair < (long long)nrc * nkb;
-  const int rc = active ? (int)(pair / nkb) : 0;
-  const int kb = active ? (int)(pair % nkb) : 0;
-  const int r0 = rc * kP2Rows;
-  const int nrows = active ? min(kP2Rows, M - r0) : 0;
-  const double kInv7 = 1.0 / 7.0;
+  const int M = p.M, K = p.K, n_sal = p.n_sal, R = p.R, rshift = p.rshift;
+  const int ipg = p.ipg, ntiles = p.ntiles;
+  const int item0 = g * ipg;
+  const double c = p.c;
+  const double kInv7 = 1.0 / 7.0, kInv127 = 1.0 / 127.0;
+  double *const sgrp = scratch[g];
 
-  // salient columns among this thread's 16 are the same for every row
-  const int col0 = kb * B + 16 * t;
-  const uint32_t mword = sal_mask[col0 >> 5];
-  const int bit0 = col0 & 31;
-  const uint32_t m16 = (mword >> bit0) & 0xFFFFu;
-  const int ebase = m16 ? sal_prefix[col0 >> 5] + __popc(mword & ((1u << bit0) - 1u)) : 0;
+  if (tid == 0) {
+    s_tile[0] = (int)atomicAdd(p.tile_ctr, 1u);
+    s_tile[1] = (int)atomicAdd(p.tile_ctr, 1u);
+  }
+  for (int i = tid; i < 2 * kTileRowsMax; i += blockDim.x) (&s_rmax[0][0])[i] = 0ull;
+  __syncthreads();
+  int cur = s_tile[0], nxt = s_tile[1];
 
-  constexpr int PIECES = B * 2 / 16;
-  auto issue = [&](int i) {
-    if (i < nrows) {
-      const uint16_t *src = W + (size_t)(r0 + i) * K + (size_t)kb * B;
-      uint16_t *dst = ring[g][i % kStages];
+  // source of row-block ii of this group in tile `tile` (nullptr: none)
+  auto src_of = [&](int tile, int ii) -> const uint16_t * {
+    if (tile >= ntiles) return nullptr;
+    const int item = item0 + ii;
+    const int kb = item >> rshift;
+    const int row = (tile << rshift) + (item - (kb << rshift));
+    if (row >= M) return nullptr;
+    return p.W + (size_t)row * K + (size_t)kb * B;
+  };
+  auto issue = [&](const uint16_t *src, int slot) {
+    if (src != nullptr) {
+      uint16_t *dst = ring[g][slot];
 #pragma unroll
-      for (int p = t; p < PIECES; p += P) cp_async16(dst + p * 8, src + p * 8);
+      for (int q = t; q < PIECES; q += P) cp_async16(dst + q * 8, src + q * 8);
     }
     cp_async_commit();
   };
 #pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
+  for (int s = 0; s < kStages - 1; ++s) issue(src_of(cur, s), s);
 
   unsigned long long unsafe = 0;
-  for (int i = 0; i < kP2Rows; ++i) {
-    issue(i + kStages - 1);
-    cp_async_wait<kStages - 1>();
-    __syncwarp();
-    double v[16];
-    const uint16_t *buf = ring[g][i % kStages];
+  int pos = 0;    // ring position of the row-block in hand
+  int k = 0;      // tiles done by this CTA: parity of the stash and the row maxima
+  while (cur < ntiles) {
+    if (tid == 0) s_tile[2 + (k & 1)] = (int)atomicAdd(p.tile_ctr, 1u);   // the tile after nxt
+    double *const stash = p.stash_smem ? stash_s + (size_t)(k & 1) * R * n_sal : nullptr;
+    for (int ii = 0; ii < ipg; ++ii, ++pos) {
+      const int ia = ii + kStages - 1;
+      issue(ia < ipg ? src_of(cur, ia) : src_of(nxt, ia - ipg), (pos + kStages - 1) % kStages);
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
+      const int item = item0 + ii;
+      const int kb = item >> rshift, r = item - (kb << rshift);
+      const int row = (cur << rshift) + r;
+      const bool valid = row < M;
+      const uint16_t *buf = ring[g][pos % kStages];
+      double v[16];
 #pragma unroll
-    for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
-    fwht_group<B>(v, scratch[g], t);
-    const int row = r0 + i;
-    // v holds the values the codes see: unscaled sums (b = 256) or w = c * sum
-    if (!kPow2) {
+      for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
+      fwht_group<B>(v, sgrp, t);
+      // v holds the values the codes see: unscaled sums (b = 256) or w = c * sum
+      if (!kPow2) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = __dmul_rn(v[j], c);
-    }
-    double amax = 0.0, amax8 = 0.0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if ((m16 >> j) & 1u) amax8 = fmax(amax8, fabs(v[j]));
-      else amax = fmax(amax, fabs(v[j]));
-    }
-    amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 64-column group
-    amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-#pragma unroll
-    for (int o = 1; o < P; o <<= 1) amax8 = fmax(amax8, __shfl_xor_sync(0xffffffffu, amax8, o));
-    // absmax of w = c * amax (exact for b = 256)
-    const uint16_t sbits = bf16_of_quotient(kPow2 ? amax * c : amax, 7.0, kInv7);
-    const double s = bf16_bits_to_f64(sbits);
-    const double inv = s > 0.0 ? recip_bf16(sbits) : 0.0;
-    const double vinv = kPow2 ? inv * c : inv;    // multiplies v
-    uint32_t word[2] = {0u, 0u};
-    int e = ebase;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      int q = 0;
-      if (!((m16 >> j) & 1u)) {
-        q = __double2int_rn(__dmul_rn(v[j], vinv));
-        q = min(7, max(-8, q));
-      } else {
-        if (i < nrows && e < n_sal) sv[(size_t)row * n_sal + e] = v[j];
-        ++e;
+        for (int j = 0; j < 16; ++j) v[j] = __dmul_rn(v[j], c);
       }
-      word[j >> 3] |= ((uint32_t)q & 0xFu) << (4 * (j & 7));
-    }
-    if (i < nrows) {
-      *reinterpret_cast<uint2 *>(q4 + (size_t)row * (K / 2) + (col0 >> 1)) =
-          make_uint2(word[0], word[1]);
-      if ((t & 3) == 0) {
-        s4[(size_t)row * (K / 64) + (col0 >> 6)] = sbits;
-        if (s > 0.0 && (s < 0x1p-17 || s > 8188.0)) ++unsafe;
-      }
-      if (t == 0 && amax8 > 0.0)
-        atomicMax(&rowmax[row], (unsigned long long)__double_as_longlong(amax8));
-      if (RESID) {
-        float rres[16];
+      double2 *stg = reinterpret_cast<double2 *>(sgrp + t * kStageStride);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const double w = kPow2 ? v[j] * c : v[j];
-          if ((m16 >> j) & 1u) {
-            rres[j] = 0.0f;
-          } else {
-            const int q = (int)((word[j >> 3] >> (4 * (j & 7))) << 28) >> 28;
-            rres[j] = (float)__dsub_rn(w, (double)q * s);
-          }
+      for (int m = 0; m < 8; ++m) stg[m] = make_double2(v[2 * m], v[2 * m + 1]);
+      __syncwarp();
+      // this block's salient columns: to the stash, then zero in the staged row
+      const int e0 = __ldg(p.sal_prefix + ((kb * B) >> 5));
+      const int e1 = (kb + 1) * B < K ? __ldg(p.sal_prefix + (((kb + 1) * B) >> 5)) : n_sal;
+      if (valid && e0 < e1) {
+        double *dst = stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal;
+        for (int e = e0 + t; e < e1; e += P) {
+          const int col = __ldg(p.sal_idx + e) - kb * B;
+          const int si = (col >> 4) * kStageStride + (col & 15);
+          dst[e] = sgrp[si];
+          sgrp[si] = 0.0;
         }
-        float4 *dst = reinterpret_cast<float4 *>(resid + (size_t)row * K + col0);
+      }
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          dst[j / 4] = make_float4(rres[j], rres[j + 1], rres[j + 2], rres[j + 3]);
+      for (int m = 0; m < 8; ++m) {
+        const double2 d = stg[m];
+        v[2 * m] = d.x;
+        v[2 * m + 1] = d.y;
+      }
+      // group absmax over 64 columns = 4 threads
+      double amax = 0.0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmax(amax, fabs(v[j]));
+      amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // absmax of w = c * amax (exact for b = 256)
+      const uint16_t sbits = bf16_of_quotient(kPow2 ? amax * c : amax, 7.0, kInv7);
+      const double s = bf16_bits_to_f64(sbits);
+      const double inv = s > 0.0 ? recip_bf16(sbits) : 0.0;
+      const double vinv = kPow2 ? inv * c : inv;    // multiplies v
+      // RN64 is monotone, so max_j |RN64(v_j vinv)| = RN64(amax vinv); below
+      // 7.5 every code is in [-7, 7] and rint is the add of 1.5 * 2^52 (exact
+      // round-half-even to an integer whose two's complement is the low word)
+      uint32_t lo[16];
+      if (__dmul_rn(amax, vinv) < 7.5) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          lo[j] = (uint32_t)__double2loint(__dadd_rn(__dmul_rn(v[j], vinv), 0x1.8p52));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          lo[j] = (uint32_t)min(7, max(-8, __double2int_rn(__dmul_rn(v[j], vinv))));
+      }
+      if (valid) {
+        const int col0 = kb * B + 16 * t;
+        *reinterpret_cast<uint2 *>(p.q4 + (size_t)row * (K / 2) + (col0 >> 1)) =
+            make_uint2(pack_nibbles8(lo), pack_nibbles8(lo + 8));
+        if ((t & 3) == 0) {
+          p.s4[(size_t)row * (K / 64) + (col0 >> 6)] = sbits;
+          if (s > 0.0 && (s < 0x1p-17 || s > 8188.0)) ++unsafe;
+        }
+        if (RESID) {
+          float rres[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const double w = kPow2 ? v[j] * c : v[j];
+            rres[j] = (float)__dsub_rn(w, (double)(int)lo[j] * s);
+          }
+          float4 *rdst = reinterpret_cast<float4 *>(p.resid + (size_t)row * K + col0);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            rdst[j / 4] = make_float4(rres[j], rres[j + 1], rres[j + 2], rres[j + 3]);
+        }
+      }
+      __syncwarp();
+    }
+
+    // INT8 tier of the tile's rows: s8 = bf16_rn(max|w| / 127), q8 = clip(rint(w / s8))
+    __syncthreads();                      // the tile's stash is complete
+    const int n8 = n_sal >> 3;
+    const double vscale = kPow2 ? c : 1.0;
+    for (int ch = tid; ch < (n8 << rshift); ch += blockDim.x) {
+      const int r = ch / n8, e = (ch - r * n8) * 8;
+      const int row = (cur << rshift) + r;
+      if (row >= M) continue;
+      const double2 *src = reinterpret_cast<const double2 *>(
+          (stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal) + e);
+      double m = 0.0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double2 d = src[u];
+        m = fmax(m, fmax(fabs(d.x), fabs(d.y)));
+      }
+      atomicMax(&s_rmax[k & 1][r], (unsigned long long)__double_as_longlong(m));
+    }
+    __syncthreads();                      // row maxima complete
+    if (tid < R) s_rmax[(k + 1) & 1][tid] = 0ull;
+    for (int ch = tid; ch < (n8 << rshift); ch += blockDim.x) {
+      const int r = ch / n8, e = (ch - r * n8) * 8;
+      const int row = (cur << rshift) + r;
+      if (row >= M) continue;
+      const double2 *src = reinterpret_cast<const double2 *>(
+          (stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal) + e);
+      const double m = __longlong_as_double((long long)s_rmax[k & 1][r]) * vscale;
+      const uint16_t sb = bf16_of_quotient(m, 127.0, kInv127);
+      const double s8v = bf16_bits_to_f64(sb);
+      const double vinv = s8v > 0.0 ? recip_bf16(sb) * vscale : 0.0;
+      uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double2 d = src[u];
+        const int qa = min(127, max(-128, __double2int_rn(__dmul_rn(d.x, vinv))));
+        const int qb = min(127, max(-128, __double2int_rn(__dmul_rn(d.y, vinv))));
+        pk[u >> 1] |= (((uint32_t)qa & 0xFFu) | (((uint32_t)qb & 0xFFu) << 8)) << (16 * (u & 1));
+      }
+      *reinterpret_cast<uint2 *>(p.q8 + (size_t)row * n_sal + e) = make_uint2(pk[0], pk[1]);
+      if (e == 0) {
+        p.s8[row] = sb;
+        if (s8v > 0.0 && (s8v < 0x1p-17 || s8v > 511.0)) ++unsafe;
       }
     }
-    __syncwarp();
+    if (n8 == 0)
+      for (int r = tid; r < R; r += blockDim.x)
+        if ((cur << rshift) + r < M) p.s8[(cur << rshift) + r] = 0;
+    cur = nxt;
+    nxt = s_tile[2 + (k & 1)];
+    ++k;
   }
   cp_async_wait<0>();
-  if (active && unsafe) atomicAdd(&info[1], unsafe);
-}
-
-// ---------------------------------------------------------------- pass 3 --
-// INT8 tier: s8 = bf16_rn(max|w| / 127), q8 = clip(rint(w * (1/s8))).  The
-// stash holds w / vscale (vscale = c for b = 256, else 1).  One thread per 8
-// entries of a row.
-__global__ void __launch_bounds__(256) enc_pass3_kernel(
-    const double *__restrict__ sv, const unsigned long long *__restrict__ rowmax, int M,
-    int n_sal, double vscale, int8_t *__restrict__ q8, uint16_t *__restrict__ s8,
-    unsigned long long *__restrict__ info) {
-  const int n8 = n_sal / 8;
-  const long long items = n8 > 0 ? (long long)M * n8 : (long long)M;
-  const double kInv127 = 1.0 / 127.0;
-  for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < items;
-       it += (long long)gridDim.x * blockDim.x) {
-    const int row = n8 > 0 ? (int)(it / n8) : (int)it;
-    const int e0 = n8 > 0 ? 8 * (int)(it % n8) : 0;
-    const double2 *src = reinterpret_cast<const double2 *>(sv + (size_t)row * n_sal + e0);
-    double2 d[4];
-    if (n8 > 0) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) d[u] = src[u];
-    }
-    const double m = __longlong_as_double((long long)rowmax[row]) * vscale;
-    const uint16_t sbits = bf16_of_quotient(m, 127.0, kInv127);
-    const double sv8 = bf16_bits_to_f64(sbits);
-    if (e0 == 0) {
-      s8[row] = sbits;
-      if (sv8 > 0.0 && (sv8 < 0x1p-17 || sv8 > 511.0)) atomicAdd(&info[1], 1ull);
-    }
-    if (n8 == 0) continue;
-    const double vinv = sv8 > 0.0 ? recip_bf16(sbits) * vscale : 0.0;
-    uint32_t pk[2] = {0u, 0u};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      int qa = __double2int_rn(__dmul_rn(d[u].x, vinv));
-      int qb = __double2int_rn(__dmul_rn(d[u].y, vinv));
-      qa = min(127, max(-128, qa));
-      qb = min(127, max(-128, qb));
-      pk[u >> 1] |= (((uint32_t)qa & 0xFFu) | (((uint32_t)qb & 0xFFu) << 8)) << (16 * (u & 1));
-    }
-    *reinterpret_cast<uint2 *>(q8 + (size_t)row * n_sal + e0) = make_uint2(pk[0], pk[1]);
-  }
+  if (unsafe) atomicAdd(&p.info[1], unsafe);
 }
 
 // --------------------------------------------------------------- launch ---
 namespace {
-struct EncodeLayout {
-  size_t info, part, score, mask, pref, rowmax, sv, total;
+constexpr int groups_per_cta(int B) { return (32 / (B / 16)) * 4; }
+
+struct Pass2Plan {
+  int R, rshift, ipg, ntiles;
+  bool smem;
+  size_t smem_bytes;
 };
-EncodeLayout encode_layout(int M, int K, int n_sal) {
+
+// Rows per tile: the smallest power of two that splits the tile's R * nkb
+// row-blocks evenly over the groups with at least kStages - 1 per group.
+Pass2Plan pass2_plan(int M, int K, int B, int n_sal) {
+  const int NG = groups_per_cta(B), nkb = K / B;
+  int R = 1;
+  while ((R * nkb) % NG != 0 || R * nkb / NG < kStages - 1) R *= 2;
+  Pass2Plan pl{};
+  pl.R = R;
+  pl.rshift = 0;
+  while ((1 << pl.rshift) < R) ++pl.rshift;
+  pl.ipg = R * nkb / NG;
+  pl.ntiles = (M + R - 1) / R;
+  const size_t bytes = (size_t)2 * R * n_sal * sizeof(double);
+  pl.smem = bytes <= (size_t)kStashSmemMax;
+  pl.smem_bytes = pl.smem ? bytes : 0;
+  return pl;
+}
+
+struct EncodeLayout {
+  size_t info, ctr, done, zero_bytes, gpart, score, pref, sv, total;
+};
+EncodeLayout encode_layout(int M, int K, int block, int n_sal) {
   const size_t nchunk = (size_t)(M + kSsqChunk - 1) / kSsqChunk;
+  const size_t nsg = (nchunk + kSsqGroup - 1) / kSsqGroup;
+  const Pass2Plan pl = pass2_plan(M, K, block, n_sal);
   EncodeLayout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -566,73 +714,88 @@ EncodeLayout encode_layout(int M, int K, int n_sal) {
     off += (bytes + 255) & ~(size_t)255;
     return o;
   };
-  L.info = take(4 * sizeof(unsigned long long));
-  L.part = take(nchunk * (size_t)K * sizeof(double));
+  // counters zeroed at the start of every encode: info[4], tile counter, done[nkb]
+  L.info = take(4 * sizeof(unsigned long long) + sizeof(unsigned int) +
+                (size_t)(K / block) * sizeof(unsigned int));
+  L.ctr = L.info + 4 * sizeof(unsigned long long);
+  L.done = L.ctr + sizeof(unsigned int);
+  L.zero_bytes = 4 * sizeof(unsigned long long) + sizeof(unsigned int) +
+                 (size_t)(K / block) * sizeof(unsigned int);
+  L.gpart = take(nsg * (size_t)K * sizeof(double));
   L.score = take((size_t)K * sizeof(double));
-  L.mask = take((size_t)((K + 31) / 32) * sizeof(uint32_t));
   L.pref = take((size_t)((K + 31) / 32) * sizeof(int32_t));
-  L.rowmax = take((size_t)M * sizeof(unsigned long long));
-  L.sv = take((size_t)M * n_sal * sizeof(double));
+  L.sv = take(pl.smem ? 0 : (size_t)M * n_sal * sizeof(double));
   L.total = off;
   return L;
 }
+
+template <int B, bool RESID>
+cudaError_t launch_pass2(const Pass2Params &pp, size_t smem, cudaStream_t st, Launcher &L) {
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, enc_pass2_kernel<B, RESID>,
+                                                                128, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const long long grid = std::max(1LL, std::min<long long>(pp.ntiles, (long long)nsm * occ));
+  return L.launch("enc_pass2", enc_pass2_kernel<B, RESID>, dim3((unsigned)grid), dim3(128), smem,
+                  st, false, pp);
+}
 }  // namespace
 
-size_t encode_workspace_bytes(int M, int K, int n_sal) { return encode_layout(M, K, n_sal).total; }
+size_t encode_workspace_bytes(int M, int K, int block, int n_sal) {
+  return encode_layout(M, K, block, n_sal).total;
+}
 
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
   const int M = a.M, K = a.K, B = a.block;
   const int nchunk = (M + kSsqChunk - 1) / kSsqChunk;
-  const EncodeLayout lay = encode_layout(M, K, a.n_sal);
+  const EncodeLayout lay = encode_layout(M, K, B, a.n_sal);
+  const Pass2Plan pl = pass2_plan(M, K, B, a.n_sal);
   char *ws = static_cast<char *>(a.workspace);
   auto *info = reinterpret_cast<unsigned long long *>(ws + lay.info);
-  auto *part = reinterpret_cast<double *>(ws + lay.part);
+  auto *ctr = reinterpret_cast<unsigned int *>(ws + lay.ctr);
+  auto *done = reinterpret_cast<unsigned int *>(ws + lay.done);
+  auto *gpart = reinterpret_cast<double *>(ws + lay.gpart);
   auto *score = reinterpret_cast<double *>(ws + lay.score);
-  auto *mask = reinterpret_cast<uint32_t *>(ws + lay.mask);
   auto *pref = reinterpret_cast<int32_t *>(ws + lay.pref);
-  auto *rowmax = reinterpret_cast<unsigned long long *>(ws + lay.rowmax);
-  auto *sv = reinterpret_cast<double *>(ws + lay.sv);
+  auto *sv = pl.smem ? nullptr : reinterpret_cast<double *>(ws + lay.sv);
   const double c = sqrt(1.0 / (double)B);
 
-  cudaError_t e = cudaMemsetAsync(info, 0, 4 * sizeof(unsigned long long), st);
+  cudaError_t e = cudaMemsetAsync(info, 0, lay.zero_bytes, st);
   if (e != cudaSuccess) return e;
   const int nkb = K / B;
-  const int P = B / 16, NG = (32 / P) * 4;
-  const long long pairs1 = (long long)nchunk * nkb;
-  dim3 g1((unsigned)((pairs1 + NG - 1) / NG));
+  const int NG = groups_per_cta(B);
+  dim3 g1((unsigned)(((nchunk + NG - 1) / NG) * nkb));
   if (B == 256)
     e = L.launch("enc_pass1", enc_pass1_kernel<256>, g1, dim3(128), 0, st, false,
-                 (const uint16_t *)a.W, M, K, c, part, info);
+                 (const uint16_t *)a.W, M, K, c, a.act_scale, gpart, score, done, info);
   else
     e = L.launch("enc_pass1", enc_pass1_kernel<128>, g1, dim3(128), 0, st, false,
-                 (const uint16_t *)a.W, M, K, c, part, info);
-  if (e != cudaSuccess) return e;
-  e = L.launch("enc_score", enc_score_kernel, dim3((K + kScoreCols - 1) / kScoreCols), dim3(256),
-               0, st, false,
-               (const double *)part, nchunk, K, a.act_scale, score, info);
+                 (const uint16_t *)a.W, M, K, c, a.act_scale, gpart, score, done, info);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = K <= kSelSmemKeys ? (size_t)K * sizeof(unsigned long long) : 0;
   e = L.launch("enc_select", enc_select_kernel, dim3(1), dim3(kSelThreads), sel_smem, st, false,
-               (const double *)score, K, a.n_sal, M, a.sal_idx, mask, pref, rowmax);
+               (const double *)score, K, a.n_sal, a.sal_idx, pref);
   if (e != cudaSuccess) return e;
-  const long long pairs2 = (long long)((M + kP2Rows - 1) / kP2Rows) * nkb;
-  dim3 g2((unsigned)((pairs2 + NG - 1) / NG));
-#define DVSSQ_PASS2(BB, RR)                                                                  \
-  L.launch("enc_pass2", enc_pass2_kernel<BB, RR>, g2, dim3(128), 0, st, false,            \
-           (const uint16_t *)a.W, M, K, a.n_sal, c, (const uint32_t *)mask,               \
-           (const int32_t *)pref, a.q4, a.s4, sv, rowmax, a.resid, info)
+
+  Pass2Params pp{};
+  pp.W = (const uint16_t *)a.W;
+  pp.M = M; pp.K = K; pp.n_sal = a.n_sal;
+  pp.R = pl.R; pp.rshift = pl.rshift; pp.ipg = pl.ipg; pp.ntiles = pl.ntiles;
+  pp.stash_smem = pl.smem ? 1 : 0;
+  pp.c = c;
+  pp.sal_idx = a.sal_idx; pp.sal_prefix = pref;
+  pp.q4 = a.q4; pp.s4 = a.s4; pp.q8 = a.q8; pp.s8 = a.s8; pp.resid = a.resid;
+  pp.sv = sv; pp.tile_ctr = ctr; pp.info = info;
   if (B == 256)
-    e = a.resid ? DVSSQ_PASS2(256, true) : DVSSQ_PASS2(256, false);
+    e = a.resid ? launch_pass2<256, true>(pp, pl.smem_bytes, st, L)
+                : launch_pass2<256, false>(pp, pl.smem_bytes, st, L);
   else
-    e = a.resid ? DVSSQ_PASS2(128, true) : DVSSQ_PASS2(128, false);
-#undef DVSSQ_PASS2
-  if (e != cudaSuccess) return e;
-  const long long items = a.n_sal > 0 ? (long long)M * (a.n_sal / 8) : (long long)M;
-  const long long g3 = std::min<long long>((items + 255) / 256, 148LL * 16);
-  const double vscale = B == 256 ? c : 1.0;
-  e = L.launch("enc_pass3", enc_pass3_kernel, dim3((unsigned)g3), dim3(256), 0, st, false,
-               (const double *)sv, (const unsigned long long *)rowmax, M, a.n_sal, vscale, a.q8,
-               a.s8, info);
+    e = a.resid ? launch_pass2<128, true>(pp, pl.smem_bytes, st, L)
+                : launch_pass2<128, false>(pp, pl.smem_bytes, st, L);
   if (e != cudaSuccess) return e;
   if (a.info_host != nullptr) {
     unsigned long long h[4];
@@ -650,12 +813,20 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
 cudaError_t prepare_encode_kernels() {
   cudaError_t e;
   for (const void *f :
-       {(const void *)enc_pass1_kernel<256>, (const void *)enc_pass1_kernel<128>,
-        (const void *)enc_pass2_kernel<256, false>, (const void *)enc_pass2_kernel<128, false>,
-        (const void *)enc_pass2_kernel<256, true>, (const void *)enc_pass2_kernel<128, true>})
+       {(const void *)enc_pass1_kernel<256>, (const void *)enc_pass1_kernel<128>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
+  for (const void *f :
+       {(const void *)enc_pass2_kernel<256, false>, (const void *)enc_pass2_kernel<128, false>,
+        (const void *)enc_pass2_kernel<256, true>, (const void *)enc_pass2_kernel<128, true>}) {
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kStashSmemMax)) != cudaSuccess)
+      return e;
+  }
   double recip[128];
   for (int m = 0; m < 128; ++m) recip[m] = 1.0 / (double)(128 + m);
   if ((e = cudaMemcpyToSymbol(kRecipMant, recip, sizeof(recip))) != cudaSuccess) return e;

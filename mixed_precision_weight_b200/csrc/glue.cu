@@ -10,12 +10,6 @@
 
 namespace dvssq {
 
-// 1 + erf(z) = erfc(-z): the complementary form keeps its relative accuracy
-// for negative v, where 1 + erf would cancel.
-__device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * erfcf(-v * 0.70710678118654752f);
-}
-
 __global__ void __launch_bounds__(256) gelu_mul_kernel(const uint16_t *__restrict__ g,
                                                        const uint16_t *__restrict__ u,
                                                        uint16_t *__restrict__ h, long long n) {

@@ -67,6 +67,35 @@ class Launcher {
     return e;
   }
 
+  // Cooperative launch: every CTA of the grid is resident at once (the
+  // kernel's blocks wait on one another through a grid barrier).
+  template <typename... KArgs, typename... Args>
+  cudaError_t launch_coop(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                          size_t smem, cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfileRecord rec{name, nullptr, nullptr};
+    if (profiling) {
+      cudaEventCreate(&rec.start);
+      cudaEventCreate(&rec.stop);
+      cudaEventRecord(rec.start, st);
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (profiling) {
+      cudaEventRecord(rec.stop, st);
+      pending.push_back(rec);
+    }
+    return e;
+  }
+
   template <typename... KArgs, typename... Args>
   cudaError_t launch(const char *name, void (*kernel)(KArgs...), dim3 grid, dim3 block,
                      size_t smem, cudaStream_t st, bool pdl, Args &&...args) {
@@ -91,9 +120,36 @@ struct EncodeArgs {
   int64_t *info_host;  // 3 counters or nullptr
   void *workspace;
 };
-size_t encode_workspace_bytes(int M, int K, int n_sal);
+size_t encode_workspace_bytes(int M, int K, int block, int n_sal);
 cudaError_t prepare_encode_kernels();
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L);
+
+// ------------------------------------------------------------- MLP stack ---
+struct StackMatDesc {           // one packed matrix (device pointers)
+  const uint8_t *q4;
+  const uint16_t *s4;
+  const int32_t *sal_idx;
+  const int8_t *q8;
+  const uint16_t *s8;
+  const uint16_t *U;
+  const uint16_t *V;
+  const float *vh;              // (V H_K) in FP32 [r][K], in the stack workspace
+  int M, K, block, n_sal, r;
+};
+struct StackLayerDesc {
+  StackMatDesc m[3];            // gate, up, down
+};
+struct StackShapeInfo {
+  int H, I, block;
+  size_t vh_floats;
+};
+bool stack_shape_info(const StackMatDesc *mats, int L, StackShapeInfo &si);
+size_t stack_workspace_bytes(const StackShapeInfo &si, int L);
+cudaError_t stack_prepare(StackMatDesc *mats, int L, const StackShapeInfo &si, void *ws,
+                          cudaStream_t st, Launcher &Lc);
+cudaError_t launch_mlp_stack(const StackMatDesc *mats, int L, const StackShapeInfo &si,
+                             const void *x, void *y, void *ws, cudaStream_t st, Launcher &Lc);
+cudaError_t prepare_stack_kernels();
 
 // ------------------------------------------------------------ activations -
 cudaError_t launch_gelu_mul(const uint16_t *g, const uint16_t *u, uint16_t *h, long long n,

@@ -7,4 +7,5 @@
 #include "decode.cu"
 #include "decode_row.cu"
 #include "prefill.cu"
+#include "stack.cu"
 #include "static_scratch.cu"

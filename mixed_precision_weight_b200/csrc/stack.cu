@@ -1,0 +1,699 @@
+// One token through a stack of gated-GELU MLP blocks ("Myric/Spark-X2.5-4B-
+// GGUF", "The model": GELU FFN; "Spark-X2.5-4B-ASHQ1-GGUF", "Architecture":
+// ffn_gate / ffn_up / ffn_down), every projection a DV-SSQ layer (MiniCPM5-
+// 2B-Hadamard-GSQ card, §2, with the Spark card's INT8 salient tier), in ONE
+// persistent cooperative kernel:
+//
+//     g = RN_bf16(gate(x)),  u = RN_bf16(up(x)),  h = RN_bf16(gelu(g) u),
+//     x <- RN_bf16(down(h)),   layer after layer.
+//
+// At one token every projection is a pure weight stream, and what a chain
+// of separate launches loses is the per-launch latency: the dependency wait,
+// the activation rotation and the partial-sum tail of every matrix.  Here the
+// weights of the whole stack stream without a break:
+//
+//   * CTA c (one per SM) owns fixed row ranges: rows [c I/G, (c+1) I/G) of
+//     every gate and up matrix and [c H/G, (c+1) H/G) of every down matrix.
+//     A row's dot product then lives in one CTA, gelu(g) u needs no exchange
+//     (gate and up rows coincide), and the CTA writes its slice of h or x.
+//   * Warp 0 streams the CTA's rows of every matrix of the stack, in order,
+//     through a ring of shared-memory slots (bulk copies of q4, s4, q8 and U
+//     rows per row tile).  Nothing it reads depends on activations, so it
+//     runs ahead across layer boundaries while the consumers wait.
+//   * The 15 consumer warps run two phases per block, each ending in a grid
+//     barrier: gate+up (x -> h) and down (h -> x).  After a barrier every CTA
+//     reads the whole input vector, rotates it (16-thread Kronecker FWHT,
+//     FP32) into int16 with one scale per 64 columns, requantises the
+//     salient entries per 64-entry chunk, and runs its rows as exact int32
+//     dot products (DP2A on bytes u = q + 8, minus 8 times the segment sums),
+//     scaled per group in FP32.
+//   * The rank-r term needs t = V (H x) = (V H) x for all of x.  With
+//     (V H) precomputed once in FP32, each CTA adds the share of the entries
+//     it produced, t_c = (V H)[:, own] x[own], at the end of the producing
+//     phase; after the barrier the consumers of t sum the G shares in a fixed
+//     order.  No extra barrier is needed for it.
+//
+// Every wait is bounded (mbarriers via mbar_wait, the grid barrier by
+// kWaitLimitCycles); a timeout sets the device error word and every warp
+// leaves at its next wait.
+#include "common.cuh"
+#include "fwht_group.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+
+namespace dvssq {
+
+constexpr int kStkWarps = 16;
+constexpr int kStkThreads = 32 * kStkWarps;
+constexpr int kStkCons = kStkWarps - 1;           // consumer warps (warp 0 streams weights)
+constexpr int kStkConsThreads = 32 * kStkCons;
+constexpr int kStkFwhtGroups = 20;                // 16-thread FWHT groups (10 warps)
+constexpr int kStkMaxRank = 32;                   // rank <= 32: one U t term per lane
+constexpr int kStkMaxSlots = 24;
+
+__device__ __forceinline__ void stk_consumer_sync() {
+  asm volatile("bar.sync 2, %0;" ::"n"(kStkConsThreads) : "memory");
+}
+
+struct StackParams {
+  const StackLayerDesc *layers;   // [L] in device memory
+  int L, H, I, G;
+  int tr_gu, tr_d;                // rows per tile of gate/up and of down
+  int slot_bytes, nslots;
+  int max_rank, max_nsal, rows_max, rounds_max;
+  const uint16_t *x;              // BF16 [H]
+  uint16_t *y;                    // BF16 [H]: the running hidden state, then the output
+  uint16_t *h;                    // BF16 [I]
+  float *tp;                      // t shares [3][kStkMaxRank][G]: gate, up, down
+  unsigned int *gbar;             // grid barrier counter, zero at launch
+  // shared-memory offsets from the 1024-aligned base
+  int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
+      o_scr, o_flag, smem_total;
+};
+
+// Row range of CTA c among G for M rows.
+__device__ __forceinline__ int stk_row(int c, int M, int G) {
+  return (int)(((long long)c * M) / G);
+}
+
+// Position of column j (0..7) of an 8-column segment in the DP2A order
+// {0, 2, 4, 6, 1, 3, 5, 7} of the stored int16 activations.
+__device__ __forceinline__ int stk_seg_pos(int j) { return (j & 1) ? 4 + (j >> 1) : (j >> 1); }
+
+__device__ __forceinline__ uint32_t stk_splice(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Bounded mbarrier wait that also gives up as soon as another warp of the CTA
+// has flagged an abort.
+__device__ __forceinline__ bool stk_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      set_error(kErrWaitMbarrier);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Activations in shared memory: 32-column units of int16 in four 16-byte
+// chunks (8 columns each, DP2A order inside), chunk i of unit v stored at
+// position i ^ ((v >> 1) & 3) so that lanes reading consecutive units hit
+// distinct banks.
+__device__ __forceinline__ int stk_chunk(int v, int i) { return i ^ ((v >> 1) & 3); }
+__device__ __forceinline__ int stk_xpos(int col) {
+  const int v = col >> 5;
+  return 32 * v + 8 * stk_chunk(v, (col >> 3) & 3) + stk_seg_pos(col & 7);
+}
+
+struct StkPhase {
+  int nm;                   // matrices of the phase (2: gate and up; 1: down)
+  StackMatDesc m[2];
+  int K, a, b, tr;          // input length, own rows [a, b), rows per tile
+  const uint16_t *src;      // input vector (BF16 [K])
+  int tslot[2];             // t-share slot of each matrix
+};
+
+template <int B>
+__global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t *ring = base + p.o_ring;
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + p.o_full);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(base + p.o_empty);
+  uint16_t *xi = reinterpret_cast<uint16_t *>(base + p.o_xi);   // [Kmax]: BF16 in, int16 out
+  float *xsc = reinterpret_cast<float *>(base + p.o_xsc);       // [Kmax / 64]
+  int *xsu = reinterpret_cast<int *>(base + p.o_xs8);           // [Kmax / 32] unit sums
+  uint16_t *xsal = reinterpret_cast<uint16_t *>(base + p.o_xs); // [2][max_nsal] int16
+  float *xss = reinterpret_cast<float *>(base + p.o_xss);       // [2][max_nsal / 32]
+  int *sidx = reinterpret_cast<int *>(base + p.o_sidx);         // [2][max_nsal]
+  float *tv = reinterpret_cast<float *>(base + p.o_t);          // [2][kStkMaxRank]
+  float *s8c = reinterpret_cast<float *>(base + p.o_s8);        // [2][rows_max]
+  float *red = reinterpret_cast<float *>(base + p.o_yv);        // [2][rows_max][rounds_max]
+  float *vals = reinterpret_cast<float *>(base + p.o_vh);       // [rows_max] produced values
+  float *scr = reinterpret_cast<float *>(base + p.o_scr);
+  volatile int *abort = reinterpret_cast<volatile int *>(base + p.o_flag);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, G = p.G;
+  const int gu_a = stk_row(c, p.I, G), gu_b = stk_row(c + 1, p.I, G);
+  const int d_a = stk_row(c, p.H, G), d_b = stk_row(c + 1, p.H, G);
+  const int NS = p.nslots;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kStkCons);
+    }
+    fence_mbarrier_init();
+    *abort = 0;
+  }
+  __syncthreads();
+
+  // ------------------------------- weight stream -------------------------------
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t seq = 0;
+      bool ok = true;
+      for (int l = 0; l < p.L && ok; ++l)
+        for (int mi = 0; mi < 3 && ok; ++mi) {
+          const StackMatDesc m = p.layers[l].m[mi];
+          const int a = mi < 2 ? gu_a : d_a, b = mi < 2 ? gu_b : d_b;
+          const int tr = mi < 2 ? p.tr_gu : p.tr_d;
+          const uint32_t kq = (uint32_t)m.K / 2, ks = (uint32_t)m.K / 32;
+          for (int i0 = a; i0 < b; i0 += tr, ++seq) {
+            const uint32_t nr = (uint32_t)min(tr, b - i0);
+            const int s = (int)(seq % (uint32_t)NS);
+            const uint32_t n = seq / (uint32_t)NS;
+            if (n > 0 && !stk_wait(&empty[s], (n - 1) & 1u, abort)) {
+              ok = false;
+              break;
+            }
+            uint8_t *dst = ring + (size_t)s * p.slot_bytes;
+            const uint32_t bq = nr * kq, bs = nr * ks, b8 = nr * (uint32_t)m.n_sal;
+            const uint32_t bu = nr * (uint32_t)m.r * 2u;
+            mbar_arrive_expect_tx(&full[s], bq + bs + b8 + bu);
+            bulk_g2s(dst, m.q4 + (size_t)i0 * kq, bq, &full[s]);
+            bulk_g2s(dst + bq, reinterpret_cast<const uint8_t *>(m.s4) + (size_t)i0 * ks, bs,
+                     &full[s]);
+            if (b8) bulk_g2s(dst + bq + bs, m.q8 + (size_t)i0 * m.n_sal, b8, &full[s]);
+            if (bu) bulk_g2s(dst + bq + bs + b8, m.U + (size_t)i0 * m.r, bu, &full[s]);
+          }
+        }
+      // copies still in flight land before the CTA may exit
+      const uint32_t issued = seq;
+      for (uint32_t q = issued > (uint32_t)NS ? issued - (uint32_t)NS : 0u; q < issued; ++q)
+        mbar_wait(&full[q % (uint32_t)NS], (q / (uint32_t)NS) & 1u);
+    }
+    return;
+  }
+
+  // --------------------------------- consumers ---------------------------------
+  const int ctid = tid - 32, cw = warp - 1;
+  const unsigned int err0 = *(volatile uint32_t *)&g_dvssq_error;
+  uint32_t seq = 0;            // ring position, in step with the producer
+  unsigned int nbar = 0;       // grid barriers passed
+  int rot = 0;                 // item -> warp rotation
+  const int rows_max = p.rows_max, rounds_max = p.rounds_max;
+  volatile int *s_live = abort + 1;
+
+  auto grid_sync = [&]() -> bool {
+    ++nbar;
+    stk_consumer_sync();
+    if (ctid == 0 && *abort == 0) {
+      __threadfence();
+      atomicAdd(p.gbar, 1u);
+      const long long t0 = clock64();
+      while (true) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.gbar) : "memory");
+        if (v >= nbar * (unsigned int)G) break;
+        if (*(volatile uint32_t *)&g_dvssq_error != err0 || clock64() - t0 > kWaitLimitCycles) {
+          set_error(kErrWaitGrid);
+          *abort = 1;
+          break;
+        }
+      }
+    }
+    // one thread decides, so that every consumer warp takes the same branches
+    if (ctid == 0) *s_live = *abort == 0;
+    stk_consumer_sync();
+    return *s_live != 0;
+  };
+
+  // t share of matrix m from the values this CTA produced: entries [a, a + n)
+  // of its input, vals[0..n).  tp[slot][k][c] = sum_i (V H)[k][a + i] vals[i]
+  auto t_share = [&](const StackMatDesc &m, int slot, int a, int n) {
+    for (int k = cw; k < m.r; k += kStkCons) {
+      const float *row = m.vh + (size_t)k * m.K + a;
+      float s = 0.0f;
+      for (int i = lane; i < n; i += 32) s = fmaf(__ldg(row + i), vals[i], s);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) p.tp[((size_t)slot * kStkMaxRank + k) * G + c] = s;
+    }
+  };
+
+  // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
+  for (int i = ctid; i < d_b - d_a; i += kStkConsThreads) vals[i] = bf16_bits_to_f32(p.x[d_a + i]);
+  stk_consumer_sync();
+  {
+    const StackMatDesc g0 = p.layers[0].m[0], u0 = p.layers[0].m[1];
+    t_share(g0, 0, d_a, d_b - d_a);
+    t_share(u0, 1, d_a, d_b - d_a);
+  }
+  bool live = grid_sync();
+
+  // ---- one phase: activations in, the CTA's rows of one or two matrices out
+  auto run_phase = [&](const StkPhase &ph) {
+    const int K = ph.K, nrows = ph.b - ph.a;
+    // input vector, scales of the salient tier, salient indices, t
+    for (int i = ctid; i < K / 8; i += kStkConsThreads)
+      reinterpret_cast<uint4 *>(xi)[i] = __ldcg(reinterpret_cast<const uint4 *>(ph.src) + i);
+    for (int mi = 0; mi < ph.nm; ++mi) {
+      const StackMatDesc &m = ph.m[mi];
+      for (int i = ctid; i < nrows; i += kStkConsThreads)
+        s8c[mi * rows_max + i] = m.n_sal > 0 ? bf16_bits_to_f32(__ldg(m.s8 + ph.a + i)) : 0.0f;
+      for (int e = ctid; e < m.n_sal; e += kStkConsThreads)
+        sidx[mi * p.max_nsal + e] = __ldg(m.sal_idx + e);
+    }
+    for (int q = cw; q < ph.nm * kStkMaxRank; q += kStkCons) {
+      const int mi = q / kStkMaxRank, k = q % kStkMaxRank;
+      if (k >= ph.m[mi].r) continue;
+      const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * G;
+      float s = 0.0f;
+      for (int i = lane; i < G; i += 32) s += __ldcg(src + i);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) tv[mi * kStkMaxRank + k] = s;
+    }
+    stk_consumer_sync();
+
+    // rotate x: BF16 in, int16 (unit/chunk layout) with one scale per 64 columns
+    {
+      constexpr int P = B / 16;
+      const int nblk = K / B;
+      const int grp = ctid / P, t = ctid % P;
+      const float cb = B == 256 ? 0.0625f : 0.08838834764831845f;
+      if (grp < kStkFwhtGroups)
+        for (int kb0 = 0; kb0 < nblk; kb0 += kStkFwhtGroups) {
+          const int kb = kb0 + grp;
+          const bool in = kb < nblk;
+          const uint16_t *blk = xi + (size_t)(in ? kb : 0) * B;
+          float v[16];
+#pragma unroll
+          for (int a = 0; a < 16; ++a) v[a] = in ? bf16_bits_to_f32(blk[P * a + t]) : 0.0f;
+          fwht_group<B>(v, scr + grp * GroupScratch<B>::kElems, t);
+          float mx = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v[j] *= cb;
+            mx = fmaxf(mx, fabsf(v[j]));
+          }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));   // 64 columns = 4 threads
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
+          int q[16], sum = 0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            q[j] = max(-32767, min(32767, __float2int_rn(v[j] * inv)));
+            sum += q[j];
+          }
+          sum += __shfl_xor_sync(0xffffffffu, sum, 1);           // 32-column unit = 2 threads
+          if (in) {
+            const int col0 = kb * B + 16 * t, vu = col0 >> 5;
+            uint4 w[2];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int *qq = q + 8 * hh;
+              w[hh].x = (uint32_t)(qq[0] & 0xFFFF) | ((uint32_t)qq[2] << 16);
+              w[hh].y = (uint32_t)(qq[4] & 0xFFFF) | ((uint32_t)qq[6] << 16);
+              w[hh].z = (uint32_t)(qq[1] & 0xFFFF) | ((uint32_t)qq[3] << 16);
+              w[hh].w = (uint32_t)(qq[5] & 0xFFFF) | ((uint32_t)qq[7] << 16);
+              const int ci = ((col0 >> 3) & 3) + hh;
+              *reinterpret_cast<uint4 *>(xi + 32 * vu + 8 * stk_chunk(vu, ci)) = w[hh];
+            }
+            if ((t & 3) == 0) xsc[col0 >> 6] = mx * (1.0f / 32767.0f);
+            if ((t & 1) == 0) xsu[vu] = sum;
+          }
+        }
+    }
+    stk_consumer_sync();
+
+    // salient activations of each matrix, requantised per 32-entry chunk
+    for (int mi = 0; mi < ph.nm; ++mi) {
+      const int ns = ph.m[mi].n_sal;
+      for (int j = cw; j < ns / 32; j += kStkCons) {
+        const int col = sidx[mi * p.max_nsal + 32 * j + lane];
+        float val = 0.0f;
+        if (col >= 0 && col < K) val = (float)(int16_t)xi[stk_xpos(col)] * xsc[col >> 6];
+        float mx = fabsf(val);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
+        const int qv = max(-32767, min(32767, __float2int_rn(val * inv)));
+        xsal[mi * p.max_nsal + 32 * j + 8 * stk_chunk(j, lane >> 3) + (lane & 7)] =
+            (uint16_t)(qv & 0xFFFF);
+        if (lane == 0) xss[mi * (p.max_nsal / 32) + j] = mx * (1.0f / 32767.0f);
+      }
+    }
+    stk_consumer_sync();
+
+    // the rows: items (row pair, round) of each tile, round-robin over the warps
+    for (int mi = 0; mi < ph.nm; ++mi) {
+      const StackMatDesc &m = ph.m[mi];
+      const int kq = m.K / 2, ks = m.K / 32, nu4 = m.K / 32, nu8 = m.n_sal / 32;
+      const int rounds = (nu4 + nu8 + 31) / 32;
+      const float *tvm = tv + mi * kStkMaxRank;
+      const uint16_t *xsm = xsal + mi * p.max_nsal;
+      const float *xssm = xss + mi * (p.max_nsal / 32);
+      for (int i0 = ph.a; i0 < ph.b; i0 += ph.tr, ++seq) {
+        const int nr = min(ph.tr, ph.b - i0), npair = (nr + 1) / 2;
+        const int s = (int)(seq % (uint32_t)NS);
+        const bool got =
+            __all_sync(0xffffffffu, stk_wait(&full[s], (seq / (uint32_t)NS) & 1u, abort));
+        const uint8_t *slot = ring + (size_t)s * p.slot_bytes;
+        const uint8_t *q4s = slot, *s4s = slot + nr * kq, *q8s = s4s + nr * ks;
+        const uint8_t *us = q8s + nr * m.n_sal;
+        const int items = npair * rounds;
+        for (int it = (cw - rot + kStkCons * 64) % kStkCons; got && it < items; it += kStkCons) {
+          const int pr = it / rounds, rd = it - pr * rounds;
+          const int r0 = 2 * pr, r1 = r0 + 1;
+          const bool two = r1 < nr;
+          const int task = 32 * rd + lane;
+          float acc0 = 0.0f, acc1 = 0.0f;
+          if (task < nu4) {
+            const int v = task, g = v >> 1;
+            uint4 xa[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
+            const int bias = 8 * xsu[v];
+            const float sc = xsc[g];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              if (rr == 1 && !two) break;
+              const int rl = r0 + rr;
+              const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl * kq + 16 * v);
+              const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+              int d = 0;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
+                const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+                d = __dp2a_lo((int)xa[i].x, (int)L, d);
+                d = __dp2a_hi((int)xa[i].y, (int)L, d);
+                d = __dp2a_lo((int)xa[i].z, (int)Hh, d);
+                d = __dp2a_hi((int)xa[i].w, (int)Hh, d);
+              }
+              const float s4v =
+                  bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl * ks)[g]);
+              const float f = s4v * sc * (float)(d - bias);
+              if (rr == 0) acc0 = f; else acc1 = f;
+            }
+          } else if (task < nu4 + nu8) {
+            const int j = task - nu4;
+            uint4 xa[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
+            const float sc = xssm[j];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              if (rr == 1 && !two) break;
+              const int rl = r0 + rr;
+              const uint4 qa = *reinterpret_cast<const uint4 *>(q8s + (size_t)rl * m.n_sal + 32 * j);
+              const uint4 qb =
+                  *reinterpret_cast<const uint4 *>(q8s + (size_t)rl * m.n_sal + 32 * j + 16);
+              const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+              int d = 0;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                d = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d);
+                d = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d);
+                d = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d);
+                d = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d);
+              }
+              const float f = s8c[mi * rows_max + (i0 - ph.a) + rl] * sc * (float)d;
+              if (rr == 0) acc0 = f; else acc1 = f;
+            }
+          }
+          if (rd == 0 && lane < m.r) {
+            const uint16_t *ur = reinterpret_cast<const uint16_t *>(us);
+            acc0 = fmaf(bf16_bits_to_f32(ur[r0 * m.r + lane]), tvm[lane], acc0);
+            if (two) acc1 = fmaf(bf16_bits_to_f32(ur[r1 * m.r + lane]), tvm[lane], acc1);
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) {
+            acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+            acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+          }
+          if (lane == 0) {
+            float *rw = red + ((size_t)mi * rows_max + (i0 - ph.a) + r0) * rounds_max + rd;
+            rw[0] = acc0;
+            if (two) rw[rounds_max] = acc1;
+          }
+        }
+        rot = (rot + items) % kStkCons;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    stk_consumer_sync();
+    // row results (rounds in order) back into red[mi][row][0]
+    for (int mi = 0; mi < ph.nm; ++mi) {
+      const int rounds = (ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32;
+      for (int i = ctid; i < nrows; i += kStkConsThreads) {
+        float *rw = red + ((size_t)mi * rows_max + i) * rounds_max;
+        float s = rw[0];
+        for (int rd = 1; rd < rounds; ++rd) s += rw[rd];
+        rw[0] = s;
+      }
+    }
+    stk_consumer_sync();
+  };
+
+  // ---- the blocks: gate+up (x -> h), then down (h -> x)
+  for (int l = 0; l < p.L; ++l) {
+    const StackLayerDesc &Ld = p.layers[l];
+    {
+      StkPhase ph;
+      ph.nm = 2;
+      ph.m[0] = Ld.m[0];
+      ph.m[1] = Ld.m[1];
+      ph.K = p.H;
+      ph.a = gu_a;
+      ph.b = gu_b;
+      ph.tr = p.tr_gu;
+      ph.src = l == 0 ? p.x : p.y;
+      ph.tslot[0] = 0;
+      ph.tslot[1] = 1;
+      if (live) run_phase(ph);
+      // h = RN_bf16(gelu(g) u), g and u rounded to BF16 first
+      const int n = gu_b - gu_a;
+      for (int i = ctid; i < n && live; i += kStkConsThreads) {
+        const float gv = bf16_bits_to_f32(f32_to_bf16_rn_bits(red[(size_t)i * rounds_max]));
+        const float uv =
+            bf16_bits_to_f32(f32_to_bf16_rn_bits(red[((size_t)rows_max + i) * rounds_max]));
+        const uint16_t hb = f32_to_bf16_rn_bits(gelu_erf(gv) * uv);
+        p.h[gu_a + i] = hb;
+        vals[i] = bf16_bits_to_f32(hb);
+      }
+      stk_consumer_sync();
+      if (live) t_share(Ld.m[2], 2, gu_a, n);
+      live = grid_sync() && live;
+    }
+    {
+      StkPhase ph;
+      ph.nm = 1;
+      ph.m[0] = Ld.m[2];
+      ph.K = p.I;
+      ph.a = d_a;
+      ph.b = d_b;
+      ph.tr = p.tr_d;
+      ph.src = p.h;
+      ph.tslot[0] = 2;
+      if (live) run_phase(ph);
+      const int n = d_b - d_a;
+      for (int i = ctid; i < n && live; i += kStkConsThreads) {
+        const uint16_t xb = f32_to_bf16_rn_bits(red[(size_t)i * rounds_max]);
+        p.y[d_a + i] = xb;
+        vals[i] = bf16_bits_to_f32(xb);
+      }
+      stk_consumer_sync();
+      if (l + 1 < p.L) {
+        if (live) {
+          t_share(p.layers[l + 1].m[0], 0, d_a, n);
+          t_share(p.layers[l + 1].m[1], 1, d_a, n);
+        }
+        live = grid_sync() && live;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------- host ---
+namespace {
+constexpr int kStkSlotTarget = 16384;      // bytes of weights per ring slot, about
+constexpr int kStkSmemLimit = 232448;      // opt-in shared memory per CTA (227 KB)
+
+int stk_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int stk_row_bytes(const StackMatDesc &m) { return m.K / 2 + m.K / 32 + m.n_sal + 2 * m.r; }
+
+struct StkWs {
+  size_t desc, vh, tp, gbar, h, total;
+};
+StkWs stk_ws_layout(const StackShapeInfo &si, int L, int G) {
+  StkWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return o;
+  };
+  w.desc = take((size_t)L * sizeof(StackLayerDesc));
+  w.vh = take(si.vh_floats * sizeof(float));
+  w.tp = take((size_t)3 * kStkMaxRank * G * sizeof(float));
+  w.gbar = take(256);
+  w.h = take((size_t)si.I * 2);
+  w.total = off;
+  return w;
+}
+
+bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &p) {
+  const int L = (int)Ls.size();
+  p.L = L;
+  p.H = Ls[0].m[2].M;
+  p.I = Ls[0].m[0].M;
+  p.G = G;
+  int rb_gu = 0, rb_d = 0, max_rank = 0, max_nsal = 0, rounds_max = 1;
+  for (const auto &Ld : Ls)
+    for (int mi = 0; mi < 3; ++mi) {
+      const StackMatDesc &m = Ld.m[mi];
+      if (mi < 2) rb_gu = std::max(rb_gu, stk_row_bytes(m));
+      else rb_d = std::max(rb_d, stk_row_bytes(m));
+      max_rank = std::max(max_rank, m.r);
+      max_nsal = std::max(max_nsal, m.n_sal);
+      rounds_max = std::max(rounds_max, (m.K / 32 + m.n_sal / 32 + 31) / 32);
+    }
+  p.tr_gu = std::max(2, (kStkSlotTarget / rb_gu) & ~1);
+  p.tr_d = std::max(2, (kStkSlotTarget / rb_d) & ~1);
+  p.slot_bytes = (std::max(p.tr_gu * rb_gu, p.tr_d * rb_d) + 127) & ~127;
+  p.max_rank = max_rank;
+  p.max_nsal = std::max(max_nsal, 32);
+  p.rows_max = (std::max(p.H, p.I) + G - 1) / G + 1;
+  p.rounds_max = rounds_max;
+  const int Kmax = std::max(p.H, p.I);
+  int off = 0;
+  auto take = [&](int bytes) {
+    const int o = off;
+    off += (bytes + 127) & ~127;
+    return o;
+  };
+  p.o_xi = take(Kmax * 2);
+  p.o_xsc = take(Kmax / 64 * 4);
+  p.o_xs8 = take(Kmax / 32 * 4);
+  p.o_xs = take(2 * p.max_nsal * 2);
+  p.o_xss = take(2 * (p.max_nsal / 32) * 4);
+  p.o_sidx = take(2 * p.max_nsal * 4);
+  p.o_t = take(2 * kStkMaxRank * 4);
+  p.o_s8 = take(2 * p.rows_max * 4);
+  p.o_yv = take(2 * p.rows_max * p.rounds_max * 4);
+  p.o_vh = take(p.rows_max * 4);
+  p.o_scr = take(kStkFwhtGroups * (B == 256 ? GroupScratch<256>::kElems : GroupScratch<128>::kElems) * 4);
+  p.o_flag = take(16);
+  const int fixed = off;
+  const int room = kStkSmemLimit - 1024 - fixed - 2 * kStkMaxSlots * 8 - 128;
+  p.nslots = std::min(kStkMaxSlots, room / p.slot_bytes);
+  if (p.nslots < 2) return false;
+  p.o_full = take(p.nslots * 8);
+  p.o_empty = take(p.nslots * 8);
+  off = (off + 1023) & ~1023;
+  p.o_ring = off;
+  off += p.nslots * p.slot_bytes;
+  p.smem_total = off + 1024;
+  return p.smem_total <= kStkSmemLimit;
+}
+}  // namespace
+
+bool stack_shape_info(const StackMatDesc *mats, int L, StackShapeInfo &si) {
+  if (L < 1) return false;
+  const int I = mats[0].M, H = mats[0].K, B = mats[0].block;
+  if (H % 512 != 0 || I % 512 != 0) return false;
+  size_t vh = 0;
+  for (int l = 0; l < L; ++l)
+    for (int mi = 0; mi < 3; ++mi) {
+      const StackMatDesc &m = mats[3 * l + mi];
+      const int M = mi < 2 ? I : H, K = mi < 2 ? H : I;
+      if (m.M != M || m.K != K || m.block != B) return false;
+      if (m.r < 0 || m.r > kStkMaxRank || m.r % 8 != 0) return false;
+      if (m.n_sal % 32 != 0 || m.n_sal > K) return false;
+      vh += (size_t)m.r * K;
+    }
+  si.H = H;
+  si.I = I;
+  si.block = B;
+  si.vh_floats = vh;
+  return true;
+}
+
+size_t stack_workspace_bytes(const StackShapeInfo &si, int L) {
+  return stk_ws_layout(si, L, std::max(1, stk_sm_count())).total;
+}
+
+cudaError_t stack_prepare(StackMatDesc *mats, int L, const StackShapeInfo &si, void *ws,
+                          cudaStream_t st, Launcher &Lc) {
+  const int G = stk_sm_count();
+  if (G <= 0) return cudaErrorNoDevice;
+  const StkWs w = stk_ws_layout(si, L, G);
+  char *base = static_cast<char *>(ws);
+  float *vh = reinterpret_cast<float *>(base + w.vh);
+  std::vector<StackLayerDesc> Ls((size_t)L);
+  for (int l = 0; l < L; ++l)
+    for (int mi = 0; mi < 3; ++mi) {
+      StackMatDesc m = mats[3 * l + mi];
+      if (m.r > 0) {
+        // (V H_K) row by row: the blockwise FWHT of each row of V (H is symmetric)
+        cudaError_t e = launch_fwht(m.V, vh, m.r, m.K, m.block, st, Lc);
+        if (e != cudaSuccess) return e;
+        m.vh = vh;
+        vh += (size_t)m.r * m.K;
+      } else {
+        m.vh = nullptr;
+      }
+      Ls[(size_t)l].m[mi] = m;
+    }
+  cudaError_t e = cudaMemcpyAsync(base + w.desc, Ls.data(), Ls.size() * sizeof(StackLayerDesc),
+                                  cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);     // Ls is a host temporary
+}
+
+cudaError_t launch_mlp_stack(const StackMatDesc *mats, int L, const StackShapeInfo &si,
+                             const void *x, void *y, void *ws, cudaStream_t st, Launcher &Lc) {
+  const int G = stk_sm_count();
+  if (G <= 0) return cudaErrorNoDevice;
+  std::vector<StackLayerDesc> Ls((size_t)L);
+  for (int l = 0; l < L; ++l)
+    for (int mi = 0; mi < 3; ++mi) Ls[(size_t)l].m[mi] = mats[3 * l + mi];
+  StackParams p{};
+  if (!stk_plan(Ls, G, si.block, p)) return cudaErrorNotSupported;
+  const StkWs w = stk_ws_layout(si, L, G);
+  char *base = static_cast<char *>(ws);
+  p.layers = reinterpret_cast<const StackLayerDesc *>(base + w.desc);
+  p.x = static_cast<const uint16_t *>(x);
+  p.y = static_cast<uint16_t *>(y);
+  p.h = reinterpret_cast<uint16_t *>(base + w.h);
+  p.tp = reinterpret_cast<float *>(base + w.tp);
+  p.gbar = reinterpret_cast<unsigned int *>(base + w.gbar);
+  cudaError_t e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned int), st);
+  if (e != cudaSuccess) return e;
+  if (si.block == 256)
+    return Lc.launch_coop("mlp_stack", mlp_stack_kernel<256>, dim3(G), dim3(kStkThreads),
+                          (size_t)p.smem_total, st, p);
+  return Lc.launch_coop("mlp_stack", mlp_stack_kernel<128>, dim3(G), dim3(kStkThreads),
+                        (size_t)p.smem_total, st, p);
+}
+
+cudaError_t prepare_stack_kernels() {
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(mlp_stack_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kStkSmemLimit)) != cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(mlp_stack_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kStkSmemLimit);
+}
+
+}  // namespace dvssq

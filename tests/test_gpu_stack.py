@@ -1,0 +1,130 @@
+"""The one-launch MLP stack (dvssq_mlp_stack_forward) against the fp64 oracle
+and against the chain of single-layer GPU calls.
+
+- Reduced Spark-shaped stacks (hidden 512, intermediate 1024, b = 256) encoded
+  by the GPU encoder with the oracle's SVD factors, two ranks: the fused
+  output against the oracle's mlp_block applied layer after layer
+  (reading R10), and against the GPU chain gate / up / gelu_mul / down.
+- Full Spark shapes (hidden 2560, intermediate 10240, rank 16 and 24): the
+  fused output against the GPU chain of the same packed layers.
+Both sides round g, u, h and each block output to BF16; the fused kernel
+differs from the chain only in FP32 summation order and in forming the
+rank-r input as (V H) x, so outputs agree up to BF16 rounding flips.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import dvssq_oracle as O
+from mixed_precision_weight_b200 import synth
+
+from test_gpu_parity import check_codes, f64, gpu_encode
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dv():
+    import mixed_precision_weight_b200 as pkg
+    return pkg.binding
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def chain(dv, layers, x):
+    cur = x
+    for (sg, pg), (su, pu), (sd, pd) in layers:
+        g = dv.dvssq_linear_forward(sg, pg, cur, y_dtype=dv.Y_BF16)
+        u = dv.dvssq_linear_forward(su, pu, cur, y_dtype=dv.Y_BF16)
+        cur = dv.dvssq_linear_forward(sd, pd, dv.dvssq_gelu_mul(g, u), y_dtype=dv.Y_BF16)
+    return cur
+
+
+def small_stack(dv, L, H, I, ranks, seed):
+    layers, encs = [], []
+    for l in range(L):
+        mats, es = [], []
+        for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
+            s = seed + 10 * l + which
+            W = synth.weight(M, K, seed=s, n_outlier_cols=2, outlier_scale=15.0)
+            act = synth.act_scale(K, seed=s)
+            enc = O.encode(f64(W), act.numpy(), 256, ranks[l])
+            U = torch.from_numpy(enc["U"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
+            V = torch.from_numpy(enc["V"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
+            shape, packed, _, _ = gpu_encode(dv, W, act, 256, ranks[l], U=U, V=V)
+            check_codes(shape, packed, enc)
+            mats.append((shape, packed))
+            es.append(enc)
+        layers.append(tuple(mats))
+        encs.append(es)
+    return layers, encs
+
+
+@pytest.mark.parametrize("ranks", [(8, 16), (16, 8)])
+def test_stack_matches_oracle_and_chain(dv, ranks):
+    H, I = 512, 1024
+    layers, encs = small_stack(dv, 2, H, I, ranks, seed=31 + ranks[0])
+    x = synth.activations(1, H, seed=9, n_outlier=3, outlier_scale=25.0)
+    stack = dv.MlpStack(layers)
+    y = stack.forward(x.cuda())
+    torch.cuda.synchronize()
+    assert dv.dvssq_device_error(clear=True) == 0
+    ref = f64(x)
+    for eg, eu, ed in encs:
+        ref = O.rn_bf16(O.mlp_block(eg, eu, ed, ref))
+    got = f64(y)
+    assert rel_l2(got, ref) <= 3e-2, rel_l2(got, ref)
+    ch = f64(chain(dv, layers, x.cuda()))
+    assert rel_l2(got, ch) <= 1e-2, rel_l2(got, ch)
+    # repeatable: the same inputs give the same bits
+    assert torch.equal(stack.forward(x.cuda()), y)
+
+
+def test_stack_output_may_alias_input(dv):
+    H, I = 512, 1024
+    layers, _ = small_stack(dv, 1, H, I, (8,), seed=77)
+    stack = dv.MlpStack(layers)
+    x = synth.activations(1, H, seed=4).cuda()
+    y = stack.forward(x)
+    xx = x.clone()
+    stack.forward(xx, y=xx)
+    assert torch.equal(xx, y)
+
+
+def test_stack_full_spark_shapes_match_chain(dv):
+    H, I = 2560, 10240
+    layers = []
+    for l in range(2):
+        r = (16, 24)[l]
+        mats = []
+        for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
+            seed = synth.layer_seed(1, l, which)
+            shape = dv.Shape.make(M, K, 256, r)
+            W = synth.weight_device(M, K, seed, "cuda", n_outlier_cols=max(1, K // 1000),
+                                    outlier_scale=15.0)
+            act = synth.act_scale(K, seed).cuda()
+            U, V = synth.lowrank_factors(M, K, r, seed=seed + 17)
+            packed = dv.PackedWeights.empty(shape, "cuda", U=U.cuda(), V=V.cuda())
+            dv.dvssq_encode(shape, W, act, packed)
+            mats.append((shape, packed))
+        layers.append(tuple(mats))
+    x = synth.activations(1, H, seed=3, n_outlier=13, outlier_scale=25.0).cuda()
+    stack = dv.MlpStack(layers)
+    y = stack.forward(x)
+    torch.cuda.synchronize()
+    assert dv.dvssq_device_error(clear=True) == 0
+    ch = chain(dv, layers, x)
+    assert rel_l2(f64(y), f64(ch)) <= 1e-2, rel_l2(f64(y), f64(ch))
+
+
+def test_stack_rejects_bad_layers(dv):
+    H, I = 512, 1024
+    layers, _ = small_stack(dv, 1, H, I, (8,), seed=5)
+    (sg, pg), (su, pu), (sd, pd) = layers[0]
+    bad = [((sd, pd), (su, pu), (sg, pg))]           # gate / down swapped
+    with pytest.raises(dv.DvssqError):
+        dv.dvssq_mlp_stack_workspace_size(bad)
+    with pytest.raises(dv.DvssqError):
+        dv.dvssq_mlp_stack_workspace_size([])
