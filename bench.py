@@ -436,6 +436,7 @@ class StackStep:
 
     name = "spark_mlp_stack_36x(gate,up,down)_T1"
     graph_slots = 1
+    n_layers = 36     # the full model; --layers sets fewer for profiling
     fused = True      # one cooperative launch per token (dvssq_mlp_stack_forward)
 
     def __init__(self, dv, synth, torch, rank_id, device):
@@ -444,7 +445,8 @@ class StackStep:
         self.H, self.I = H, I
         self.layers = []
         ws = 0
-        for l in range(36):
+        self.nl = self.n_layers
+        for l in range(self.nl):
             r = synth.stack_rank(l)
             mats = []
             for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
@@ -498,7 +500,7 @@ class StackStep:
                    for sh, _ in mats)
 
     def launches_per_step(self):
-        return 1 if self.fused else 36 * (3 * 2 + 1)
+        return 1 if self.fused else self.nl * (3 * 2 + 1)
 
     def kernel_work(self, name):
         if name == "mlp_stack":
@@ -513,12 +515,12 @@ class StackStep:
         return sum(per) / len(per)
 
     def config(self):
-        return {"workload": self.name, "layers": 36, "hidden": self.H, "intermediate": self.I,
+        return {"workload": self.name, "layers": self.nl, "hidden": self.H, "intermediate": self.I,
                 "block": 256, "rank": "16 (layers 0-13, 29-35), 24 (14-28)",
                 "n_sal": "K/8 per matrix", "tokens": 1,
-                "step": ("dvssq_mlp_stack_forward: the 36 blocks in one cooperative launch"
+                "step": (f"dvssq_mlp_stack_forward: the {self.nl} blocks in one cooperative launch"
                          if self.fused else
-                         "36 x (dvssq_linear_forward gate, up -> dvssq_gelu_mul -> down)")
+                         f"{self.nl} x (dvssq_linear_forward gate, up -> dvssq_gelu_mul -> down)")
                         + ", BF16 hidden states, one CUDA graph per token",
                 "packed_bytes_per_token": self.bytes_per_step(),
                 "l2": "1.9 GB of packed weights per token > 126 MB L2",
@@ -600,6 +602,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--layers", type=int, default=36,
+                    help="blocks of the stack workloads (36 is the full model; fewer for profiling)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -621,6 +625,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device(device))
+    StackStep.n_layers = args.layers
     work = WORKLOADS[args.workload](dv, synth, torch, rank, device)
     unit = getattr(work, "unit", "GB/s")
     W = max(3, args.warmup)

@@ -41,6 +41,7 @@
 #include "kernels.h"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace dvssq {
 
@@ -62,6 +63,7 @@ struct StackParams {
   int tr_gu, tr_d;                // rows per tile of gate/up and of down
   int slot_bytes, nslots;
   int max_rank, max_nsal, rows_max, rounds_max;
+  int rg_gu, rg_d;                // rows per item of gate/up and of down
   const uint16_t *x;              // BF16 [H]
   uint16_t *y;                    // BF16 [H]: the running hidden state, then the output
   uint16_t *h;                    // BF16 [I]
@@ -69,8 +71,12 @@ struct StackParams {
   unsigned int *gbar;             // grid barrier counter, zero at launch
   // shared-memory offsets from the 1024-aligned base
   int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
-      o_scr, o_flag, smem_total;
+      o_scr, o_flag, o_tq, o_vhs, smem_total;
 };
+
+// Entries per matrix of the BF16 s8 staging: the own rows plus the partial
+// 16-byte words at both ends, rounded up to whole words.
+__host__ __device__ constexpr int stk_s8_stride(int rows_max) { return (rows_max + 16 + 7) & ~7; }
 
 // Row range of CTA c among G for M rows.
 __device__ __forceinline__ int stk_row(int c, int M, int G) {
@@ -116,10 +122,30 @@ __device__ __forceinline__ int stk_xpos(int col) {
 struct StkPhase {
   int nm;                   // matrices of the phase (2: gate and up; 1: down)
   StackMatDesc m[2];
-  int K, a, b, tr;          // input length, own rows [a, b), rows per tile
+  int K, a, b, tr, rg;      // input length, own rows [a, b), rows per tile, rows per item
   const uint16_t *src;      // input vector (BF16 [K])
   int tslot[2];             // t-share slot of each matrix
+  // the matrices that consume this phase's output: their (V H) columns [a, b)
+  // give this CTA's t shares
+  int nout;
+  const float *ovh[2];
+  int oK[2], orank[2], oslot[2];
 };
+
+__device__ __forceinline__ void stk_cp_async4(void *smem, const void *gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void stk_cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void stk_cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void stk_cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
 
 template <int B>
 __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackParams p) {
@@ -135,7 +161,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   float *xss = reinterpret_cast<float *>(base + p.o_xss);       // [2][max_nsal / 32]
   int *sidx = reinterpret_cast<int *>(base + p.o_sidx);         // [2][max_nsal]
   float *tv = reinterpret_cast<float *>(base + p.o_t);          // [2][kStkMaxRank]
-  float *s8c = reinterpret_cast<float *>(base + p.o_s8);        // [2][rows_max]
+  uint16_t *s8c = reinterpret_cast<uint16_t *>(base + p.o_s8);  // [2][s8_stride] BF16
   float *red = reinterpret_cast<float *>(base + p.o_yv);        // [2][rows_max][rounds_max]
   float *vals = reinterpret_cast<float *>(base + p.o_vh);       // [rows_max] produced values
   float *scr = reinterpret_cast<float *>(base + p.o_scr);
@@ -201,14 +227,25 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   unsigned int nbar = 0;       // grid barriers passed
   int rot = 0;                 // item -> warp rotation
   const int rows_max = p.rows_max, rounds_max = p.rounds_max;
+  // per-matrix BF16 staging of s8: 16-byte words covering the own rows, so a
+  // multiple of 8 entries (each slice starts 16-byte aligned)
+  const int s8_stride = stk_s8_stride(rows_max);
   volatile int *s_live = abort + 1;
+  float *tq = reinterpret_cast<float *>(base + p.o_tq);         // t-share partial sums
+  float *vhs = reinterpret_cast<float *>(base + p.o_vhs);       // (V H) columns of own outputs
 
-  auto grid_sync = [&]() -> bool {
+  // Split grid barrier: a CTA arrives as soon as its outputs are written,
+  // prefetches what the next phase needs from the weights, then waits.
+  auto grid_arrive = [&]() {
     ++nbar;
     stk_consumer_sync();
     if (ctid == 0 && *abort == 0) {
       __threadfence();
       atomicAdd(p.gbar, 1u);
+    }
+  };
+  auto grid_wait = [&]() -> bool {
+    if (ctid == 0 && *abort == 0) {
       const long long t0 = clock64();
       while (true) {
         unsigned int v;
@@ -227,53 +264,123 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     return *s_live != 0;
   };
 
-  // t share of matrix m from the values this CTA produced: entries [a, a + n)
-  // of its input, vals[0..n).  tp[slot][k][c] = sum_i (V H)[k][a + i] vals[i]
-  auto t_share = [&](const StackMatDesc &m, int slot, int a, int n) {
-    for (int k = cw; k < m.r; k += kStkCons) {
-      const float *row = m.vh + (size_t)k * m.K + a;
-      float s = 0.0f;
-      for (int i = lane; i < n; i += 32) s = fmaf(__ldg(row + i), vals[i], s);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) p.tp[((size_t)slot * kStkMaxRank + k) * G + c] = s;
+  // phase descriptors: layer l, kind 0 = gate and up (x -> h), 1 = down (h -> x)
+  auto make_phase = [&](int l, int kind) {
+    StkPhase ph;
+    const StackLayerDesc *Ld = p.layers + l;
+    if (kind == 0) {
+      ph.nm = 2;
+      ph.m[0] = Ld->m[0];
+      ph.m[1] = Ld->m[1];
+      ph.K = p.H;
+      ph.a = gu_a;
+      ph.b = gu_b;
+      ph.tr = p.tr_gu;
+      ph.rg = p.rg_gu;
+      ph.src = l == 0 ? p.x : p.y;
+      ph.tslot[0] = 0;
+      ph.tslot[1] = 1;
+      ph.nout = 1;
+      ph.ovh[0] = Ld->m[2].vh;
+      ph.oK[0] = Ld->m[2].K;
+      ph.orank[0] = Ld->m[2].r;
+      ph.oslot[0] = 2;
+    } else {
+      ph.nm = 1;
+      ph.m[0] = Ld->m[2];
+      ph.K = p.I;
+      ph.a = d_a;
+      ph.b = d_b;
+      ph.tr = p.tr_d;
+      ph.rg = p.rg_d;
+      ph.src = p.h;
+      ph.tslot[0] = 2;
+      ph.nout = l + 1 < p.L ? 2 : 0;
+      for (int j = 0; j < ph.nout; ++j) {
+        ph.ovh[j] = Ld[1].m[j].vh;
+        ph.oK[j] = Ld[1].m[j].K;
+        ph.orank[j] = Ld[1].m[j].r;
+        ph.oslot[j] = j;
+      }
     }
+    return ph;
   };
 
-  // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
-  for (int i = ctid; i < d_b - d_a; i += kStkConsThreads) vals[i] = bf16_bits_to_f32(p.x[d_a + i]);
-  stk_consumer_sync();
-  {
-    const StackMatDesc g0 = p.layers[0].m[0], u0 = p.layers[0].m[1];
-    t_share(g0, 0, d_a, d_b - d_a);
-    t_share(u0, 1, d_a, d_b - d_a);
-  }
-  bool live = grid_sync();
+  // weight-side data of a phase, loaded while the grid barrier is pending:
+  // INT8 scales of the own rows, salient indices, (V H) columns for the t shares
+  auto prefetch = [&](const StkPhase &ph) {
+    const int n = ph.b - ph.a;
+    for (int mi = 0; mi < ph.nm; ++mi) {
+      const StackMatDesc &m = ph.m[mi];
+      if (m.n_sal == 0) continue;
+      // the 16-byte words of s8 that hold rows [a, b) (M is a multiple of 8)
+      const int w0 = ph.a >> 3, w1 = (ph.b + 7) >> 3;
+      for (int w = w0 + ctid; w < w1; w += kStkConsThreads)
+        stk_cp_async16(s8c + mi * s8_stride + 8 * (w - w0), m.s8 + 8 * w);
+      for (int e = 4 * ctid; e < m.n_sal; e += 4 * kStkConsThreads)
+        stk_cp_async16(sidx + mi * p.max_nsal + e, m.sal_idx + e);
+    }
+    int off = 0;
+    for (int j = 0; j < ph.nout; ++j) {
+      for (int q = ctid; q < ph.orank[j] * n; q += kStkConsThreads) {
+        const int k = q / n, i = q - k * n;
+        stk_cp_async4(vhs + off + q, ph.ovh[j] + (size_t)k * ph.oK[j] + ph.a + i);
+      }
+      off += ph.orank[j] * n;
+    }
+    stk_cp_async_commit();
+  };
+
+  // this CTA's t shares for the consumers of its outputs vals[0..n)
+  auto t_share_out = [&](const StkPhase &ph) {
+    const int n = ph.b - ph.a;
+    int off = 0;
+    for (int j = 0; j < ph.nout; ++j) {
+      for (int k = cw; k < ph.orank[j]; k += kStkCons) {
+        const float *row = vhs + off + k * n;
+        float s = 0.0f;
+        for (int i = lane; i < n; i += 32) s = fmaf(row[i], vals[i], s);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) p.tp[((size_t)ph.oslot[j] * kStkMaxRank + k) * G + c] = s;
+      }
+      off += ph.orank[j] * n;
+    }
+  };
 
   // ---- one phase: activations in, the CTA's rows of one or two matrices out
   auto run_phase = [&](const StkPhase &ph) {
     const int K = ph.K, nrows = ph.b - ph.a;
-    // input vector, scales of the salient tier, salient indices, t
+    // input vector and t: the G shares of each (matrix, k), NP parts per
+    // pair summed in parallel, then the parts in order
     for (int i = ctid; i < K / 8; i += kStkConsThreads)
       reinterpret_cast<uint4 *>(xi)[i] = __ldcg(reinterpret_cast<const uint4 *>(ph.src) + i);
-    for (int mi = 0; mi < ph.nm; ++mi) {
-      const StackMatDesc &m = ph.m[mi];
-      for (int i = ctid; i < nrows; i += kStkConsThreads)
-        s8c[mi * rows_max + i] = m.n_sal > 0 ? bf16_bits_to_f32(__ldg(m.s8 + ph.a + i)) : 0.0f;
-      for (int e = ctid; e < m.n_sal; e += kStkConsThreads)
-        sidx[mi * p.max_nsal + e] = __ldg(m.sal_idx + e);
-    }
-    for (int q = cw; q < ph.nm * kStkMaxRank; q += kStkCons) {
-      const int mi = q / kStkMaxRank, k = q % kStkMaxRank;
-      if (k >= ph.m[mi].r) continue;
+    const int r0m = ph.m[0].r, npair = r0m + (ph.nm > 1 ? ph.m[1].r : 0);
+    const int NP = npair > 0 ? max(1, min(16, kStkConsThreads / npair)) : 1;
+    const int Gp = (G + NP - 1) / NP;
+    for (int tau = ctid; tau < npair * NP; tau += kStkConsThreads) {
+      const int q = tau / NP, j = tau - q * NP;
+      const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
       const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * G;
+      const int c0 = j * Gp, c1 = min(G, c0 + Gp);
       float s = 0.0f;
-      for (int i = lane; i < G; i += 32) s += __ldcg(src + i);
+      for (int i0 = c0; i0 < c1; i0 += 16) {
+        float v[16];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) tv[mi * kStkMaxRank + k] = s;
+        for (int u = 0; u < 16; ++u) v[u] = i0 + u < c1 ? __ldcg(src + i0 + u) : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s += v[u];
+      }
+      tq[tau] = s;
     }
+    stk_cp_async_wait_all();             // this phase's prefetched s8 and salient indices
     stk_consumer_sync();
+    for (int q = ctid; q < npair; q += kStkConsThreads) {
+      float s = 0.0f;
+      for (int j = 0; j < NP; ++j) s += tq[q * NP + j];
+      const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
+      tv[mi * kStkMaxRank + k] = s;
+    }
 
     // rotate x: BF16 in, int16 (unit/chunk layout) with one scale per 64 columns
     {
@@ -345,135 +452,171 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     }
     stk_consumer_sync();
 
-    // the rows: items (row pair, round) of each tile, round-robin over the warps
+    // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
+    // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
+    // RR rounds (RG RR = 8 independent dot products per lane); the items of
+    // a tile go round-robin over the consumer warps.
     for (int mi = 0; mi < ph.nm; ++mi) {
       const StackMatDesc &m = ph.m[mi];
-      const int kq = m.K / 2, ks = m.K / 32, nu4 = m.K / 32, nu8 = m.n_sal / 32;
+      const int nsal = m.n_sal, rk = m.r;
+      const int kq = m.K / 2, ks = m.K / 32, nu4 = m.K / 32, nu8 = nsal / 32;
       const int rounds = (nu4 + nu8 + 31) / 32;
+      const int RG = ph.rg, RR = 8 / RG;
+      const int nrg = (rounds + RR - 1) / RR;
       const float *tvm = tv + mi * kStkMaxRank;
       const uint16_t *xsm = xsal + mi * p.max_nsal;
       const float *xssm = xss + mi * (p.max_nsal / 32);
+      const uint16_t *s8m = s8c + mi * s8_stride + (ph.a & 7);
       for (int i0 = ph.a; i0 < ph.b; i0 += ph.tr, ++seq) {
-        const int nr = min(ph.tr, ph.b - i0), npair = (nr + 1) / 2;
+        const int nr = min(ph.tr, ph.b - i0), ngr = (nr + RG - 1) / RG;
         const int s = (int)(seq % (uint32_t)NS);
         const bool got =
             __all_sync(0xffffffffu, stk_wait(&full[s], (seq / (uint32_t)NS) & 1u, abort));
-        const uint8_t *slot = ring + (size_t)s * p.slot_bytes;
-        const uint8_t *q4s = slot, *s4s = slot + nr * kq, *q8s = s4s + nr * ks;
-        const uint8_t *us = q8s + nr * m.n_sal;
-        const int items = npair * rounds;
-        for (int it = (cw - rot + kStkCons * 64) % kStkCons; got && it < items; it += kStkCons) {
-          const int pr = it / rounds, rd = it - pr * rounds;
-          const int r0 = 2 * pr, r1 = r0 + 1;
-          const bool two = r1 < nr;
-          const int task = 32 * rd + lane;
-          float acc0 = 0.0f, acc1 = 0.0f;
-          if (task < nu4) {
-            const int v = task, g = v >> 1;
-            uint4 xa[4];
+        const uint8_t *q4s = ring + (size_t)s * p.slot_bytes;
+        const uint8_t *s4s = q4s + nr * kq, *q8s = s4s + nr * ks;
+        const uint16_t *us = reinterpret_cast<const uint16_t *>(q8s + nr * nsal);
+        const int items = ngr * nrg;
+        // RG rows x RR rounds per item, straight-line: rows past the tile
+        // repeat its last row and are masked when accumulated
+        auto run_items = [&](auto rg_tag) {
+          constexpr int RGc = decltype(rg_tag)::value, RRc = 8 / RGc;
+          for (int it = (cw - rot + kStkCons * 64) % kStkCons; got && it < items; it += kStkCons) {
+            const int gi = it / nrg, rq = it - gi * nrg;
+            const int r0 = gi * RGc;
+            int rl[RGc];
+            float acc[RGc];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
-            const int bias = 8 * xsu[v];
-            const float sc = xsc[g];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              if (rr == 1 && !two) break;
-              const int rl = r0 + rr;
-              const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl * kq + 16 * v);
-              const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-              int d = 0;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
-                const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
-                d = __dp2a_lo((int)xa[i].x, (int)L, d);
-                d = __dp2a_hi((int)xa[i].y, (int)L, d);
-                d = __dp2a_lo((int)xa[i].z, (int)Hh, d);
-                d = __dp2a_hi((int)xa[i].w, (int)Hh, d);
-              }
-              const float s4v =
-                  bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl * ks)[g]);
-              const float f = s4v * sc * (float)(d - bias);
-              if (rr == 0) acc0 = f; else acc1 = f;
+            for (int ri = 0; ri < RGc; ++ri) {
+              rl[ri] = min(r0 + ri, nr - 1);
+              acc[ri] = 0.0f;
             }
-          } else if (task < nu4 + nu8) {
-            const int j = task - nu4;
-            uint4 xa[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
-            const float sc = xssm[j];
+            for (int u = 0; u < RRc; ++u) {
+              const int task = 32 * (rq * RRc + u) + lane;
+              float f[RGc];
+              if (task < nu4) {
+                const int v = task, g = v >> 1;
+                uint4 xa[4];
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              if (rr == 1 && !two) break;
-              const int rl = r0 + rr;
-              const uint4 qa = *reinterpret_cast<const uint4 *>(q8s + (size_t)rl * m.n_sal + 32 * j);
-              const uint4 qb =
-                  *reinterpret_cast<const uint4 *>(q8s + (size_t)rl * m.n_sal + 32 * j + 16);
-              const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-              int d = 0;
+                for (int i = 0; i < 4; ++i)
+                  xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
+                const int bias = 8 * xsu[v];
+                const float sc = xsc[g];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                d = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d);
-                d = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d);
-                d = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d);
-                d = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d);
+                for (int ri = 0; ri < RGc; ++ri) {
+                  const uint4 w4 =
+                      *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
+                  const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+                  int d[4] = {0, 0, 0, 0};
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
+                    const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+                    d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
+                    d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
+                    d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
+                    d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
+                  }
+                  const float s4v = bf16_bits_to_f32(
+                      reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
+                  f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
+                }
+              } else if (task < nu4 + nu8) {
+                const int j = task - nu4;
+                uint4 xa[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
+                const float sc = xssm[j];
+#pragma unroll
+                for (int ri = 0; ri < RGc; ++ri) {
+                  const uint8_t *qr = q8s + (size_t)rl[ri] * nsal + 32 * j;
+                  const uint4 qa = *reinterpret_cast<const uint4 *>(qr);
+                  const uint4 qb = *reinterpret_cast<const uint4 *>(qr + 16);
+                  const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                  int d[4] = {0, 0, 0, 0};
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    d[i] = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d[i]);
+                    d[i] = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d[i]);
+                    d[i] = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d[i]);
+                    d[i] = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d[i]);
+                  }
+                  f[ri] = bf16_bits_to_f32(s8m[(i0 - ph.a) + rl[ri]]) * sc *
+                          (float)((d[0] + d[1]) + (d[2] + d[3]));
+                }
+              } else {
+#pragma unroll
+                for (int ri = 0; ri < RGc; ++ri) f[ri] = 0.0f;
               }
-              const float f = s8c[mi * rows_max + (i0 - ph.a) + rl] * sc * (float)d;
-              if (rr == 0) acc0 = f; else acc1 = f;
+#pragma unroll
+              for (int ri = 0; ri < RGc; ++ri) acc[ri] += f[ri];
+            }
+            if (rq == 0 && lane < rk) {
+#pragma unroll
+              for (int ri = 0; ri < RGc; ++ri)
+                acc[ri] = fmaf(bf16_bits_to_f32(us[rl[ri] * rk + lane]), tvm[lane], acc[ri]);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+#pragma unroll
+              for (int ri = 0; ri < RGc; ++ri) acc[ri] += __shfl_xor_sync(0xffffffffu, acc[ri], o);
+            }
+            if (lane == 0) {
+#pragma unroll
+              for (int ri = 0; ri < RGc; ++ri)
+                if (r0 + ri < nr)
+                  red[((size_t)mi * rows_max + (i0 - ph.a) + r0 + ri) * rounds_max + rq] = acc[ri];
             }
           }
-          if (rd == 0 && lane < m.r) {
-            const uint16_t *ur = reinterpret_cast<const uint16_t *>(us);
-            acc0 = fmaf(bf16_bits_to_f32(ur[r0 * m.r + lane]), tvm[lane], acc0);
-            if (two) acc1 = fmaf(bf16_bits_to_f32(ur[r1 * m.r + lane]), tvm[lane], acc1);
-          }
-#pragma unroll
-          for (int o = 16; o; o >>= 1) {
-            acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
-            acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
-          }
-          if (lane == 0) {
-            float *rw = red + ((size_t)mi * rows_max + (i0 - ph.a) + r0) * rounds_max + rd;
-            rw[0] = acc0;
-            if (two) rw[rounds_max] = acc1;
-          }
-        }
+        };
+        if (RG == 4) run_items(std::integral_constant<int, 4>{});
+        else run_items(std::integral_constant<int, 2>{});
         rot = (rot + items) % kStkCons;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
     stk_consumer_sync();
-    // row results (rounds in order) back into red[mi][row][0]
+    // row results (round groups in order) back into red[mi][row][0]
     for (int mi = 0; mi < ph.nm; ++mi) {
       const int rounds = (ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32;
+      const int nrg = (rounds + 8 / ph.rg - 1) / (8 / ph.rg);
       for (int i = ctid; i < nrows; i += kStkConsThreads) {
         float *rw = red + ((size_t)mi * rows_max + i) * rounds_max;
-        float s = rw[0];
-        for (int rd = 1; rd < rounds; ++rd) s += rw[rd];
-        rw[0] = s;
+        float sum = rw[0];
+        for (int rd = 1; rd < nrg; ++rd) sum += rw[rd];
+        rw[0] = sum;
       }
     }
     stk_consumer_sync();
   };
 
+  // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
+  StkPhase ph = make_phase(0, 0);
+  prefetch(ph);
+  {
+    const int n = d_b - d_a;
+    for (int i = ctid; i < n; i += kStkConsThreads) vals[i] = bf16_bits_to_f32(p.x[d_a + i]);
+    stk_consumer_sync();
+    for (int j = 0; j < 2; ++j) {
+      const StackMatDesc &m = ph.m[j];
+      for (int k = cw; k < m.r; k += kStkCons) {
+        const float *row = m.vh + (size_t)k * m.K + d_a;
+        float sacc = 0.0f;
+        for (int i = lane; i < n; i += 32) sacc = fmaf(__ldg(row + i), vals[i], sacc);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+        if (lane == 0) p.tp[((size_t)j * kStkMaxRank + k) * G + c] = sacc;
+      }
+    }
+  }
+  grid_arrive();
+  bool live = grid_wait();
+
   // ---- the blocks: gate+up (x -> h), then down (h -> x)
   for (int l = 0; l < p.L; ++l) {
-    const StackLayerDesc &Ld = p.layers[l];
     {
-      StkPhase ph;
-      ph.nm = 2;
-      ph.m[0] = Ld.m[0];
-      ph.m[1] = Ld.m[1];
-      ph.K = p.H;
-      ph.a = gu_a;
-      ph.b = gu_b;
-      ph.tr = p.tr_gu;
-      ph.src = l == 0 ? p.x : p.y;
-      ph.tslot[0] = 0;
-      ph.tslot[1] = 1;
       if (live) run_phase(ph);
       // h = RN_bf16(gelu(g) u), g and u rounded to BF16 first
       const int n = gu_b - gu_a;
@@ -485,20 +628,15 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         p.h[gu_a + i] = hb;
         vals[i] = bf16_bits_to_f32(hb);
       }
+      stk_cp_async_wait_all();
       stk_consumer_sync();
-      if (live) t_share(Ld.m[2], 2, gu_a, n);
-      live = grid_sync() && live;
+      if (live) t_share_out(ph);
+      grid_arrive();
+      ph = make_phase(l, 1);
+      prefetch(ph);
+      live = grid_wait() && live;
     }
     {
-      StkPhase ph;
-      ph.nm = 1;
-      ph.m[0] = Ld.m[2];
-      ph.K = p.I;
-      ph.a = d_a;
-      ph.b = d_b;
-      ph.tr = p.tr_d;
-      ph.src = p.h;
-      ph.tslot[0] = 2;
       if (live) run_phase(ph);
       const int n = d_b - d_a;
       for (int i = ctid; i < n && live; i += kStkConsThreads) {
@@ -506,13 +644,14 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         p.y[d_a + i] = xb;
         vals[i] = bf16_bits_to_f32(xb);
       }
+      stk_cp_async_wait_all();
       stk_consumer_sync();
       if (l + 1 < p.L) {
-        if (live) {
-          t_share(p.layers[l + 1].m[0], 0, d_a, n);
-          t_share(p.layers[l + 1].m[1], 1, d_a, n);
-        }
-        live = grid_sync() && live;
+        if (live) t_share_out(ph);
+        grid_arrive();
+        ph = make_phase(l + 1, 0);
+        prefetch(ph);
+        live = grid_wait() && live;
       }
     }
   }
@@ -570,6 +709,8 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &
     }
   p.tr_gu = std::max(2, (kStkSlotTarget / rb_gu) & ~1);
   p.tr_d = std::max(2, (kStkSlotTarget / rb_d) & ~1);
+  p.rg_gu = p.tr_gu >= 4 ? 4 : 2;
+  p.rg_d = p.tr_d >= 4 ? 4 : 2;
   p.slot_bytes = (std::max(p.tr_gu * rb_gu, p.tr_d * rb_d) + 127) & ~127;
   p.max_rank = max_rank;
   p.max_nsal = std::max(max_nsal, 32);
@@ -589,9 +730,14 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &
   p.o_xss = take(2 * (p.max_nsal / 32) * 4);
   p.o_sidx = take(2 * p.max_nsal * 4);
   p.o_t = take(2 * kStkMaxRank * 4);
-  p.o_s8 = take(2 * p.rows_max * 4);
+  p.o_s8 = take(2 * stk_s8_stride(p.rows_max) * 2);
   p.o_yv = take(2 * p.rows_max * p.rounds_max * 4);
   p.o_vh = take(p.rows_max * 4);
+  p.o_tq = take(kStkConsThreads * 4);
+  {
+    const int rg = (p.I + G - 1) / G, rd = (p.H + G - 1) / G;
+    p.o_vhs = take(std::max(max_rank * rg, 2 * max_rank * rd) * 4);
+  }
   p.o_scr = take(kStkFwhtGroups * (B == 256 ? GroupScratch<256>::kElems : GroupScratch<128>::kElems) * 4);
   p.o_flag = take(16);
   const int fixed = off;
