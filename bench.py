@@ -79,10 +79,27 @@ def kernel_bytes(name, M, K, rank, n_sal, T):
     return None
 
 
-def source_hash():
+# The source files each kernel is built from: a recorded DRAM count stays valid
+# while these files are unchanged.
+KERNEL_SOURCES = {
+    "enc_pass1": ("encode.cu", "fwht_group.cuh"),
+    "enc_pass2": ("encode.cu", "fwht_group.cuh"),
+    "enc_select": ("encode.cu",),
+    "dec_row": ("decode_row.cu", "fwht_group.cuh"),
+    "dec_main": ("decode.cu", "fwht_group.cuh"),
+    "dec_tail": ("decode.cu",),
+    "pre_act": ("prefill.cu", "fwht_group.cuh"),
+    "pre_mat": ("prefill.cu",),
+    "pre_gemm": ("prefill.cu", "common.cuh"),
+    "mlp_stack": ("stack.cu", "fwht_group.cuh"),
+}
+
+
+def source_hash(kernel=None):
     d = os.path.join(ROOT, "mixed_precision_weight_b200", "csrc")
+    files = KERNEL_SOURCES.get(kernel) or tuple(sorted(os.listdir(d)))
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
+    for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -97,7 +114,7 @@ def dram_traffic(kernel, workload):
     except OSError:
         return None
     ent = rec.get(f"{kernel}@{workload}")
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash(kernel):
         return None
     return ent.get("bytes_per_launch")
 

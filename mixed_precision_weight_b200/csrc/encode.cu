@@ -25,7 +25,8 @@ namespace dvssq {
 
 constexpr int kSsqChunk = 16;     // rows per fixed-order partial (salience)
 constexpr int kSsqGroup = 8;      // chunk partials per group sum
-constexpr int kStages = 4;        // cp.async ring depth per group (row-blocks)
+constexpr int kStages = 4;        // cp.async ring depth per group (row-blocks), pass 1
+constexpr int kP2Stages = 3;      // the same for pass 2 (fewer: five CTAs per SM fit)
 constexpr int kTileRowsMax = 64;  // rows per pass-2 tile, upper bound
 constexpr int kStashSmemMax = 96 * 1024;
 
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
 // ---------------------------------------------------------------- pass 2 --
 // A CTA takes tiles of R whole rows from a global counter.  Within a tile the
 // R * nkb row-blocks are ordered column-block-major and split into NG equal
-// runs of ipg >= kStages - 1 row-blocks, one run per group, so a group's
+// runs of ipg >= kP2Stages - 1 row-blocks, one run per group, so a group's
 // cp.async ring can run ahead into the next tile (whose index is fetched one
 // tile early).  Per row-block the group rotates again, stages its outputs in
 // shared memory, moves the block's salient values to the stash and zeroes
@@ -442,7 +443,7 @@ struct Pass2Params {
   int R, rshift;      // rows per tile (a power of two) and its log2
   int ipg;            // row-blocks per group and tile
   int ntiles;
-  int stash_smem;     // 1: stash in dynamic shared memory [2][R][n_sal]; 0: in sv [M][n_sal]
+  int stash_smem;     // 1: stash in dynamic shared memory [R][n_sal]; 0: in sv [M][n_sal]
   double c;
   const int32_t *sal_idx, *sal_prefix;
   uint8_t *q4;
@@ -455,7 +456,13 @@ struct Pass2Params {
   unsigned long long *info;
 };
 
-constexpr int kStageStride = 18;   // doubles per thread's 16 staged outputs (+2: no bank conflicts)
+// Staged outputs: thread t's 16 values at [16 t, 16 t + 16), the 16-byte
+// pair m at pair position m ^ (t & 7), so that the eight threads of a
+// quarter-warp store to distinct banks.
+__device__ __forceinline__ int stage_pos(int col) {
+  const int t = col >> 4, j = col & 15;
+  return 16 * t + 2 * ((j >> 1) ^ (t & 7)) + (j & 1);
+}
 
 // Eight 4-bit codes (two's complement in the low bits of l[0..7]) into one
 // word, code 2m in the low nibble of byte m.
@@ -473,13 +480,13 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
   constexpr int GPW = 32 / P;
   constexpr int NG = GPW * 4;
   constexpr int SCR0 = GroupScratch<B>::kElems;
-  constexpr int SCR1 = P * kStageStride;
+  constexpr int SCR1 = 16 * P;
   constexpr int SCR = ((SCR0 > SCR1 ? SCR0 : SCR1) + 1) & ~1;   // even: 16-byte aligned rows
   constexpr bool kPow2 = B == 256;
   constexpr int PIECES = B * 2 / 16;
   __shared__ __align__(16) double scratch[NG][SCR];
-  __shared__ __align__(16) uint16_t ring[NG][kStages][B];
-  __shared__ unsigned long long s_rmax[2][kTileRowsMax];
+  __shared__ __align__(16) uint16_t ring[NG][kP2Stages][B];
+  __shared__ unsigned long long s_rmax[kTileRowsMax];
   __shared__ int s_tile[4];
   extern __shared__ __align__(16) double stash_s[];
 
@@ -497,7 +504,7 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
     s_tile[0] = (int)atomicAdd(p.tile_ctr, 1u);
     s_tile[1] = (int)atomicAdd(p.tile_ctr, 1u);
   }
-  for (int i = tid; i < 2 * kTileRowsMax; i += blockDim.x) (&s_rmax[0][0])[i] = 0ull;
+  for (int i = tid; i < kTileRowsMax; i += blockDim.x) s_rmax[i] = 0ull;
   __syncthreads();
   int cur = s_tile[0], nxt = s_tile[1];
 
@@ -519,24 +526,24 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
     cp_async_commit();
   };
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) issue(src_of(cur, s), s);
+  for (int s = 0; s < kP2Stages - 1; ++s) issue(src_of(cur, s), s);
 
   unsigned long long unsafe = 0;
   int pos = 0;    // ring position of the row-block in hand
-  int k = 0;      // tiles done by this CTA: parity of the stash and the row maxima
+  int k = 0;      // tiles done by this CTA: parity of the next-tile slots
   while (cur < ntiles) {
     if (tid == 0) s_tile[2 + (k & 1)] = (int)atomicAdd(p.tile_ctr, 1u);   // the tile after nxt
-    double *const stash = p.stash_smem ? stash_s + (size_t)(k & 1) * R * n_sal : nullptr;
+    double *const stash = p.stash_smem ? stash_s : nullptr;
     for (int ii = 0; ii < ipg; ++ii, ++pos) {
-      const int ia = ii + kStages - 1;
-      issue(ia < ipg ? src_of(cur, ia) : src_of(nxt, ia - ipg), (pos + kStages - 1) % kStages);
-      cp_async_wait<kStages - 1>();
+      const int ia = ii + kP2Stages - 1;
+      issue(ia < ipg ? src_of(cur, ia) : src_of(nxt, ia - ipg), (pos + kP2Stages - 1) % kP2Stages);
+      cp_async_wait<kP2Stages - 1>();
       __syncwarp();
       const int item = item0 + ii;
       const int kb = item >> rshift, r = item - (kb << rshift);
       const int row = (cur << rshift) + r;
       const bool valid = row < M;
-      const uint16_t *buf = ring[g][pos % kStages];
+      const uint16_t *buf = ring[g][pos % kP2Stages];
       double v[16];
 #pragma unroll
       for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
@@ -546,9 +553,9 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __dmul_rn(v[j], c);
       }
-      double2 *stg = reinterpret_cast<double2 *>(sgrp + t * kStageStride);
+      double2 *stg = reinterpret_cast<double2 *>(sgrp + 16 * t);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) stg[m] = make_double2(v[2 * m], v[2 * m + 1]);
+      for (int m = 0; m < 8; ++m) stg[m ^ (t & 7)] = make_double2(v[2 * m], v[2 * m + 1]);
       __syncwarp();
       // this block's salient columns: to the stash, then zero in the staged row
       const int e0 = __ldg(p.sal_prefix + ((kb * B) >> 5));
@@ -557,7 +564,7 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
         double *dst = stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal;
         for (int e = e0 + t; e < e1; e += P) {
           const int col = __ldg(p.sal_idx + e) - kb * B;
-          const int si = (col >> 4) * kStageStride + (col & 15);
+          const int si = stage_pos(col);
           dst[e] = sgrp[si];
           sgrp[si] = 0.0;
         }
@@ -565,7 +572,7 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
       __syncwarp();
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        const double2 d = stg[m];
+        const double2 d = stg[m ^ (t & 7)];
         v[2 * m] = d.x;
         v[2 * m + 1] = d.y;
       }
@@ -633,17 +640,16 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
         const double2 d = src[u];
         m = fmax(m, fmax(fabs(d.x), fabs(d.y)));
       }
-      atomicMax(&s_rmax[k & 1][r], (unsigned long long)__double_as_longlong(m));
+      atomicMax(&s_rmax[r], (unsigned long long)__double_as_longlong(m));
     }
     __syncthreads();                      // row maxima complete
-    if (tid < R) s_rmax[(k + 1) & 1][tid] = 0ull;
     for (int ch = tid; ch < (n8 << rshift); ch += blockDim.x) {
       const int r = ch / n8, e = (ch - r * n8) * 8;
       const int row = (cur << rshift) + r;
       if (row >= M) continue;
       const double2 *src = reinterpret_cast<const double2 *>(
           (stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal) + e);
-      const double m = __longlong_as_double((long long)s_rmax[k & 1][r]) * vscale;
+      const double m = __longlong_as_double((long long)s_rmax[r]) * vscale;
       const uint16_t sb = bf16_of_quotient(m, 127.0, kInv127);
       const double s8v = bf16_bits_to_f64(sb);
       const double vinv = s8v > 0.0 ? recip_bf16(sb) * vscale : 0.0;
@@ -664,6 +670,8 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
     if (n8 == 0)
       for (int r = tid; r < R; r += blockDim.x)
         if ((cur << rshift) + r < M) p.s8[(cur << rshift) + r] = 0;
+    __syncthreads();                      // stash and row maxima free for the next tile
+    if (tid < R) s_rmax[tid] = 0ull;
     cur = nxt;
     nxt = s_tile[2 + (k & 1)];
     ++k;
@@ -683,18 +691,18 @@ struct Pass2Plan {
 };
 
 // Rows per tile: the smallest power of two that splits the tile's R * nkb
-// row-blocks evenly over the groups with at least kStages - 1 per group.
+// row-blocks evenly over the groups with at least kP2Stages - 1 per group.
 Pass2Plan pass2_plan(int M, int K, int B, int n_sal) {
   const int NG = groups_per_cta(B), nkb = K / B;
   int R = 1;
-  while ((R * nkb) % NG != 0 || R * nkb / NG < kStages - 1) R *= 2;
+  while ((R * nkb) % NG != 0 || R * nkb / NG < kP2Stages - 1) R *= 2;
   Pass2Plan pl{};
   pl.R = R;
   pl.rshift = 0;
   while ((1 << pl.rshift) < R) ++pl.rshift;
   pl.ipg = R * nkb / NG;
   pl.ntiles = (M + R - 1) / R;
-  const size_t bytes = (size_t)2 * R * n_sal * sizeof(double);
+  const size_t bytes = (size_t)R * n_sal * sizeof(double);
   pl.smem = bytes <= (size_t)kStashSmemMax;
   pl.smem_bytes = pl.smem ? bytes : 0;
   return pl;
