@@ -45,35 +45,50 @@ struct PrefillParams {
   int y_bf16;
   __half *xc;      // [T][Kc]
   __half *a;       // [M][Kc]
+  int nsplit;      // CTAs per 16-token group in pre_act, each a run of Hadamard blocks
+  float *tpart;    // [nsplit][T][rank] t partials when nsplit > 1
+  unsigned int *tdone;   // [T/16] finished splits per token group (zero at launch)
 };
 
 // ------------------------------------------------------------------ pre_act
-// Dynamic shared memory of pre_act: fp32 block [16][B+1], FP16 block
-// [16][B+8], FP16 V block [rank][B+8], sal_idx copy [n_sal].
+// Dynamic shared memory of pre_act: FP16 block [16][B+8], FP16 V block
+// [rank][B+8], sal_idx copy [n_sal], first salient entry of each Hadamard
+// block [K/B + 1] (K/B <= 512).
 static size_t pre_act_smem_bytes(int B, int rank, int n_sal) {
-  return (size_t)16 * (B + 1) * 4 + (size_t)16 * (B + 8) * 2 + (size_t)rank * (B + 8) * 2 +
-         (size_t)n_sal * 4;
+  return (size_t)16 * (B + 8) * 2 + (size_t)rank * (B + 8) * 2 + (size_t)n_sal * 4 + 513 * 4;
 }
 
-template <int B>
-__device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int blk) {
+template <int B, int VPT>
+__device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int blk,
+                                              const int split) {
   constexpr int P = B / 16;
   constexpr int NW = B / 32;
   __shared__ float scratch[16][GroupScratch<B>::kElems];
   extern __shared__ __align__(16) uint8_t dsm[];
-  float (*xr)[B + 1] = reinterpret_cast<float (*)[B + 1]>(dsm);
-  __half (*xh)[B + 8] = reinterpret_cast<__half (*)[B + 8]>(dsm + 16 * (B + 1) * 4);
-  __half (*vh)[B + 8] =
-      reinterpret_cast<__half (*)[B + 8]>(dsm + 16 * (B + 1) * 4 + 16 * (B + 8) * 2);
-  int *sidx = reinterpret_cast<int *>(dsm + 16 * (B + 1) * 4 + 16 * (B + 8) * 2 +
-                                      (size_t)p.rank * (B + 8) * 2);
+  __half (*xh)[B + 8] = reinterpret_cast<__half (*)[B + 8]>(dsm);
+  __half (*vh)[B + 8] = reinterpret_cast<__half (*)[B + 8]>(dsm + 16 * (B + 8) * 2);
+  int *sidx = reinterpret_cast<int *>(dsm + 16 * (B + 8) * 2 + (size_t)p.rank * (B + 8) * 2);
+  int *sblk = sidx + p.n_sal;        // first salient entry at or after column kb B
 
   const int tid = threadIdx.x, tok = tid / P, t = tid % P;
   const int t0 = blk * 16, gt = t0 + tok;
   const bool live = gt < p.T;
   const int nkb = p.K / B;
+  // this CTA's run of Hadamard blocks
+  const int kbA = (int)((long long)split * nkb / p.nsplit);
+  const int kbB = (int)((long long)(split + 1) * nkb / p.nsplit);
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
   for (int e = tid; e < p.n_sal; e += B) sidx[e] = p.sal_idx[e];
+  __syncthreads();
+  // salient entries of block kb: [sblk[kb], sblk[kb + 1]) (sal_idx is ascending)
+  for (int kb = tid; kb <= nkb; kb += B) {
+    int lo = 0, hi = p.n_sal;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sidx[mid] < kb * B) lo = mid + 1; else hi = mid;
+    }
+    sblk[kb] = lo;
+  }
 
   // t accumulators: n-tile (8 ranks) nt = warp + NW * j, j = 0, 1
   float tacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -81,8 +96,7 @@ __device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int 
 
   // the next block's x (registers) and V rows (registers, stored to vh at the
   // top of its iteration) are loaded one block ahead, so that their latency
-  // overlaps the current block's work
-  constexpr int VPT = 64 * (B / 8) / B;          // uint4 of V per thread (rank <= 64)
+  // overlaps the current block's work; VPT uint4 of V per thread cover the rank
   uint16_t xn[16];
   uint4 vn[VPT];
   auto fetch = [&](int kb) {
@@ -98,8 +112,8 @@ __device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int 
                   : make_uint4(0u, 0u, 0u, 0u);
     }
   };
-  fetch(0);
-  for (int kb = 0; kb < nkb; ++kb) {
+  if (kbA < kbB) fetch(kbA);
+  for (int kb = kbA; kb < kbB; ++kb) {
     float v[16];
 #pragma unroll
     for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f32(xn[a]);
@@ -118,16 +132,12 @@ __device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int 
         *reinterpret_cast<uint4 *>(&vh[rr][cc * 8]) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    if (kb + 1 < nkb) fetch(kb + 1);
+    if (kb + 1 < kbB) fetch(kb + 1);
     fwht_group<B>(v, scratch[tok], t);
     uint32_t h[8];
 #pragma unroll
-    for (int j = 0; j < 16; j += 2) {
-      const float a0 = v[j] * p.c, a1 = v[j + 1] * p.c;
-      xr[tok][16 * t + j] = a0;
-      xr[tok][16 * t + j + 1] = a1;
-      h[j / 2] = pack_half2(__float2half_rn(a0), __float2half_rn(a1));
-    }
+    for (int j = 0; j < 16; j += 2)
+      h[j / 2] = pack_half2(__float2half_rn(v[j] * p.c), __float2half_rn(v[j + 1] * p.c));
     *reinterpret_cast<uint4 *>(&xh[tok][16 * t]) = make_uint4(h[0], h[1], h[2], h[3]);
     *reinterpret_cast<uint4 *>(&xh[tok][16 * t + 8]) = make_uint4(h[4], h[5], h[6], h[7]);
     if (live) {
@@ -136,25 +146,15 @@ __device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int 
       dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
     }
     __syncthreads();
-    // salient gather: entries whose column lies in this block (sal_idx sorted)
+    // salient gather: the block's entries, consecutive lanes on consecutive
+    // entries of one token (the FP16 block holds RN16 of the rotated values)
     {
-      int lo = 0, hi = p.n_sal;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (sidx[mid] < kb * B) lo = mid + 1; else hi = mid;
-      }
-      const int e_lo = lo;
-      hi = p.n_sal;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (sidx[mid] < (kb + 1) * B) lo = mid + 1; else hi = mid;
-      }
-      const int e_hi = lo;
-      for (int i = tid; i < (e_hi - e_lo) * 16; i += B) {
-        const int e = e_lo + i / 16, q = i % 16;
+      const int e_lo = sblk[kb], ne = sblk[kb + 1] - e_lo;
+      for (int i = tid; i < ne * 16; i += B) {
+        const int q = i / ne, e = e_lo + (i - q * ne);
         const int col = sidx[e] - kb * B;
         if (t0 + q < p.T && col >= 0 && col < B)
-          p.xc[(size_t)(t0 + q) * p.Kc + p.K + e] = __float2half_rn(xr[q][col]);
+          p.xc[(size_t)(t0 + q) * p.Kc + p.K + e] = xh[q][col];
       }
     }
     // t += xr_block (16 x B) . V_block^T (B x 8) per n-tile of 8 ranks
@@ -178,19 +178,51 @@ __device__ __forceinline__ void pre_act_block(const PrefillParams &p, const int 
     }
     __syncthreads();
   }
-  // t and the zero padding of the salient and low-rank sections
+  // t: one split writes it directly; several write FP32 partials and the
+  // last to finish adds them in split order
+  if (p.nsplit > 1) {
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int nt = warp + NW * j;
-    if (nt >= ntiles) break;
-    const int n = 8 * nt + 2 * tig;
+    for (int j = 0; j < 2; ++j) {
+      const int nt = warp + NW * j;
+      if (nt >= ntiles) break;
+      const int n = 8 * nt + 2 * tig;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int q = g + 8 * (i >> 1), rr = n + (i & 1);
-      if (t0 + q < p.T && rr < p.rank)
-        p.xc[(size_t)(t0 + q) * p.Kc + p.K + p.salp + rr] = __float2half_rn(tacc[j][i]);
+      for (int i = 0; i < 4; ++i) {
+        const int q = g + 8 * (i >> 1), rr = n + (i & 1);
+        if (t0 + q < p.T && rr < p.rank)
+          p.tpart[((size_t)split * p.T + t0 + q) * p.rank + rr] = tacc[j][i];
+      }
+    }
+    __shared__ unsigned int s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.tdone[blk], 1u) == (unsigned int)(p.nsplit - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int i = tid; i < 16 * p.rank; i += B) {
+      const int q = i / p.rank, rr = i - q * p.rank;
+      if (t0 + q >= p.T) continue;
+      float v = 0.0f;
+      for (int sp = 0; sp < p.nsplit; ++sp)
+        v += __ldcg(p.tpart + ((size_t)sp * p.T + t0 + q) * p.rank + rr);
+      p.xc[(size_t)(t0 + q) * p.Kc + p.K + p.salp + rr] = __float2half_rn(v);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int nt = warp + NW * j;
+      if (nt >= ntiles) break;
+      const int n = 8 * nt + 2 * tig;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = g + 8 * (i >> 1), rr = n + (i & 1);
+        if (t0 + q < p.T && rr < p.rank)
+          p.xc[(size_t)(t0 + q) * p.Kc + p.K + p.salp + rr] = __float2half_rn(tacc[j][i]);
+      }
     }
   }
+  // the zero padding of the salient and low-rank sections
   const int npad1 = p.salp - p.n_sal, npad2 = 64 - p.rank;
   for (int i = tid; i < 16 * (npad1 + npad2); i += B) {
     const int q = i / (npad1 + npad2), j = i % (npad1 + npad2);
@@ -271,10 +303,10 @@ __device__ __forceinline__ void pre_mat_item(const PrefillParams &p, const long 
 // latency-bound activation pass leaves idle.  pre_mat reads only the packed
 // weights; it waits for pre_act only before it exits, so that its completion
 // (which orders the GEMM) implies pre_act's.
-template <int B>
-__global__ void __launch_bounds__(B) pre_act_kernel(PrefillParams p) {
+template <int B, int VPT>
+__global__ void __launch_bounds__(B, 768 / B) pre_act_kernel(PrefillParams p) {
   pdl_launch_dependents();
-  pre_act_block<B>(p, blockIdx.x);
+  pre_act_block<B, VPT>(p, blockIdx.x, blockIdx.y);
 }
 
 __global__ void __launch_bounds__(256) pre_mat_kernel(PrefillParams p, long long items) {
@@ -422,12 +454,26 @@ static size_t pre_smem_bytes(int BN) {
   return 1024 + (size_t)kPreStages * (kPreBM * 128 + BN * 128) + 256;   // + barriers, TMEM slot
 }
 
+// CTAs per 16-token group in pre_act: enough for about four resident CTAs
+// on each of B200's 148 SMs, each a run of at least one Hadamard block.  A
+// host-side constant (no device query), so the workspace size stays a pure
+// function of the shape; any split count gives the same result.
+constexpr int kPreActSlots = 4 * 148;
+static int pre_act_splits(int nkb, int T) {
+  const int ntg = (T + 15) / 16;
+  const int want = (kPreActSlots + ntg - 1) / ntg;
+  return std::max(1, std::min(nkb, want));
+}
+
 size_t prefill_workspace_bytes(int M, int K, int block, int n_sal, int rank, int T) {
   (void)block; (void)rank;
   const int salp = (n_sal + 63) / 64 * 64;
   const size_t Kc = (size_t)K + salp + 64;
-  // Xc [T][Kc] and the materialised A [M][Kc], FP16
-  return (((size_t)T * Kc * 2 + 255) & ~(size_t)255) + (((size_t)M * Kc * 2 + 255) & ~(size_t)255);
+  // Xc [T][Kc] and the materialised A [M][Kc], FP16; pre_act's t partials
+  // [nsplit][T][rank] and per-16-token counters
+  const int ns = pre_act_splits(K / block, T);
+  return (((size_t)T * Kc * 2 + 255) & ~(size_t)255) + (((size_t)M * Kc * 2 + 255) & ~(size_t)255) +
+         (((size_t)ns * T * 64 * 4 + 255) & ~(size_t)255) + (((size_t)(T + 15) / 16 * 4 + 255) & ~(size_t)255);
 }
 
 cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
@@ -445,13 +491,31 @@ cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   p.a = reinterpret_cast<__half *>(static_cast<char *>(a.workspace) +
                                    (((size_t)a.T * p.Kc * 2 + 255) & ~(size_t)255));
 
+  {
+    const size_t off_tp = (((size_t)a.T * p.Kc * 2 + 255) & ~(size_t)255) +
+                          (((size_t)a.M * p.Kc * 2 + 255) & ~(size_t)255);
+    p.nsplit = pre_act_splits(a.K / a.block, a.T);
+    p.tpart = reinterpret_cast<float *>(static_cast<char *>(a.workspace) + off_tp);
+    p.tdone = reinterpret_cast<unsigned int *>(
+        static_cast<char *>(a.workspace) + off_tp +
+        (((size_t)p.nsplit * a.T * 64 * 4 + 255) & ~(size_t)255));
+  }
   const size_t act_smem = pre_act_smem_bytes(a.block, a.rank, a.n_sal);
   cudaError_t e;
-  const dim3 ga((a.T + 15) / 16);
+  if (p.nsplit > 1) {
+    e = cudaMemsetAsync(p.tdone, 0, (size_t)(a.T + 15) / 16 * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 ga((a.T + 15) / 16, p.nsplit);
+#define DVSSQ_PRE_ACT(BB, VV) \
+  L.launch("pre_act", pre_act_kernel<BB, VV>, ga, dim3(BB), act_smem, st, false, p)
   if (a.block == 256)
-    e = L.launch("pre_act", pre_act_kernel<256>, ga, dim3(256), act_smem, st, false, p);
+    e = a.rank <= 16 ? DVSSQ_PRE_ACT(256, 2) : a.rank <= 32 ? DVSSQ_PRE_ACT(256, 4)
+                                                            : DVSSQ_PRE_ACT(256, 8);
   else
-    e = L.launch("pre_act", pre_act_kernel<128>, ga, dim3(128), act_smem, st, false, p);
+    e = a.rank <= 16 ? DVSSQ_PRE_ACT(128, 2) : a.rank <= 32 ? DVSSQ_PRE_ACT(128, 4)
+                                                            : DVSSQ_PRE_ACT(128, 8);
+#undef DVSSQ_PRE_ACT
   if (e != cudaSuccess) return e;
   const long long items = (long long)a.M * (p.Kc / 8);
   const long long mat_blocks = std::min<long long>((items + 255) / 256, (long long)sm_count() * 8);
@@ -484,10 +548,18 @@ cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
 
 cudaError_t prepare_prefill_kernels() {
   cudaError_t e;
-  for (const void *f : {(const void *)pre_act_kernel<256>, (const void *)pre_act_kernel<128>})
-    if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+  const void *acts[] = {(const void *)pre_act_kernel<256, 2>, (const void *)pre_act_kernel<256, 4>,
+                        (const void *)pre_act_kernel<256, 8>, (const void *)pre_act_kernel<128, 2>,
+                        (const void *)pre_act_kernel<128, 4>, (const void *)pre_act_kernel<128, 8>};
+  for (int i = 0; i < 6; ++i) {
+    if ((e = cudaFuncSetAttribute(acts[i], cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
+    if ((e = cudaFuncSetAttribute(acts[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)pre_act_smem_bytes(i < 3 ? 256 : 128, 64, kMaxSalient))) !=
+        cudaSuccess)
+      return e;
+  }
   e = cudaFuncSetAttribute(pre_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)pre_smem_bytes(256));
   if (e != cudaSuccess) return e;
@@ -497,11 +569,7 @@ cudaError_t prepare_prefill_kernels() {
   e = cudaFuncSetAttribute(pre_gemm_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)pre_smem_bytes(64));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(pre_act_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)pre_act_smem_bytes(256, 64, kMaxSalient));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(pre_act_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)pre_act_smem_bytes(128, 64, kMaxSalient));
+  return cudaSuccess;
 }
 
 }  // namespace dvssq
