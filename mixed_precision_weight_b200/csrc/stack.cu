@@ -94,7 +94,8 @@ __device__ __forceinline__ uint32_t stk_splice(uint32_t a, uint32_t b, uint32_t 
 }
 
 // Bounded mbarrier wait that also gives up as soon as another warp of the CTA
-// has flagged an abort.
+// has flagged an abort.  Between polls the warp sleeps briefly, so that a
+// waiting warp does not take issue slots from the warps that compute.
 __device__ __forceinline__ bool stk_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -105,6 +106,7 @@ __device__ __forceinline__ bool stk_wait(uint64_t *bar, uint32_t parity, volatil
       *abort = 1;
       return false;
     }
+    __nanosleep(64);
   }
   return true;
 }
@@ -256,6 +258,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
           *abort = 1;
           break;
         }
+        __nanosleep(32);
       }
     }
     // one thread decides, so that every consumer warp takes the same branches
