@@ -5,6 +5,8 @@ and against the chain of single-layer GPU calls.
   by the GPU encoder with the oracle's SVD factors, two ranks: the fused
   output against the oracle's mlp_block applied layer after layer
   (reading R10), and against the GPU chain gate / up / gelu_mul / down.
+- The same with the MiniCPM Hadamard block (b = 128) and without the rank-r
+  term (rank 0).
 - Full Spark shapes (hidden 2560, intermediate 10240, rank 16 and 24): the
   fused output against the GPU chain of the same packed layers.
 Both sides round g, u, h and each block output to BF16; the fused kernel
@@ -42,7 +44,7 @@ def chain(dv, layers, x):
     return cur
 
 
-def small_stack(dv, L, H, I, ranks, seed):
+def small_stack(dv, L, H, I, ranks, seed, block=256):
     layers, encs = [], []
     for l in range(L):
         mats, es = [], []
@@ -50,10 +52,12 @@ def small_stack(dv, L, H, I, ranks, seed):
             s = seed + 10 * l + which
             W = synth.weight(M, K, seed=s, n_outlier_cols=2, outlier_scale=15.0)
             act = synth.act_scale(K, seed=s)
-            enc = O.encode(f64(W), act.numpy(), 256, ranks[l])
-            U = torch.from_numpy(enc["U"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
-            V = torch.from_numpy(enc["V"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
-            shape, packed, _, _ = gpu_encode(dv, W, act, 256, ranks[l], U=U, V=V)
+            enc = O.encode(f64(W), act.numpy(), block, ranks[l])
+            U = V = None
+            if ranks[l] > 0:
+                U = torch.from_numpy(enc["U"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
+                V = torch.from_numpy(enc["V"].astype(np.float32)).to(torch.bfloat16).cuda().contiguous()
+            shape, packed, _, _ = gpu_encode(dv, W, act, block, ranks[l], U=U, V=V)
             check_codes(shape, packed, enc)
             mats.append((shape, packed))
             es.append(enc)
@@ -80,6 +84,23 @@ def test_stack_matches_oracle_and_chain(dv, ranks):
     assert rel_l2(got, ch) <= 1e-2, rel_l2(got, ch)
     # repeatable: the same inputs give the same bits
     assert torch.equal(stack.forward(x.cuda()), y)
+
+
+@pytest.mark.parametrize("block,ranks", [(128, (24, 8)), (256, (0, 0))])
+def test_stack_block128_and_rank0(dv, block, ranks):
+    # the MiniCPM Hadamard block (H_128) and a stack without the rank-r term
+    H, I = 512, 1024
+    layers, encs = small_stack(dv, 2, H, I, ranks, seed=51 + ranks[0], block=block)
+    x = synth.activations(1, H, seed=13, n_outlier=3, outlier_scale=25.0)
+    y = dv.MlpStack(layers).forward(x.cuda())
+    torch.cuda.synchronize()
+    assert dv.dvssq_device_error(clear=True) == 0
+    ref = f64(x)
+    for eg, eu, ed in encs:       # rank 0: the oracle's factors are [M][0] and [0][K]
+        ref = O.rn_bf16(O.mlp_block(eg, eu, ed, ref))
+    assert rel_l2(f64(y), ref) <= 3e-2, rel_l2(f64(y), ref)
+    ch = f64(chain(dv, layers, x.cuda()))
+    assert rel_l2(f64(y), ch) <= 1e-2, rel_l2(f64(y), ch)
 
 
 def test_stack_output_may_alias_input(dv):
