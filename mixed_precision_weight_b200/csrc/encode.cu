@@ -250,7 +250,15 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(
   for (int col = threadIdx.x; col < B; col += blockDim.x) {
     const int j = kb * B + col;
     double tot = 0.0;
-    for (int sg = 0; sg < nsg; ++sg) tot = __dadd_rn(tot, __ldcg(gpart + (size_t)sg * K + j));
+    for (int sg0 = 0; sg0 < nsg; sg0 += 16) {
+      double gv[16];          // loads in flight together, adds in ascending order
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        gv[u] = sg0 + u < nsg ? __ldcg(gpart + (size_t)(sg0 + u) * K + j) : 0.0;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (sg0 + u < nsg) tot = __dadd_rn(tot, gv[u]);
+    }
     const double s = __dmul_rn((double)act_scale[j], __dsqrt_rn(tot));
     bad += !isfinite(s);
     score[j] = s;
@@ -320,23 +328,70 @@ __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
     for (int w = tid; w < (K + 31) / 32; w += kSelThreads) sal_prefix[w] = 0;
     return;
   }
-  if (in_smem)
-    for (int j = tid; j < K; j += kSelThreads) skeys[j] = order_key(score[j]);
-  __syncthreads();
-  auto key = [&](int j) { return in_smem ? skeys[j] : order_key(score[j]); };
   // this thread's keys j = tid + 1024 i live in registers while K <= 16384
+  // (all loads issued together), and in shared memory for the index-order
+  // passes at the end
   constexpr int KPT = kSelSmemKeys / kSelThreads;
   unsigned long long rk[KPT];
+  double sv[KPT];
 #pragma unroll
   for (int i = 0; i < KPT; ++i) {
     const int j = tid + i * kSelThreads;
-    rk[i] = (in_smem && j < K) ? skeys[j] : 0ull;
+    sv[i] = (in_smem && j < K) ? __ldcg(score + j) : 0.0;
   }
+  unsigned long long kmax = 0ull, kmin = ~0ull;
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const int j = tid + i * kSelThreads;
+    rk[i] = (in_smem && j < K) ? order_key(sv[i]) : 0ull;
+    if (in_smem && j < K) {
+      skeys[j] = rk[i];
+      kmax = max(kmax, rk[i]);
+      kmin = min(kmin, rk[i]);
+    }
+  }
+  auto key = [&](int j) { return in_smem ? skeys[j] : order_key(score[j]); };
   const int iters = (K + kSelThreads - 1) / kSelThreads;
-
-  unsigned long long prefix = 0, pmask = 0;
+  if (!in_smem)
+    for (int j = tid; j < K; j += kSelThreads) {
+      const unsigned long long k = key(j);
+      kmax = max(kmax, k);
+      kmin = min(kmin, k);
+    }
+  // the high bits every key shares need no radix pass: start at the 8-bit
+  // digit that holds the highest bit where the largest and smallest keys differ
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+  }
+  __shared__ unsigned long long s_kmax[32], s_kmin[32];
+  if (lane == 0) {
+    s_kmax[warp] = kmax;
+    s_kmin[warp] = kmin;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    kmax = s_kmax[lane];
+    kmin = s_kmin[lane];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    }
+    if (lane == 0) {
+      s_kmax[0] = kmax;
+      s_kmin[0] = kmin;
+    }
+  }
+  __syncthreads();
+  const unsigned long long diff = s_kmax[0] ^ s_kmin[0];
+  const int hb = diff ? 63 - __clzll((long long)diff) : 0;      // highest differing bit
+  const int top = (hb / 8) * 8;                                  // its digit's shift
+  unsigned long long pmask = top >= 56 ? 0ull : ~((1ull << (top + 8)) - 1ull);
+  unsigned long long prefix = s_kmax[0] & pmask;
   unsigned int krem = (unsigned int)n_sal;
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  for (int shift = top; shift >= 0; shift -= 8) {
     if (tid < 256) hist[tid] = 0;
     __syncthreads();
     auto count = [&](unsigned long long k, int j) {
