@@ -40,6 +40,9 @@ constexpr int kSlab = 256;                   // rotated columns per slab
 constexpr int kUnitRows = 16;                // rows per work unit
 constexpr int kDecWarps = 16;
 constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecCons = kDecWarps - 1;        // consumer warps (warp 0 issues the weight stream)
+constexpr int kDecConsThreads = 32 * kDecCons;
+constexpr int kDecNV = (64 + kDecCons - 1) / kDecCons;   // rank rows per consumer warp (rank <= 64)
 constexpr int kDecMaxUnits = 48;             // units per CTA staged at once
 constexpr int kDecMaxSlabs = 4;              // distinct slabs per CTA
 constexpr int kQ4Unit = kUnitRows * 128;     // one q4 box: 16 rows x 128 B
@@ -53,8 +56,13 @@ constexpr int kSmemLimit = 232448;           // opt-in shared memory per CTA (22
 
 // Shared-memory layout of dec_main: byte offsets from the 1024-aligned base.
 struct DecLayout {
-  int q4, s4, q8, xq, xs, corr, c8, s8, colpos, samp, scr, meta, bars, total;
+  int q4, s4, q8, xq, xs, corr, c8, s8, colpos, samp, scr, meta, bars, vs, total;
 };
+
+// Barrier among the consumer warps only (the producer warp leaves early).
+__device__ __forceinline__ void dec_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecConsThreads) : "memory");
+}
 
 struct DecodeParams {
   int M, K, T, n_sal, rank, block;
@@ -119,7 +127,8 @@ __device__ __forceinline__ void dequant_q8_biased(uint32_t w, uint32_t &p01, uin
 template <int B, int NT>
 __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
     const __grid_constant__ CUtensorMap mq4, const __grid_constant__ CUtensorMap ms4,
-    const __grid_constant__ CUtensorMap mq8, DecodeParams p) {
+    const __grid_constant__ CUtensorMap mq8, const __grid_constant__ CUtensorMap mv,
+    DecodeParams p) {
   constexpr int NTOK = 8 * NT;
   constexpr int P = B / 16;                 // threads per Hadamard block-row
   constexpr int NBLK = kSlab / B;           // Hadamard blocks per slab
@@ -137,7 +146,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
   int *samp = reinterpret_cast<int *>(base + p.L.samp);       // [kSamples]
   float *scr = reinterpret_cast<float *>(base + p.L.scr);
   int *meta = reinterpret_cast<int *>(base + p.L.meta);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(base + p.L.bars);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + p.L.bars);   // [upc_max + 2]
+  uint16_t *vs = reinterpret_cast<uint16_t *>(base + p.L.vs);       // [rank][kSlab] BF16
   int *lo = meta;                                   // [kDecMaxSlabs + 1]
   int *lo16 = meta + 8;                             // [kDecMaxSlabs]
   int *nch = meta + 16;                             // [kDecMaxSlabs]
@@ -163,13 +173,39 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
     return;
   }
 
+  // the first slab whose t share this CTA writes (the CTA holding its first unit)
+  int own_si = -1;
+  for (int si = 0; si < ns; ++si)
+    if ((s_first + si) * p.ntile >= u0) { own_si = si; break; }
+  uint64_t *q8bar = bars + p.upc_max;       // consumers -> producer: the INT8 layout is ready
+  uint64_t *vbar = bars + p.upc_max + 1;    // V rows of the owned slab have landed
+
   // ------------- before the dependency wait: packed weights only -------------
-  // warp 0: one lane per unit initialises its barrier and issues its boxes
+  // Warp 0 is the producer: it initialises the barriers, issues the V rows
+  // of the owned slab and every weight box, waits for the consumers' INT8
+  // layout and issues the INT8 chunks, then leaves.  An issue can block while
+  // the copy queue is full; the consumers (warps 1..15, named barrier 1)
+  // never wait behind it.
   if (warp == 0) {
     for (int k = lane; k < nu; k += 32) mbar_init(&bars[k], 2);
+    if (lane == 0) {
+      mbar_init(q8bar, 1);
+      mbar_init(vbar, 1);
+    }
     fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&mq4);
+      if (own_si >= 0 && p.rank > 0) {
+        mbar_arrive_expect_tx(vbar, (uint32_t)(p.rank * kSlab * 2));
+        tma_load_2d(vs, &mv, kSlab * (s_first + own_si), 0, vbar);
+      } else {
+        mbar_arrive(vbar);
+      }
+    }
     __syncwarp();
-    if (lane == 0) prefetch_tensormap(&mq4);
     const uint32_t bytes = kQ4Unit + (p.s4_tma ? kS4Unit : 0);
     for (int k = lane; k < nu; k += 32) {
       const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
@@ -178,13 +214,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       if (p.s4_tma)
         tma_load_2d(s4s + k * (kS4Unit / 2), &ms4, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
     }
+    // INT8 chunks: staged by TMA when they fit, read from global memory otherwise
+    const bool ready = mbar_wait(q8bar, 0);
+    const int staged = ready ? flags[0] : 0;
+    for (int k = lane; k < nu; k += 32) {
+      const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
+      const int n = staged ? nch[si] : 0;
+      mbar_arrive_expect_tx(&bars[k], (uint32_t)(n * kQ8Chunk));
+      for (int c = 0; c < n; ++c)
+        tma_load_2d(q8s + q8off[k] + c * kQ8Chunk, &mq8, lo16[si] + 16 * c, tile * kUnitRows,
+                    &bars[k]);
+    }
+    return;
   }
+  const int ctid = tid - 32, cw = warp - 1;
   const int KG = p.K / 64;
   const int step = (p.n_sal + kSamples - 1) / kSamples;
   if (p.n_sal > 0)
-    for (int i = tid; i < kSamples; i += kDecThreads)
+    for (int i = ctid; i < kSamples; i += kDecConsThreads)
       samp[i] = __ldg(p.sal_idx + min(i * step, p.n_sal - 1));
-  for (int i = tid; i < nu * kUnitRows; i += kDecThreads) {
+  for (int i = ctid; i < nu * kUnitRows; i += kDecConsThreads) {
     const int k = i >> 4, r = i & 15;
     const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
     const int m = tile * kUnitRows + r;
@@ -192,34 +241,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
   }
   if (!p.s4_tma) {
     // scale rows whose stride a tensor map cannot carry: plain loads
-    for (int i = tid; i < nu * kUnitRows * 8; i += kDecThreads) {
+    for (int i = ctid; i < nu * kUnitRows * 8; i += kDecConsThreads) {
       const int k = i >> 7, r = (i >> 3) & 15, j = i & 7;
       const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
       const int m = tile * kUnitRows + r, gcol = 8 * (s >> 1) + j;
       s4s[i] = (m < p.M && gcol < KG) ? p.s4[(size_t)m * KG + gcol] : (uint16_t)0;
     }
   }
-  for (int i = tid; i < ns * kSlab; i += kDecThreads) colpos[i] = -1;
-  for (int i = tid; i < ns * NTOK * kXsRow / 2; i += kDecThreads)
+  for (int i = ctid; i < ns * kSlab; i += kDecConsThreads) colpos[i] = -1;
+  for (int i = ctid; i < ns * NTOK * kXsRow / 2; i += kDecConsThreads)
     reinterpret_cast<uint32_t *>(xs)[i] = 0u;
-  // rows of V for the slabs whose first unit this CTA holds: warm L2
+  // rows of V for further owned slabs (rare): warm L2
   if (p.rank > 0)
-    for (int si = 0; si < ns; ++si) {
+    for (int si = own_si + 1; own_si >= 0 && si < ns; ++si) {
       const int s = s_first + si;
       if (s * p.ntile < u0) continue;
-      for (int i = tid; i < p.rank * 4; i += kDecThreads) {
+      for (int i = ctid; i < p.rank * 4; i += kDecConsThreads) {
         const int rr = i >> 2, col = kSlab * s + 64 * (i & 3);
         if (col < p.K)
           asm volatile("prefetch.global.L2 [%0];" ::"l"(p.V + (size_t)rr * p.K + col));
       }
     }
-  __syncthreads();
+  dec_consumer_sync();
 
   // salient entries of each slab: lo[b] = #{e : sal_idx[e] < 256 (s_first + b)}
-  if (warp <= ns) {
+  if (cw <= ns) {
     int l = 0;
     if (p.n_sal > 0) {
-      const int v = kSlab * (s_first + warp);
+      const int v = kSlab * (s_first + cw);
       int j = 0;
       for (int i0 = 0; i0 < kSamples; i0 += 32) {
         const int i = i0 + lane;
@@ -234,17 +283,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
       l = lb + cnt;
     }
-    if (lane == 0) lo[warp] = l;
+    if (lane == 0) lo[cw] = l;
   }
-  __syncthreads();
-  if (tid < ns) {
-    const int a = lo[tid], b = lo[tid + 1];
-    lo16[tid] = a & ~15;
-    nch[tid] = b > a ? (b - (a & ~15) + 15) >> 4 : 0;
+  dec_consumer_sync();
+  if (ctid < ns) {
+    const int a = lo[ctid], b = lo[ctid + 1];
+    lo16[ctid] = a & ~15;
+    nch[ctid] = b > a ? (b - (a & ~15) + 15) >> 4 : 0;
   }
-  __syncthreads();
-  if (warp == 0) {
-    // q8 staging offsets: exclusive scan of the units' chunk bytes
+  dec_consumer_sync();
+  if (cw == 0) {
+    // q8 staging offsets: exclusive scan of the units' chunk bytes, then the
+    // producer may issue the chunks (the arrive releases these writes)
     int run = 0;
     for (int k0 = 0; k0 < nu; k0 += 32) {
       const int k = k0 + lane;
@@ -258,50 +308,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       if (k < nu) q8off[k] = run + inc - b;
       run += __shfl_sync(0xffffffffu, inc, 31);
     }
-    const int staged = run <= p.q8_budget;
-    if (lane == 0) flags[0] = staged;
-    for (int k = lane; k < nu; k += 32) {
-      const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
-      const int n = staged ? nch[si] : 0;
-      mbar_arrive_expect_tx(&bars[k], (uint32_t)(n * kQ8Chunk));
-      for (int c = 0; c < n; ++c)
-        tma_load_2d(q8s + q8off[k] + c * kQ8Chunk, &mq8, lo16[si] + 16 * c, tile * kUnitRows,
-                    &bars[k]);
-    }
+    if (lane == 0) flags[0] = run <= p.q8_budget;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q8bar);
   } else {
     // column -> position of each salient entry in its slab's chunk range
     for (int si = 0; si < ns; ++si) {
       const int a = lo[si], b = lo[si + 1], s = s_first + si;
-      for (int e = a + tid - 32; e < b; e += kDecThreads - 32) {
+      for (int e = a + ctid - 32; e < b; e += kDecConsThreads - 32) {
         const int col = __ldg(p.sal_idx + e) - kSlab * s;
         if (col >= 0 && col < kSlab) colpos[si * kSlab + col] = (int16_t)(e - (a & ~15));
       }
     }
   }
-  __syncthreads();
+  dec_consumer_sync();
 
   // ------------------------- after the wait: activations -------------------------
   pdl_wait();
   pdl_launch_dependents();
 
-  // V rows of the first owned slab, into registers (consumed after the FWHT)
-  int own_si = -1;
-  for (int si = 0; si < ns; ++si)
-    if ((s_first + si) * p.ntile >= u0) { own_si = si; break; }
-  uint4 vreg[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    vreg[i] = make_uint4(0u, 0u, 0u, 0u);
-    const int rr = warp + kDecWarps * i, col = kSlab * (s_first + own_si) + 8 * lane;
-    if (own_si >= 0 && rr < p.rank && col < p.K)
-      vreg[i] = *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + col);
-  }
-
   // rotate x for the CTA's slabs: block-row br = (si * NBLK + blk) * T + tok
   {
     const int nbr = ns * NBLK * p.T;
-    const int grp = tid / P, t = tid % P;
-    const int wgrp = (warp * 32) / P;            // first group of this warp
+    const int grp = ctid / P, t = ctid % P;
+    const int wgrp = (cw * 32) / P;              // first group of this warp
     for (int br0 = 0; br0 < nbr; br0 += p.nscr) {
       if (wgrp >= p.nscr || br0 + wgrp >= nbr) continue;   // whole warp idle
       const int br = br0 + grp;
@@ -350,10 +380,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       }
     }
   }
-  __syncthreads();
+  dec_consumer_sync();
 
   // salient bias terms: c8[si][tok] = 1152 * sum of the slab's salient x
-  for (int q = warp; q < ns * p.T; q += kDecWarps) {
+  for (int q = cw; q < ns * p.T; q += kDecCons) {
     const int si = q / p.T, tok = q % p.T;
     const __half *xrow = xs + (size_t)(si * NTOK + tok) * kXsRow;
     float sum = 0.0f;
@@ -363,53 +393,78 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
     if (lane == 0) c8[si * NTOK + tok] = 1152.0f * sum;
   }
 
-  // t share of each owned slab: tpart[s][rr][tok] = sum_j V[rr][j] x_rot[j]
-  if (p.rank > 0)
+  // t share of each owned slab: tpart[s][rr][tok] = sum_j V[rr][j] x_rot[j],
+  // on the tensor cores against the FP16 x_rot already in shared memory:
+  // A = V in the same column order, odd columns scaled by 16 (x_rot holds
+  // them divided by 16).  Warps split the 16-rank tiles and the K steps;
+  // their partials go to the rotation scratch (free now) and are added in
+  // warp order.  The first owned slab's V rows came by TMA; a further one is
+  // read from global memory.
+  const bool v_ok = p.rank == 0 || mbar_wait(vbar, 0);
+  if (p.rank > 0) {
+    const int mtiles = (p.rank + 15) / 16;
+    const int kgp = max(1, kDecCons / mtiles);       // warps per rank tile
+    float *tps = scr;                                // [mtiles][kgp][16][NTOK]
+    const int mt = cw / kgp, kg = cw - mt * kgp;
     for (int si = own_si; si >= 0 && si < ns; ++si) {
       const int s = s_first + si;
       if (s * p.ntile < u0) continue;
-      if (si != own_si) {
+      if (mt < mtiles) {
+        const bool staged_v = si == own_si && v_ok;
+        float d[NT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          vreg[i] = make_uint4(0u, 0u, 0u, 0u);
-          const int rr = warp + kDecWarps * i, col = kSlab * s + 8 * lane;
-          if (rr < p.rank && col < p.K)
-            vreg[i] = *reinterpret_cast<const uint4 *>(p.V + (size_t)rr * p.K + col);
-        }
-      }
-      for (int tok = 0; tok < p.T; ++tok) {
-        float xv[8];
-        const __half *xrow = xq + (size_t)(si * NTOK + tok) * kXRow;
+        for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.0f;
+        for (int ks = kg; ks < kSlab / 16; ks += kgp) {
+          const int k0 = 16 * ks;
+          uint32_t a[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int cn = 8 * lane + j;
-          const float hv = __half2float(xrow[(cn & ~15) + inv_perm16(cn & 15)]);
-          xv[j] = (cn & 1) ? hv * 16.0f : hv;
-        }
+          for (int h = 0; h < 4; ++h) {
+            const int rr = 16 * mt + g + 8 * (h & 1);
+            const int pos = k0 + 2 * tig + 8 * (h >> 1);
+            __half e[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int rr = warp + kDecWarps * i;
-          if (rr >= p.rank) break;
-          const uint32_t w[4] = {vreg[i].x, vreg[i].y, vreg[i].z, vreg[i].w};
-          float d = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            d = fmaf(bf16_bits_to_f32(w[q] & 0xFFFFu), xv[2 * q], d);
-            d = fmaf(bf16_bits_to_f32(w[q] >> 16), xv[2 * q + 1], d);
+            for (int q = 0; q < 2; ++q) {
+              const int col = ((pos + q) & ~15) + perm16((pos + q) & 15);
+              float v = 0.0f;
+              if (rr < p.rank && kSlab * s + col < p.K)
+                v = bf16_bits_to_f32(staged_v ? vs[rr * kSlab + col]
+                                              : p.V[(size_t)rr * p.K + kSlab * s + col]);
+              e[q] = __float2half_rn((col & 1) ? v * 16.0f : v);
+            }
+            a[h] = pack_half2(e[0], e[1]);
           }
 #pragma unroll
-          for (int o = 16; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-          if (lane == 0) p.tpart[((size_t)s * p.rank + rr) * p.T + tok] = d;
+          for (int nt = 0; nt < NT; ++nt) {
+            const __half *xrow = xq + (size_t)(si * NTOK + 8 * nt + g) * kXRow + k0 + 2 * tig;
+            const uint32_t b0 = *reinterpret_cast<const uint32_t *>(xrow);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t *>(xrow + 8);
+            mma_16816(d[nt], a, b0, b1, d[nt]);
+          }
         }
+        float *dst = tps + (size_t)(mt * kgp + kg) * 16 * NTOK;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[(g + 8 * (i >> 1)) * NTOK + 8 * nt + 2 * tig + (i & 1)] = d[nt][i];
       }
+      dec_consumer_sync();
+      for (int i = ctid; i < p.rank * p.T; i += kDecConsThreads) {
+        const int rr = i / p.T, tok = i - rr * p.T, m16 = rr >> 4, r = rr & 15;
+        float v = 0.0f;
+        for (int j = 0; j < kgp; ++j) v += tps[((size_t)(m16 * kgp + j) * 16 + r) * NTOK + tok];
+        p.tpart[((size_t)s * p.rank + rr) * p.T + tok] = v;
+      }
+      dec_consumer_sync();
     }
-  __syncthreads();
+  }
+  dec_consumer_sync();
 
   // ----------------------------------- units -----------------------------------
   const bool staged = flags[0] != 0;
   uint32_t bq[NT == 1 ? 4 : 1][8];
   int cur = -1;
-  for (int k = warp; k < nu; k += kDecWarps) {
+  for (int k = cw; k < nu; k += kDecCons) {
     const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
     if constexpr (NT == 1) {
       if (si != cur) {
@@ -660,7 +715,7 @@ int slabs_spanned(long long units, int grid, int ntile, int c) {
 }
 
 // Grid, per-CTA maxima and the shared-memory layout of one decode call.
-DecPlan dec_plan(int M, int K, int block, int T, int nsm) {
+DecPlan dec_plan(int M, int K, int block, int T, int rank, int nsm) {
   DecPlan d{};
   d.nslab = (K + kSlab - 1) / kSlab;
   d.ntile = (M + kUnitRows - 1) / kUnitRows;
@@ -699,9 +754,12 @@ DecPlan dec_plan(int M, int K, int block, int T, int nsm) {
   L.s8 = off;     off += al(d.upc_max * kUnitRows * 4, 128);
   L.colpos = off; off += al(d.ns_max * kSlab * 2, 128);
   L.samp = off;   off += kSamples * 4;
-  L.scr = off;    off += al(d.nscr * scr_elems * 4, 128);
+  // the rotation scratch also holds the t-share partials: at most 15 warps x
+  // 16 ranks x the token tile, FP32
+  L.scr = off;    off += al(std::max(d.nscr * scr_elems * 4, kDecCons * 16 * d.ntok * 4), 128);
   L.meta = off;   off += 512;
-  L.bars = off;   off += al(d.upc_max * 8, 128);
+  L.bars = off;   off += al((d.upc_max + 2) * 8, 128);
+  L.vs = off;     off += al(rank * kSlab * 2, 128);
   L.q8 = off;
   const int room = kSmemLimit - 1024 - off;
   d.q8_budget = std::max(0, std::min(room, d.upc_max * 4 * kQ8Chunk)) / kQ8Chunk * kQ8Chunk;
@@ -734,7 +792,7 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
     const cudaError_t e = launch_decode_row(a, st, L);
     if (e != cudaErrorNotSupported) return e;
   }
-  const DecPlan d = dec_plan(a.M, a.K, a.block, a.T, sm_count());
+  const DecPlan d = dec_plan(a.M, a.K, a.block, a.T, a.rank, sm_count());
   if (!d.ok) {
     set_last_error("decode: no shared-memory plan fits this shape");
     return cudaErrorInvalidConfiguration;
@@ -755,7 +813,7 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   p.part = reinterpret_cast<float *>(take((size_t)d.nslab * a.T * a.M * 4));
   p.tpart = reinterpret_cast<float *>(take((size_t)d.nslab * a.rank * a.T * 4 + 16));
 
-  CUtensorMap mq4, ms4, mq8;
+  CUtensorMap mq4, ms4, mq8, mv;
   if (encode_tmap_2d(&mq4, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q4, (uint64_t)a.K / 2, (uint64_t)a.M,
                      (uint64_t)a.K / 2, 128, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B) !=
       CUDA_SUCCESS)
@@ -767,6 +825,13 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
                                  (uint64_t)a.M, (uint64_t)a.K / 32, 8, kUnitRows,
                                  CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
     p.s4_tma = 0;
+  // V rows of one slab: box {256 columns, rank rows}
+  mv = mq4;    // never read when rank == 0
+  if (a.rank > 0 &&
+      encode_tmap_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.V, (uint64_t)a.K, (uint64_t)a.rank,
+                     (uint64_t)a.K * 2, kSlab, (uint32_t)a.rank, CU_TENSOR_MAP_SWIZZLE_NONE) !=
+          CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   mq8 = mq4;   // never read when there are no salient columns
   if (a.n_sal > 0 &&
       encode_tmap_2d(&mq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q8, (uint64_t)a.n_sal, (uint64_t)a.M,
@@ -779,14 +844,14 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   const size_t smem = d.L.total;
   if (a.block == 256)
     e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<256, 1>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, p)
+                             mq4, ms4, mq8, mv, p)
                   : L.launch("dec_main", dec_main_kernel<256, 2>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, p);
+                             mq4, ms4, mq8, mv, p);
   else
     e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<128, 1>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, p)
+                             mq4, ms4, mq8, mv, p)
                   : L.launch("dec_main", dec_main_kernel<128, 2>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, p);
+                             mq4, ms4, mq8, mv, p);
   if (e != cudaSuccess) return e;
   return L.launch("dec_tail", dec_tail_kernel, dim3((a.M + kTailThreads / 4 - 1) / (kTailThreads / 4), a.T),
                   dim3(kTailThreads), 0, st, true, p);
