@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
   int *lo16 = meta + 8;                             // [kDecMaxSlabs]
   int *nch = meta + 16;                             // [kDecMaxSlabs]
   int *q8off = meta + 24;                           // [kDecMaxUnits]
-  int *flags = meta + 24 + kDecMaxUnits;            // [0]: q8 staged
+  int *flags = meta + 24 + kDecMaxUnits;            // [0]: the INT8 layout is valid
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
@@ -214,12 +214,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       if (p.s4_tma)
         tma_load_2d(s4s + k * (kS4Unit / 2), &ms4, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
     }
-    // INT8 chunks: staged by TMA when they fit, read from global memory otherwise
+    // INT8 chunks: a unit's chunks are staged by TMA when they fit in the
+    // budget (units in order), read from global memory otherwise
     const bool ready = mbar_wait(q8bar, 0);
-    const int staged = ready ? flags[0] : 0;
     for (int k = lane; k < nu; k += 32) {
       const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile, si = s - s_first;
-      const int n = staged ? nch[si] : 0;
+      const int n = (ready && q8off[k] + nch[si] * kQ8Chunk <= p.q8_budget) ? nch[si] : 0;
       mbar_arrive_expect_tx(&bars[k], (uint32_t)(n * kQ8Chunk));
       for (int c = 0; c < n; ++c)
         tma_load_2d(q8s + q8off[k] + c * kQ8Chunk, &mq8, lo16[si] + 16 * c, tile * kUnitRows,
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       if (k < nu) q8off[k] = run + inc - b;
       run += __shfl_sync(0xffffffffu, inc, 31);
     }
-    if (lane == 0) flags[0] = run <= p.q8_budget;
+    if (lane == 0) flags[0] = 1;
     __syncwarp();
     if (lane == 0) mbar_arrive(q8bar);
   } else {
@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
   dec_consumer_sync();
 
   // ----------------------------------- units -----------------------------------
-  const bool staged = flags[0] != 0;
+  (void)flags;
   uint32_t bq[NT == 1 ? 4 : 1][8];
   int cur = -1;
   for (int k = cw; k < nu; k += kDecCons) {
@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       const int mlo = tile * kUnitRows + g;
       for (int c = 0; c < nc; ++c) {
         uint32_t wl = 0u, wh = 0u;
-        if (staged) {
+        if (q8off[k] + nc * kQ8Chunk <= p.q8_budget) {
           const uint8_t *cb = q8s + q8off[k] + c * kQ8Chunk;
           wl = *reinterpret_cast<const uint32_t *>(cb + g * 16 + 4 * tig);
           wh = *reinterpret_cast<const uint32_t *>(cb + (g + 8) * 16 + 4 * tig);
@@ -762,7 +762,7 @@ DecPlan dec_plan(int M, int K, int block, int T, int rank, int nsm) {
   L.vs = off;     off += al(rank * kSlab * 2, 128);
   L.q8 = off;
   const int room = kSmemLimit - 1024 - off;
-  d.q8_budget = std::max(0, std::min(room, d.upc_max * 4 * kQ8Chunk)) / kQ8Chunk * kQ8Chunk;
+  d.q8_budget = std::max(0, std::min(room, d.upc_max * 17 * kQ8Chunk)) / kQ8Chunk * kQ8Chunk;
   off += d.q8_budget;
   L.total = off + 1024;
   d.ok = room >= 0 && d.upc_max <= kDecMaxUnits && d.ns_max <= kDecMaxSlabs;
