@@ -95,13 +95,31 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without // comments and blank lines: a comment edit does
+    not change the kernel, so it must not invalidate a capture."""
+    out = []
+    for line in text.splitlines():
+        q, cut = False, len(line)
+        for i, ch in enumerate(line):
+            if ch == '"' and (i == 0 or line[i - 1] != "\\"):
+                q = not q
+            elif not q and line.startswith("//", i):
+                cut = i
+                break
+        line = line[:cut].rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def source_hash(kernel=None):
     d = os.path.join(ROOT, "mixed_precision_weight_b200", "csrc")
     files = KERNEL_SOURCES.get(kernel) or tuple(sorted(os.listdir(d)))
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update((f + _code_only(fh.read())).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,23 +7,29 @@
 // one contiguous, equal share per CTA (one CTA per SM), so every SM streams
 // the same number of weight bytes.
 //
-// dec_main (programmatic dependent launch):
-//   before the dependency wait - reads only the packed weights: TMA brings
-//     every unit's q4 box (16 x 128 B, 128B swizzle) and s4 box into shared
-//     memory; a two-round parallel search of sal_idx finds each slab's
-//     salient entries, whose INT8 columns then follow by TMA in 16-entry
-//     chunks; s8 is staged.
+// dec_main (programmatic dependent launch), warp 0 a producer, warps 1..15
+// consumers that never wait behind it:
+//   before the dependency wait - reads only the packed weights.  The
+//     producer issues by TMA the V rows of the slab whose t share the CTA
+//     writes, then every unit's q4 box (16 x 128 B, 128B swizzle) and s4
+//     box.  The consumers find each slab's salient entries (a two-round
+//     parallel search of sal_idx), lay out the INT8 chunks (16 entries each)
+//     unit by unit and hand the layout to the producer through an mbarrier;
+//     the producer stages the chunks of the units that fit in the free
+//     shared memory, in unit order, and exits.  Units past that budget read
+//     their chunks from global memory (L2).
 //   after the wait - the CTA rotates x for its (at most kDecMaxSlabs) slabs
 //     itself (16-thread Kronecker FWHT, fp32), stores it as FP16 in the
 //     GEMV's k-order, scatters the salient entries, and forms per-group
-//     bias terms.  Warps then take units round-robin: nibbles become FP16
-//     1024+u (even columns) or 1024+16u (odd columns, whose activations are
-//     stored pre-divided by 16) with one LOP3 each; the MMA chain of a
-//     64-column group starts from minus the group's bias term, so its sum is
-//     the exact-code dot product; acc += s4 * group sum.  The salient chunks
-//     run the same way (1152 + q) and are scaled by s8.  Each unit writes its
-//     16 x T partial for its slab; the CTA that holds a slab's first unit
-//     also writes that slab's share of t = V x_rot.
+//     bias terms.  The owned slab's t share (V x_rot over 256 columns) runs
+//     on the tensor cores, its k range split over the warps and the warps'
+//     pieces added in warp order.  Warps then take units round-robin:
+//     nibbles become FP16 1024+u (even columns) or 1024+16u (odd columns,
+//     whose activations are stored pre-divided by 16) with one LOP3 each;
+//     the MMA chain of a 64-column group starts from minus the group's bias
+//     term, so its sum is the exact-code dot product; acc += s4 * group sum.
+//     The salient chunks run the same way (1152 + q) and are scaled by s8.
+//     Each unit writes its 16 x T partial for its slab.
 // dec_tail: y = sum over slabs of the partials (slab order, deterministic)
 //   + U t + bias, in FP32, optionally rounded to BF16.
 #include "common.cuh"
