@@ -70,10 +70,22 @@ __device__ __forceinline__ void dec_consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kDecConsThreads) : "memory");
 }
 
+// Tiles 4i..4i+3 of one slab whose units all lie in the CTA's range travel
+// as one q4 box (and one s4 box) that lands exactly where four single-unit
+// boxes would.  Returns the index within the CTA of the quad's first unit,
+// or -1 for a unit staged on its own.
+__device__ __forceinline__ int quad_lead(int u, int u0, int u1, int ntile, int quad) {
+  if (!quad) return -1;
+  const int s = u / ntile, tq = (u - s * ntile) & ~3;
+  const int uq = s * ntile + tq;
+  return (tq + 3 < ntile && uq >= u0 && uq + 3 < u1) ? uq - u0 : -1;
+}
+
 struct DecodeParams {
   int M, K, T, n_sal, rank, block;
   int nslab, ntile, units, grid, upc_max, ns_max, ntok, nscr;
   int q8_budget, s4_tma;
+  int quad;       // four consecutive tiles of a slab may travel as one box
   float c;
   const uint16_t *s4;
   const int32_t *sal_idx;
@@ -134,6 +146,7 @@ template <int B, int NT>
 __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
     const __grid_constant__ CUtensorMap mq4, const __grid_constant__ CUtensorMap ms4,
     const __grid_constant__ CUtensorMap mq8, const __grid_constant__ CUtensorMap mv,
+    const __grid_constant__ CUtensorMap mq4q, const __grid_constant__ CUtensorMap ms4q,
     DecodeParams p) {
   constexpr int NTOK = 8 * NT;
   constexpr int P = B / 16;                 // threads per Hadamard block-row
@@ -215,10 +228,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
     const uint32_t bytes = kQ4Unit + (p.s4_tma ? kS4Unit : 0);
     for (int k = lane; k < nu; k += 32) {
       const int u = u0 + k, s = u / p.ntile, tile = u - s * p.ntile;
-      mbar_arrive_expect_tx(&bars[k], bytes);
-      tma_load_2d(q4s + k * kQ4Unit, &mq4, s * 128, tile * kUnitRows, &bars[k]);
-      if (p.s4_tma)
-        tma_load_2d(s4s + k * (kS4Unit / 2), &ms4, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
+      const int lead = quad_lead(u, u0, u1, p.ntile, p.quad);
+      if (lead == k) {
+        mbar_arrive_expect_tx(&bars[k], 4 * bytes);
+        tma_load_2d(q4s + k * kQ4Unit, &mq4q, s * 128, tile * kUnitRows, &bars[k]);
+        if (p.s4_tma)
+          tma_load_2d(s4s + k * (kS4Unit / 2), &ms4q, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
+      } else if (lead >= 0) {
+        mbar_arrive(&bars[k]);          // its data comes with the quad's first unit
+      } else {
+        mbar_arrive_expect_tx(&bars[k], bytes);
+        tma_load_2d(q4s + k * kQ4Unit, &mq4, s * 128, tile * kUnitRows, &bars[k]);
+        if (p.s4_tma)
+          tma_load_2d(s4s + k * (kS4Unit / 2), &ms4, 8 * (s >> 1), tile * kUnitRows, &bars[k]);
+      }
     }
     // INT8 chunks: a unit's chunks are staged by TMA when they fit in the
     // budget (units in order), read from global memory otherwise
@@ -486,6 +509,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       }
     }
     if (!mbar_wait(&bars[k], 0)) break;
+    {
+      const int lead = quad_lead(u, u0, u1, p.ntile, p.quad);
+      if (lead >= 0 && lead != k && !mbar_wait(&bars[lead], 0)) break;
+    }
     const uint8_t *bx = q4s + k * kQ4Unit;
     const uint16_t *sb = s4s + k * (kS4Unit / 2) + 4 * (s & 1);
     const uint2 sl = *reinterpret_cast<const uint2 *>(sb + g * 8);
@@ -831,6 +858,15 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
                                  (uint64_t)a.M, (uint64_t)a.K / 32, 8, kUnitRows,
                                  CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
     p.s4_tma = 0;
+  // four tiles of one slab per box (the same bytes, a quarter of the copies)
+  CUtensorMap mq4q = mq4, ms4q = mq4;
+  p.quad = encode_tmap_2d(&mq4q, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q4, (uint64_t)a.K / 2,
+                          (uint64_t)a.M, (uint64_t)a.K / 2, 128, 4 * kUnitRows,
+                          CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS &&
+           (!p.s4_tma ||
+            encode_tmap_2d(&ms4q, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s4, (uint64_t)a.K / 64,
+                           (uint64_t)a.M, (uint64_t)a.K / 32, 8, 4 * kUnitRows,
+                           CU_TENSOR_MAP_SWIZZLE_NONE) == CUDA_SUCCESS);
   // V rows of one slab: box {256 columns, rank rows}
   mv = mq4;    // never read when rank == 0
   if (a.rank > 0 &&
@@ -850,14 +886,14 @@ cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L) {
   const size_t smem = d.L.total;
   if (a.block == 256)
     e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<256, 1>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, mv, p)
+                             mq4, ms4, mq8, mv, mq4q, ms4q, p)
                   : L.launch("dec_main", dec_main_kernel<256, 2>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, mv, p);
+                             mq4, ms4, mq8, mv, mq4q, ms4q, p);
   else
     e = d.NT == 1 ? L.launch("dec_main", dec_main_kernel<128, 1>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, mv, p)
+                             mq4, ms4, mq8, mv, mq4q, ms4q, p)
                   : L.launch("dec_main", dec_main_kernel<128, 2>, grid, block, smem, st, true,
-                             mq4, ms4, mq8, mv, p);
+                             mq4, ms4, mq8, mv, mq4q, ms4q, p);
   if (e != cudaSuccess) return e;
   return L.launch("dec_tail", dec_tail_kernel, dim3((a.M + kTailThreads / 4 - 1) / (kTailThreads / 4), a.T),
                   dim3(kTailThreads), 0, st, true, p);

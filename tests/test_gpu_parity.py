@@ -153,8 +153,10 @@ def test_encode_zero_rows_and_wide_exponent_spread(dv):
 # ---------------------------------------------------------------- forward ---
 
 @pytest.mark.parametrize("name,T", [("tiny", 4), ("tiny", 1), ("spark_down", 1),
-                                    ("spark_down", 16), ("minicpm_k", 1), ("minicpm_k", 8),
-                                    ("minicpm_up", 8), ("minicpm_up", 16)])
+                                    ("spark_down", 2), ("spark_down", 16), ("minicpm_k", 1),
+                                    ("minicpm_k", 8), ("minicpm_up", 1), ("minicpm_up", 2),
+                                    ("minicpm_up", 8), ("minicpm_up", 16),
+                                    ("spark_up_prefill", 1), ("spark_up_prefill", 16)])
 def test_forward_decode_parity(dv, name, T):
     L = layer(dv, name)
     x = L.wl.activations(T)
