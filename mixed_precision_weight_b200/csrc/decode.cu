@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
   __half *xq = reinterpret_cast<__half *>(base + p.L.xq);     // [ns][NTOK][kXRow]
   __half *xs = reinterpret_cast<__half *>(base + p.L.xs);     // [ns][NTOK][kXsRow]
   float *corr = reinterpret_cast<float *>(base + p.L.corr);   // [ns][4][NTOK]
-  float *c8 = reinterpret_cast<float *>(base + p.L.c8);       // [ns][NTOK]
+  float *c8 = reinterpret_cast<float *>(base + p.L.c8);       // [ns][NBLK][NTOK]
   float *s8s = reinterpret_cast<float *>(base + p.L.s8);      // [upc][16]
   int16_t *colpos = reinterpret_cast<int16_t *>(base + p.L.colpos);   // [ns][256]
   int *samp = reinterpret_cast<int *>(base + p.L.samp);       // [kSamples]
@@ -399,28 +399,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
         dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
         dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
         if ((t & 3) == 0) corr[(si * 4 + cs / 64) * NTOK + tok] = cp;
+      }
+      // salient bias term of the block: 1152 x the sum of its salient x, as
+      // stored in FP16 (the group's threads are adjacent lanes)
+      float sal = 0.0f;
+      if (live) {
         const int16_t *cpos = colpos + si * kSlab + cs;
         __half *xrow = xs + (size_t)(si * NTOK + tok) * kXsRow;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int pos = cpos[j];
-          if (pos >= 0) xrow[pos] = __float2half_rn(v[j]);
+          if (pos >= 0) {
+            const __half hv = __float2half_rn(v[j]);
+            xrow[pos] = hv;
+            sal += __half2float(hv);
+          }
         }
       }
+#pragma unroll
+      for (int o = 1; o < P; o <<= 1) sal += __shfl_xor_sync(0xffffffffu, sal, o);
+      if (live && t == 0) c8[(si * NBLK + blk) * NTOK + tok] = 1152.0f * sal;
     }
   }
   dec_consumer_sync();
-
-  // salient bias terms: c8[si][tok] = 1152 * sum of the slab's salient x
-  for (int q = cw; q < ns * p.T; q += kDecCons) {
-    const int si = q / p.T, tok = q % p.T;
-    const __half *xrow = xs + (size_t)(si * NTOK + tok) * kXsRow;
-    float sum = 0.0f;
-    for (int i = lane; i < 16 * nch[si]; i += 32) sum += __half2float(xrow[i]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) c8[si * NTOK + tok] = 1152.0f * sum;
-  }
 
   // t share of each owned slab: tpart[s][rr][tok] = sum_j V[rr][j] x_rot[j],
   // on the tensor cores against the FP16 x_rot already in shared memory:
@@ -572,7 +573,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_main_kernel(
       float d8[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const float2 cc = *reinterpret_cast<const float2 *>(c8 + si * NTOK + 8 * nt + 2 * tig);
+        float2 cc = *reinterpret_cast<const float2 *>(c8 + si * NBLK * NTOK + 8 * nt + 2 * tig);
+        if constexpr (NBLK == 2) {
+          const float2 c2 = *reinterpret_cast<const float2 *>(c8 + (si * NBLK + 1) * NTOK + 8 * nt + 2 * tig);
+          cc.x += c2.x;
+          cc.y += c2.y;
+        }
         d8[nt][0] = -cc.x; d8[nt][1] = -cc.y; d8[nt][2] = -cc.x; d8[nt][3] = -cc.y;
       }
       const int mlo = tile * kUnitRows + g;
@@ -783,7 +789,7 @@ DecPlan dec_plan(int M, int K, int block, int T, int rank, int nsm) {
   L.xq = off;     off += al(d.ns_max * d.ntok * kXRow * 2, 128);
   L.xs = off;     off += al(d.ns_max * d.ntok * kXsRow * 2, 128);
   L.corr = off;   off += al(d.ns_max * 4 * d.ntok * 4, 128);
-  L.c8 = off;     off += al(d.ns_max * d.ntok * 4, 128);
+  L.c8 = off;     off += al(d.ns_max * 2 * d.ntok * 4, 128);
   L.s8 = off;     off += al(d.upc_max * kUnitRows * 4, 128);
   L.colpos = off; off += al(d.ns_max * kSlab * 2, 128);
   L.samp = off;   off += kSamples * 4;
