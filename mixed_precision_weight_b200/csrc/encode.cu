@@ -323,6 +323,10 @@ __global__ void __launch_bounds__(kSelThreads) enc_select_kernel(
   __shared__ unsigned int s_krem, s_whole;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool in_smem = K <= kSelSmemKeys;
+  // launched with programmatic dependent launch: the scores come from pass 1;
+  // pass 2 may start its salient-independent prologue now
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (n_sal == 0) {
     for (int w = tid; w < (K + 31) / 32; w += kSelThreads) sal_prefix[w] = 0;
@@ -584,6 +588,7 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
   for (int s = 0; s < kP2Stages - 1; ++s) issue(src_of(cur, s), s);
 
   unsigned long long unsafe = 0;
+  bool sal_ready = false;   // the salient set (from the select kernel) is visible
   int pos = 0;    // ring position of the row-block in hand
   int k = 0;      // tiles done by this CTA: parity of the next-tile slots
   while (cur < ntiles) {
@@ -613,12 +618,21 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
       for (int m = 0; m < 8; ++m) stg[m ^ (t & 7)] = make_double2(v[2 * m], v[2 * m + 1]);
       __syncwarp();
       // this block's salient columns: to the stash, then zero in the staged row
-      const int e0 = __ldg(p.sal_prefix + ((kb * B) >> 5));
-      const int e1 = (kb + 1) * B < K ? __ldg(p.sal_prefix + (((kb + 1) * B) >> 5)) : n_sal;
+      // everything above (tile claims, the W ring, the rotation) is
+      // independent of the salient set and overlaps the select kernel.  The
+      // salient set is read with plain loads (cached in L1: the rows of a
+      // column block reuse it): a read-only-cache load counts as invariant
+      // over the kernel and may be hoisted above the wait.
+      if (!sal_ready) {
+        pdl_wait();
+        sal_ready = true;
+      }
+      const int e0 = p.sal_prefix[(kb * B) >> 5];
+      const int e1 = (kb + 1) * B < K ? p.sal_prefix[((kb + 1) * B) >> 5] : n_sal;
       if (valid && e0 < e1) {
         double *dst = stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal;
         for (int e = e0 + t; e < e1; e += P) {
-          const int col = __ldg(p.sal_idx + e) - kb * B;
+          const int col = p.sal_idx[e] - kb * B;
           const int si = stage_pos(col);
           dst[e] = sgrp[si];
           sgrp[si] = 0.0;
@@ -804,7 +818,7 @@ cudaError_t launch_pass2(const Pass2Params &pp, size_t smem, cudaStream_t st, La
     return e;
   const long long grid = std::max(1LL, std::min<long long>(pp.ntiles, (long long)nsm * occ));
   return L.launch("enc_pass2", enc_pass2_kernel<B, RESID>, dim3((unsigned)grid), dim3(128), smem,
-                  st, false, pp);
+                  st, true, pp);
 }
 }  // namespace
 
@@ -840,7 +854,7 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
                  (const uint16_t *)a.W, M, K, c, a.act_scale, gpart, score, done, info);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = K <= kSelSmemKeys ? (size_t)K * sizeof(unsigned long long) : 0;
-  e = L.launch("enc_select", enc_select_kernel, dim3(1), dim3(kSelThreads), sel_smem, st, false,
+  e = L.launch("enc_select", enc_select_kernel, dim3(1), dim3(kSelThreads), sel_smem, st, true,
                (const double *)score, K, a.n_sal, a.sal_idx, pref);
   if (e != cudaSuccess) return e;
 
