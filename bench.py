@@ -627,6 +627,24 @@ def run_oracle(work, O, synth, budget_s=20.0, min_steps=1, max_steps=10):
     return n, dt
 
 
+def max_over_ranks(x, world, device):
+    """The largest value of x over the ranks (the job's time is its slowest
+    rank's).  Every rank must call it, in the same order."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, ms_step, scale):
+    """Whole-job throughput: every rank processes units_per_rank_step per
+    step (weak scaling), and a step takes ms_step on the slowest rank."""
+    return world * units_per_rank_step / (ms_step * 1e-3) / scale
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -707,19 +725,15 @@ def main():
             timed_step(i)
         stop.record(stream)
         barrier()
-    ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(stop), world, device)
     err = dv.dvssq_device_error(clear=True)
     ms_step = ms / args.steps
     if unit == "TFLOP/s":
         bytes_step = None
-        value = world * work.work_per_step() / (ms_step * 1e-3) / 1e12
+        value = job_throughput(world, work.work_per_step(), ms_step, 1e12)
     else:
         bytes_step = work.bytes_per_step()
-        value = world * bytes_step / (ms_step * 1e-3) / 1e9
+        value = job_throughput(world, bytes_step, ms_step, 1e9)
 
     # per-kernel device times: the same K steps again with events around each launch
     dv.dvssq_profile_reset()
@@ -786,13 +800,9 @@ def main():
             work.e2e_step()
         e_stop.record(stream)
         barrier()
-        ems = e_start.elapsed_time(e_stop) / n_e2e
-        if world > 1:
-            t = torch.tensor([ems], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e_start.elapsed_time(e_stop) / n_e2e, world, device)
         h2d, d2h = work.e2e_bytes()
-        e2e = {"value": round(world * bytes_step / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e = {"value": round(job_throughput(world, bytes_step, ems, 1e9), 2), "unit": "GB/s",
                "ms_per_step": round(ems, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
