@@ -71,7 +71,8 @@ typedef enum {
  *   group  INT4 group size: must be 64
  *   n_sal  number of salient (INT8) columns: 0 <= n_sal <= K, n_sal % 16 == 0;
  *          the method uses n_sal = K / 8 (top 12.5 %)
- *   rank   rank r of the residual factors: 0 <= r <= 64                    */
+ *   rank   rank r of the residual factors: 0 <= r <= 64, r % 8 == 0 (the
+ *          rows of U travel as 16-byte vectors)                          */
 typedef struct {
   int32_t M;
   int32_t K;

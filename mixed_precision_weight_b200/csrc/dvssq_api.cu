@@ -52,7 +52,8 @@ dvssq_status check_shape(const dvssq_shape *s) {
   if (s->K % s->block != 0) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
   if (s->n_sal > s->K || s->n_sal % 16 != 0 || s->n_sal > kMaxSalient)
     return DVSSQ_ERR_UNSUPPORTED_SHAPE;
-  if (s->rank > 64) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  // U rows travel as 16-byte vectors of 8 BF16 values
+  if (s->rank > 64 || s->rank % 8 != 0) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
   return DVSSQ_OK;
 }
 

@@ -65,7 +65,7 @@ def test_workspace_sizes(dv):
 @pytest.mark.parametrize("kw,status", [
     (dict(block=64), 2), (dict(group=32), 2), (dict(K=500), 2), (dict(K=384, block=256), 2),
     (dict(n_sal=65), 2), (dict(n_sal=1024), 2), (dict(rank=65), 2), (dict(M=0), 2),
-    (dict(rank=-1), 2), (dict(K=131072), 2),
+    (dict(rank=-1), 2), (dict(rank=12), 2), (dict(K=131072), 2),
 ])
 def test_bad_shapes_rejected(dv, kw, status):
     n = ctypes.c_size_t(0)
