@@ -534,7 +534,7 @@ __device__ __forceinline__ uint32_t pack_nibbles8(const uint32_t *l) {
 }
 
 template <int B, bool RESID>
-__global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) {
+__global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) {
   constexpr int P = B / 16;
   constexpr int GPW = 32 / P;
   constexpr int NG = GPW * 4;
@@ -587,6 +587,11 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
 #pragma unroll
   for (int s = 0; s < kP2Stages - 1; ++s) issue(src_of(cur, s), s);
 
+  // Salient tables, built once per CTA (a CTA's groups meet the same column
+  // blocks in every tile): each block's first entry in sal_idx (and n_sal
+  // at the end) and each entry's position in the staged row.
+  int16_t *tab_pos = reinterpret_cast<int16_t *>(stash_s + (p.stash_smem ? (size_t)R * n_sal : 0));
+  int *tab_pref = reinterpret_cast<int *>(tab_pos + ((n_sal + 3) & ~3));
   unsigned long long unsafe = 0;
   bool sal_ready = false;   // the salient set (from the select kernel) is visible
   int pos = 0;    // ring position of the row-block in hand
@@ -625,15 +630,20 @@ __global__ void __launch_bounds__(128, 4) enc_pass2_kernel(const Pass2Params p) 
       // over the kernel and may be hoisted above the wait.
       if (!sal_ready) {
         pdl_wait();
+        // every thread of the CTA is here, in its first row-block
+        for (int e = tid; e < n_sal; e += blockDim.x)
+          tab_pos[e] = (int16_t)stage_pos(p.sal_idx[e] & (B - 1));
+        const int nkb = K / B;
+        for (int k = tid; k <= nkb; k += blockDim.x)
+          tab_pref[k] = k < nkb ? p.sal_prefix[(k * B) >> 5] : n_sal;
+        __syncthreads();
         sal_ready = true;
       }
-      const int e0 = p.sal_prefix[(kb * B) >> 5];
-      const int e1 = (kb + 1) * B < K ? p.sal_prefix[((kb + 1) * B) >> 5] : n_sal;
+      const int e0 = tab_pref[kb], e1 = tab_pref[kb + 1];
       if (valid && e0 < e1) {
         double *dst = stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal;
         for (int e = e0 + t; e < e1; e += P) {
-          const int col = p.sal_idx[e] - kb * B;
-          const int si = stage_pos(col);
+          const int si = tab_pos[e];
           dst[e] = sgrp[si];
           sgrp[si] = 0.0;
         }
@@ -758,6 +768,11 @@ struct Pass2Plan {
   bool smem;
   size_t smem_bytes;
 };
+// shared memory of pass 2's salient tables: n_sal positions, nkb + 1 block starts
+size_t sal_tab_bytes(int n_sal, int nkb) {
+  return (size_t)((n_sal + 3) & ~3) * sizeof(int16_t) + (size_t)(nkb + 1) * sizeof(int);
+}
+constexpr size_t kSalTabMax = (size_t)kMaxSalient * 2 + (65536 / 128 + 1) * 4;
 
 // Rows per tile: the smallest power of two that splits the tile's R * nkb
 // row-blocks evenly over the groups with at least kP2Stages - 1 per group.
@@ -774,6 +789,7 @@ Pass2Plan pass2_plan(int M, int K, int B, int n_sal) {
   const size_t bytes = (size_t)R * n_sal * sizeof(double);
   pl.smem = bytes <= (size_t)kStashSmemMax;
   pl.smem_bytes = pl.smem ? bytes : 0;
+  pl.smem_bytes += sal_tab_bytes(n_sal, nkb);
   return pl;
 }
 
@@ -901,7 +917,7 @@ cudaError_t prepare_encode_kernels() {
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kStashSmemMax)) != cudaSuccess)
+                                  (int)(kStashSmemMax + kSalTabMax))) != cudaSuccess)
       return e;
   }
   double recip[128];
