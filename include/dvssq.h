@@ -107,7 +107,8 @@ typedef struct {
 typedef struct {
   /* row-blocks whose +-1 Hadamard sums are not provably exact in fp64
      (BF16 exponent spread above 45 - log2(b) bits); codes of such blocks
-     may differ from an exact-arithmetic encoder in the last rounding     */
+     may differ from an exact-arithmetic encoder in the last rounding.  The
+     test runs only in calls that ask for this struct.                    */
   int64_t inexact_rotation_blocks;
   /* INT4 groups with a nonzero scale outside [2^-17, 8188] and rows with a
      nonzero INT8 scale outside [2^-17, 511]: the prefill path stages q*s

@@ -102,7 +102,9 @@ __device__ __forceinline__ bool spread_exceeds(int emax, int emin1, int lg) {
 // CTA then forms the 8-chunk group sums (ascending chunks, from 0.0) in shared
 // memory, and the CTA that finishes a column block last adds that block's
 // group sums in ascending order and writes the scores.
-template <int B>
+// STATS: also the exact-sum test behind info.inexact_rotation_blocks (only
+// when the caller asks for the diagnostics; the codes do not depend on it)
+template <int B, bool STATS>
 __global__ void __launch_bounds__(128) enc_pass1_kernel(
     const uint16_t *__restrict__ W, int M, int K, double c, const float *__restrict__ act_scale,
     double *__restrict__ gpart, double *__restrict__ score, unsigned int *__restrict__ done,
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(
     cp_async_wait<kStages - 1>();
     __syncwarp();
     const uint16_t *buf = ring[g][i % kStages];
-    if (i < nrows) {
+    if (STATS && i < nrows) {
       // this thread's 32 contiguous bytes of the row-block, for the exact-sum test
       const uint4 *wq = reinterpret_cast<const uint4 *>(buf) + 2 * t;
       const uint4 a = wq[0], b = wq[1];
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(
   // Exact-sum test, first over the whole chunk: the chunk's spread bounds the
   // spread of each of its row-blocks.  Only a chunk that fails it is checked
   // row by row (from global memory).
-  {
+  if (STATS) {
     const uint32_t mxh = max(mx & 0xFFFFu, mx >> 16), mnh = min(mn & 0xFFFFu, mn >> 16);
     const int emax = (int)(mxh >> 7);
     const int emin1 = mnh == 0xFFFFu ? 0xFFFF : max((int)((mnh + 1u) >> 7), 1);
@@ -862,12 +864,11 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
   const int nkb = K / B;
   const int NG = groups_per_cta(B);
   dim3 g1((unsigned)(((nchunk + NG - 1) / NG) * nkb));
-  if (B == 256)
-    e = L.launch("enc_pass1", enc_pass1_kernel<256>, g1, dim3(128), 0, st, false,
-                 (const uint16_t *)a.W, M, K, c, a.act_scale, gpart, score, done, info);
-  else
-    e = L.launch("enc_pass1", enc_pass1_kernel<128>, g1, dim3(128), 0, st, false,
-                 (const uint16_t *)a.W, M, K, c, a.act_scale, gpart, score, done, info);
+  const bool stats = a.info_host != nullptr;
+  auto p1 = B == 256 ? (stats ? enc_pass1_kernel<256, true> : enc_pass1_kernel<256, false>)
+                     : (stats ? enc_pass1_kernel<128, true> : enc_pass1_kernel<128, false>);
+  e = L.launch("enc_pass1", p1, g1, dim3(128), 0, st, false, (const uint16_t *)a.W, M, K, c,
+               a.act_scale, gpart, score, done, info);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = K <= kSelSmemKeys ? (size_t)K * sizeof(unsigned long long) : 0;
   e = L.launch("enc_select", enc_select_kernel, dim3(1), dim3(kSelThreads), sel_smem, st, true,
@@ -906,7 +907,8 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
 cudaError_t prepare_encode_kernels() {
   cudaError_t e;
   for (const void *f :
-       {(const void *)enc_pass1_kernel<256>, (const void *)enc_pass1_kernel<128>})
+       {(const void *)enc_pass1_kernel<256, true>, (const void *)enc_pass1_kernel<128, true>,
+        (const void *)enc_pass1_kernel<256, false>, (const void *)enc_pass1_kernel<128, false>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
