@@ -547,7 +547,9 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
   constexpr int PIECES = B * 2 / 16;
   __shared__ __align__(16) double scratch[NG][SCR];
   __shared__ __align__(16) uint16_t ring[NG][kP2Stages][B];
-  __shared__ unsigned long long s_rmax[kTileRowsMax];
+  // |w| maxima of the salient values per tile row (fp64 bit patterns,
+  // ordered as unsigned integers), double-buffered by tile parity
+  __shared__ unsigned long long s_rmax2[2][kTileRowsMax];
   __shared__ int s_tile[4];
   extern __shared__ __align__(16) double stash_s[];
 
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
     s_tile[0] = (int)atomicAdd(p.tile_ctr, 1u);
     s_tile[1] = (int)atomicAdd(p.tile_ctr, 1u);
   }
-  for (int i = tid; i < kTileRowsMax; i += blockDim.x) s_rmax[i] = 0ull;
+  for (int i = tid; i < 2 * kTileRowsMax; i += blockDim.x) s_rmax2[i >> 6][i & 63] = 0ull;
   __syncthreads();
   int cur = s_tile[0], nxt = s_tile[1];
 
@@ -642,14 +644,21 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
         sal_ready = true;
       }
       const int e0 = tab_pref[kb], e1 = tab_pref[kb + 1];
+      double lm = 0.0;                    // this thread's share of the row's salient |w| max
       if (valid && e0 < e1) {
         double *dst = stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal;
         for (int e = e0 + t; e < e1; e += P) {
           const int si = tab_pos[e];
-          dst[e] = sgrp[si];
+          const double w = sgrp[si];
+          dst[e] = w;
+          lm = fmax(lm, fabs(w));
           sgrp[si] = 0.0;
         }
       }
+#pragma unroll
+      for (int o = 1; o < P; o <<= 1) lm = fmax(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+      if (t == 0 && lm > 0.0)
+        atomicMax(&s_rmax2[k & 1][r], (unsigned long long)__double_as_longlong(lm));
       __syncwarp();
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -706,24 +715,10 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
     }
 
     // INT8 tier of the tile's rows: s8 = bf16_rn(max|w| / 127), q8 = clip(rint(w / s8))
-    __syncthreads();                      // the tile's stash is complete
+    __syncthreads();                      // the tile's stash and row maxima are complete
     const int n8 = n_sal >> 3;
     const double vscale = kPow2 ? c : 1.0;
-    for (int ch = tid; ch < (n8 << rshift); ch += blockDim.x) {
-      const int r = ch / n8, e = (ch - r * n8) * 8;
-      const int row = (cur << rshift) + r;
-      if (row >= M) continue;
-      const double2 *src = reinterpret_cast<const double2 *>(
-          (stash != nullptr ? stash + (size_t)r * n_sal : p.sv + (size_t)row * n_sal) + e);
-      double m = 0.0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const double2 d = src[u];
-        m = fmax(m, fmax(fabs(d.x), fabs(d.y)));
-      }
-      atomicMax(&s_rmax[r], (unsigned long long)__double_as_longlong(m));
-    }
-    __syncthreads();                      // row maxima complete
+    unsigned long long *s_rmax = s_rmax2[k & 1];
     for (int ch = tid; ch < (n8 << rshift); ch += blockDim.x) {
       const int r = ch / n8, e = (ch - r * n8) * 8;
       const int row = (cur << rshift) + r;
@@ -735,11 +730,20 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
       const double s8v = bf16_bits_to_f64(sb);
       const double vinv = s8v > 0.0 ? recip_bf16(sb) * vscale : 0.0;
       uint32_t pk[2] = {0u, 0u};
+      // w vinv is either NaN (a non-finite weight; it codes to -128, as
+      // rint's integer conversion gives) or at most 127.5 in magnitude: rint
+      // is then the add of 1.5 * 2^52 (exact round-half-even, the integer in
+      // the low word)
+      auto q8_of = [&](double w) {
+        const double x = __dmul_rn(w, vinv);
+        const int q = __double2loint(__dadd_rn(x, 0x1.8p52));
+        return x != x ? -128 : min(127, max(-128, q));
+      };
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const double2 d = src[u];
-        const int qa = min(127, max(-128, __double2int_rn(__dmul_rn(d.x, vinv))));
-        const int qb = min(127, max(-128, __double2int_rn(__dmul_rn(d.y, vinv))));
+        const int qa = q8_of(d.x);
+        const int qb = q8_of(d.y);
         pk[u >> 1] |= (((uint32_t)qa & 0xFFu) | (((uint32_t)qb & 0xFFu) << 8)) << (16 * (u & 1));
       }
       *reinterpret_cast<uint2 *>(p.q8 + (size_t)row * n_sal + e) = make_uint2(pk[0], pk[1]);
@@ -751,7 +755,8 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
     if (n8 == 0)
       for (int r = tid; r < R; r += blockDim.x)
         if ((cur << rshift) + r < M) p.s8[(cur << rshift) + r] = 0;
-    __syncthreads();                      // stash and row maxima free for the next tile
+    __syncthreads();                      // the stash is free for the next tile
+    // this buffer serves tile k + 2, whose stash starts after tile k + 1's barriers
     if (tid < R) s_rmax[tid] = 0ull;
     cur = nxt;
     nxt = s_tile[2 + (k & 1)];
