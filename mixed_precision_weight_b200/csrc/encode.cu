@@ -105,7 +105,7 @@ __device__ __forceinline__ bool spread_exceeds(int emax, int emin1, int lg) {
 // STATS: also the exact-sum test behind info.inexact_rotation_blocks (only
 // when the caller asks for the diagnostics; the codes do not depend on it)
 template <int B, bool STATS>
-__global__ void __launch_bounds__(128) enc_pass1_kernel(
+__global__ void __launch_bounds__(128, 6) enc_pass1_kernel(
     const uint16_t *__restrict__ W, int M, int K, double c, const float *__restrict__ act_scale,
     double *__restrict__ gpart, double *__restrict__ score, unsigned int *__restrict__ done,
     unsigned long long *__restrict__ info) {
@@ -249,21 +249,37 @@ __global__ void __launch_bounds__(128) enc_pass1_kernel(
   if (!s_last) return;
   __threadfence();
   unsigned long long bad = 0;
-  for (int col = threadIdx.x; col < B; col += blockDim.x) {
-    const int j = kb * B + col;
-    double tot = 0.0;
-    for (int sg0 = 0; sg0 < nsg; sg0 += 16) {
-      double gv[16];          // loads in flight together, adds in ascending order
+  // CPT columns per thread, their loads in flight together (10 group sums
+  // of each column per batch, within pass 1's register budget); each
+  // column's adds stay in ascending order
+  constexpr int CPT = B / 128;
+  static_assert(CPT * 128 == B, "pass 1 runs 128 threads");
+  const float *as = act_scale + (size_t)kb * B + threadIdx.x;
+  float a[CPT];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        gv[u] = sg0 + u < nsg ? __ldcg(gpart + (size_t)(sg0 + u) * K + j) : 0.0;
+  for (int c2 = 0; c2 < CPT; ++c2) a[c2] = as[128 * c2];
+  double tot[CPT];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        if (sg0 + u < nsg) tot = __dadd_rn(tot, gv[u]);
-    }
-    const double s = __dmul_rn((double)act_scale[j], __dsqrt_rn(tot));
+  for (int c2 = 0; c2 < CPT; ++c2) tot[c2] = 0.0;
+  const double *gp = gpart + (size_t)kb * B + threadIdx.x;
+  for (int sg0 = 0; sg0 < nsg; sg0 += 10) {
+    double gv[CPT][10];
+#pragma unroll
+    for (int c2 = 0; c2 < CPT; ++c2)
+#pragma unroll
+      for (int u = 0; u < 10; ++u)
+        gv[c2][u] = sg0 + u < nsg ? __ldcg(gp + (size_t)(sg0 + u) * K + 128 * c2) : 0.0;
+#pragma unroll
+    for (int c2 = 0; c2 < CPT; ++c2)
+#pragma unroll
+      for (int u = 0; u < 10; ++u)
+        if (sg0 + u < nsg) tot[c2] = __dadd_rn(tot[c2], gv[c2][u]);
+  }
+#pragma unroll
+  for (int c2 = 0; c2 < CPT; ++c2) {
+    const double s = __dmul_rn((double)a[c2], __dsqrt_rn(tot[c2]));
     bad += !isfinite(s);
-    score[j] = s;
+    score[(size_t)kb * B + threadIdx.x + 128 * c2] = s;
   }
   if (bad) atomicAdd(&info[2], bad);
 }
