@@ -127,27 +127,11 @@ __host__ __device__ inline int t_owner_unit(int s, const RowGeom &G) {
   return first + i;
 }
 
-// A q4 segment (the slabs of one tile in one column group) that lies wholly
-// in the CTA's range travels as one 3-D box when its group size has a map
-// (seg3d); all its units then wait on the barrier of its first unit.
-// Returns that unit's index within the CTA, or -1 for a unit staged on its own.
-__device__ __forceinline__ int seg_lead(const RowUnit &ru, int k, int u0, int u1,
-                                        const RowGeom &G, int seg3d) {
-  if (ru.q8) return -1;
-  const int Sg = ru.g < G.ng - 1 ? G.S : G.Slast;
-  if (!(seg3d & (Sg == G.S ? 1 : 2))) return -1;
-  const int jj = ru.j - ru.g * G.S;
-  const int uf = u0 + k - jj;
-  return (uf >= u0 && uf + Sg <= u1) ? k - jj : -1;
-}
-
 struct RowParams {
   int M, K, T, n_sal, rank, block;
   RowGeom G;
   int units, grid, upc_max, maxq8, nscr;
   int s4_tma;
-  int seg3d;        // bit 0: segments of S slabs travel as one 3-D box (q4) and
-                    // one s4 box; bit 1: so do those of the last group (Slast)
   int QW;           // salient entries per q8 unit: 128, or n_sal when smaller
   float c;
   const uint16_t *s4;
@@ -175,9 +159,7 @@ template <int B, int T>
 __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
     const __grid_constant__ CUtensorMap mq4, const __grid_constant__ CUtensorMap ms4,
     const __grid_constant__ CUtensorMap mq8, const __grid_constant__ CUtensorMap ms8,
-    const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mq4s,
-    const __grid_constant__ CUtensorMap ms4s, const __grid_constant__ CUtensorMap mq4l,
-    const __grid_constant__ CUtensorMap ms4l, RowParams p) {
+    const __grid_constant__ CUtensorMap mv, RowParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t *us = base + p.L.units;                                        // [upc][2048]
@@ -262,21 +244,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
         const RowUnit ru = row_unit(u, G);
         if (ru.q8 != (pass == 0)) continue;
         if (!ru.q8) {
-          const int lead = seg_lead(ru, k, u0, u1, G, p.seg3d);
-          if (lead == k) {
-            // the whole segment: Sg units laid out as Sg consecutive 2 KB
-            // units (slab-major), and its 4 Sg scales per row
-            const bool last = ru.g == G.ng - 1 && G.Slast != G.S;
-            const int Sg = last ? G.Slast : G.S;
-            mbar_arrive_expect_tx(&bars[k], (uint32_t)(Sg * (kRowUnit + 128)));
-            tma_load_3d(us + k * kRowUnit, last ? &mq4l : &mq4s, 0, ru.t * 16, ru.g * G.S, &bars[k]);
-            tma_load_2d(s4s + k * 128, last ? &ms4l : &ms4s, 4 * G.S * ru.g, ru.t * 16, &bars[k]);
-          } else if (lead < 0) {
-            mbar_arrive_expect_tx(&bars[k], kRowUnit + (p.s4_tma ? 256 : 0));
-            tma_load_2d(us + k * kRowUnit, &mq4, ru.j * 128, ru.t * 16, &bars[k]);
-            if (p.s4_tma)
-              tma_load_2d(s4s + k * 128, &ms4, 8 * (ru.j >> 1), ru.t * 16, &bars[k]);
-          }
+          mbar_arrive_expect_tx(&bars[k], kRowUnit + (p.s4_tma ? 256 : 0));
+          tma_load_2d(us + k * kRowUnit, &mq4, ru.j * 128, ru.t * 16, &bars[k]);
+          if (p.s4_tma)
+            tma_load_2d(s4s + k * 128, &ms4, 8 * (ru.j >> 1), ru.t * 16, &bars[k]);
         } else {
           const int slot = u - q8first;
           mbar_arrive_expect_tx(&bars[k], 16 * p.QW + 32);
@@ -521,16 +492,11 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
       ++slot_i;
       scur = ru.key - key0;
     }
-    const int lead = seg_lead(ru, k, u0, u1, G, p.seg3d);
-    if (!mbar_wait(&bars[lead >= 0 ? lead : k], 0)) { ok = false; break; }
+    if (!mbar_wait(&bars[k], 0)) { ok = false; break; }
     const uint8_t *row = us + k * kRowUnit + r * 128;
     if (!ru.q8) {
       const int j = ru.j;
-      // scales: [16][8] per unit (two slabs), or [16][4 Sg] per segment
-      const int Sg = ru.g < G.ng - 1 ? G.S : G.Slast;
-      const uint16_t *sb =
-          lead >= 0 ? s4s + lead * 128 + r * (4 * Sg) + 4 * (j - ru.g * G.S) + 2 * h
-                    : s4s + k * 128 + r * 8 + 4 * (j & 1) + 2 * h;
+      const uint16_t *sb = s4s + k * 128 + r * 8 + 4 * (j & 1) + 2 * h;
 #pragma unroll
       for (int gi = 0; gi < 2; ++gi) {
         const int gcol = 4 * j + 2 * h + gi;
@@ -768,29 +734,6 @@ cudaError_t launch_decode_row(const ForwardArgs &a, cudaStream_t st, Launcher &L
                      p.QW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE) !=
           CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // q4 as [slab][row][128 B] (strides 128 B and K/2 B): one box of Sg slabs
-  // x 16 rows lands as Sg consecutive swizzled units; s4 of the same
-  // segment.  A pair of maps for groups of S slabs and one for the last
-  // group when it is narrower; only for even sizes (the s4 box starts at
-  // scale 4 S g, on 16 bytes).  A map the driver rejects leaves those units
-  // on their own boxes.
-  CUtensorMap mq4s = mq4, ms4s = mq4, mq4l = mq4, ms4l = mq4;
-  p.seg3d = 0;
-  auto seg_maps = [&](int Sg, CUtensorMap *mq, CUtensorMap *ms) {
-    if (!p.s4_tma || Sg % 2 != 0 || a.K % 256 != 0) return false;
-    const uint64_t dims[3] = {128, (uint64_t)a.M, (uint64_t)d.G.nslab};
-    const uint64_t strides[2] = {(uint64_t)a.K / 2, 128};
-    const uint32_t box[3] = {128, 16, (uint32_t)Sg};
-    return encode_tmap_3d(mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q4, dims, strides, box,
-                          CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS &&
-           encode_tmap_2d(ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.s4, (uint64_t)a.K / 64,
-                          (uint64_t)a.M, (uint64_t)a.K / 32, 4 * (uint32_t)Sg, 16,
-                          CU_TENSOR_MAP_SWIZZLE_NONE) == CUDA_SUCCESS;
-  };
-  if (seg_maps(d.G.S, &mq4s, &ms4s)) p.seg3d |= 1;
-  // (the last group's scales start at 4 S (ng - 1): on 16 bytes when S (ng - 1) is even)
-  if (d.G.Slast != d.G.S && d.G.S * (d.G.ng - 1) % 2 == 0 && seg_maps(d.G.Slast, &mq4l, &ms4l))
-    p.seg3d |= 2;
   // V [rank][K] BF16, one slab (256 columns x rank rows) per box
   CUtensorMap mv = mq4;
   if (a.rank > 0 &&
@@ -803,11 +746,11 @@ cudaError_t launch_decode_row(const ForwardArgs &a, cudaStream_t st, Launcher &L
   const size_t smem = d.L.total;
   cudaError_t e;
   if (a.block == 256)
-    e = a.T == 1 ? Lc.launch("dec_row", dec_row_kernel<256, 1>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, mq4s, ms4s, mq4l, ms4l, p)
-                 : Lc.launch("dec_row", dec_row_kernel<256, 2>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, mq4s, ms4s, mq4l, ms4l, p);
+    e = a.T == 1 ? Lc.launch("dec_row", dec_row_kernel<256, 1>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, p)
+                 : Lc.launch("dec_row", dec_row_kernel<256, 2>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, p);
   else
-    e = a.T == 1 ? Lc.launch("dec_row", dec_row_kernel<128, 1>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, mq4s, ms4s, mq4l, ms4l, p)
-                 : Lc.launch("dec_row", dec_row_kernel<128, 2>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, mq4s, ms4s, mq4l, ms4l, p);
+    e = a.T == 1 ? Lc.launch("dec_row", dec_row_kernel<128, 1>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, p)
+                 : Lc.launch("dec_row", dec_row_kernel<128, 2>, grid, block, smem, st, true, mq4, ms4, mq8, ms8, mv, p);
   if (e != cudaSuccess) return e;
 
   DecodeParams tp{};

@@ -122,19 +122,6 @@ CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-CUresult encode_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
-                        const uint64_t dims[3], const uint64_t strides_bytes[2],
-                        const uint32_t box[3], CUtensorMapSwizzle swz) {
-  EncodeTiledFn fn = tiled_encoder();
-  if (fn == nullptr) return CUDA_ERROR_NOT_FOUND;
-  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
-  cuuint32_t b[3] = {box[0], box[1], box[2]};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, dtype, 3, const_cast<void *>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-}
-
 cudaError_t prepare_decode_kernels();
 cudaError_t prepare_prefill_kernels();
 

@@ -185,10 +185,5 @@ cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L);
 CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                         uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
-// Three dimensions with free strides (bytes) for dimensions 1 and 2, which
-// need not grow with the dimension: a box may walk a tensor in any order.
-CUresult encode_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
-                        const uint64_t dims[3], const uint64_t strides_bytes[2],
-                        const uint32_t box[3], CUtensorMapSwizzle swz);
 
 }  // namespace dvssq
