@@ -838,7 +838,14 @@ def run_reference(args, world, rank):
     from mixed_precision_weight_b200 import synth
     from oracle import dvssq_oracle as O
 
-    class _W(SparkDownStep):
+    base = WORKLOADS.get(args.workload)
+    if base not in (SparkDownStep, DecodeStep):
+        print(json.dumps({"impl": "reference", "unavailable":
+                          f"the oracle arm times the spark_down and decode workloads; "
+                          f"{args.workload} has no host step of its own"}))
+        return
+
+    class _W(base):
         def __init__(self):
             wl = synth.WORKLOADS["spark_down"]
             self.wl = wl
@@ -857,7 +864,7 @@ def run_reference(args, world, rank):
             "n_gpus": world, "steps": nst, "warmup": min(args.warmup, 1),
             "ms_per_step": round(dt / nst * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": SparkDownStep.config(work),
+            "data": "synthetic", "config": work.config(),
             "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "kind": "oracle",
                              "cores": threads_used(),
                              "sample": f"{nst} full steps of the workload on the host"},
