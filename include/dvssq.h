@@ -210,10 +210,15 @@ DVSSQ_API dvssq_status dvssq_forward_workspace_size(const dvssq_shape *shape, in
  *            nearest even of the fp32 result)
  *   path     DVSSQ_PATH_*
  *   workspace device scratch of at least dvssq_forward_workspace_size bytes
- * Arithmetic: the GEMV path multiplies exact FP16 codes by the FP16-rounded
- * xr on tensor cores with FP32 accumulation and applies s4/s8 in FP32; the
- * GEMM path stages q*s in FP16 (exact for INT4 inside the ranges of
- * fp16_unsafe_scales) and xr in FP16, accumulating in FP32.
+ * Arithmetic:
+ *   T <= 2: exact int32 dot products (DP2A) of the codes with xr held as
+ *     int16, one FP32 scale per 64 columns (relative step 2^-15; salient
+ *     entries one scale per 128-entry chunk); s4/s8 applied in FP32.
+ *   3 <= T <= 16: exact FP16 codes times the FP16-rounded xr on tensor cores
+ *     with FP32 accumulation; s4/s8 applied in FP32.
+ *   T > 16 (GEMM): q*s staged in FP16 (exact for INT4 inside the ranges of
+ *     fp16_unsafe_scales) and xr in FP16, accumulating in FP32.
+ *   The partial sums are added in a fixed order: results are deterministic.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
 DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvssq_weights *w,
                                   const void *x, int64_t T, const void *bias,
