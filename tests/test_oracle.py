@@ -453,3 +453,177 @@ def test_mlp_block_matches_dense_composition():
     # may differ only where a sum lands within ~1e-12 of a rounding boundary
     assert np.mean(y == ref) > 0.99
     assert np.max(np.abs(y - ref)) <= 2.0 ** -7 * np.max(np.abs(ref))
+
+
+# ------------------------------------------- planted pins (independent) -----
+
+def _HK(K, b):
+    """H_K = diag(H_b, ...) from scipy's Sylvester Hadamard, divided by sqrt(b)
+    (for b = 256 the division by 16 is exact)."""
+    from scipy.linalg import block_diag, hadamard
+    Hb = hadamard(b).astype(np.float64) / math.sqrt(b)
+    return block_diag(*([Hb] * (K // b)))
+
+
+def test_salience_activation_factor_planted():
+    # Tier A salience on the ROTATED weights times the activation scale of
+    # the rotated column: six planted rotated columns with exact norms n and
+    # scales a.  a*n = (8, 7, 4, 8, 2, 12) selects {0, 3, 5}; each plausible
+    # mistake selects another set: a^2*n {0, 2, 5}, sqrt(a)*n {0, 1, 3},
+    # n alone {0, 3, 4}, a*n^2 {0, 1, 3}, n/a {0, 3, 4}.  Scoring the
+    # unrotated W (all of whose columns have equal norms here) would select
+    # by a alone.
+    b, K, M = 256, 256, 6
+    n = np.array([8.0, 7.0, 2.0, 8.0, 8.0, 3.0])
+    a = np.array([1.0, 1.0, 2.0, 1.0, 0.25, 4.0], dtype=np.float32)
+    pos = np.array([3, 40, 77, 130, 200, 251])
+    W_rot = np.zeros((M, K))
+    for c in range(6):
+        W_rot[c, pos[c]] = n[c]                 # one nonzero per row: exact norms
+    W = W_rot @ _HK(K, b)                       # original domain, every entry +-n/16
+    assert np.array_equal(W, O.rn_bf16(W))      # BF16 values, as the encoder takes
+    act = np.full(K, 3.0, dtype=np.float32)     # columns with zero norm score 0
+    act[pos] = a
+    enc = O.encode(W, act, b, 0, n_sal=3, with_svd=False)
+    assert list(enc["sal_idx"]) == [3, 130, 251]
+    assert list(enc["score"][pos]) == [8.0, 7.0, 4.0, 8.0, 2.0, 12.0]
+
+
+def _planted_grid(seed, M=8, K=512, b=256, n_sal=64):
+    """Rotated-domain weights on the INT4/INT8 grids: W_rot = Q s4 outside the
+    salient set P and Q8 s8 on it, every group with a +-7 (so s4 comes back)
+    and every row with a +-127 in P (so s8 comes back); |Q8| >= 64 keeps P
+    the top n_sal columns by norm for activation scales in [1, 1.5]."""
+    rng = np.random.default_rng(seed)
+    P = np.sort(rng.choice(K, n_sal, replace=False))
+    nonsal = np.setdiff1d(np.arange(K), P)
+    s4 = 2.0 ** rng.integers(-12, -7, size=(M, K // 64))
+    s8 = 2.0 ** rng.integers(-4, -1, size=M)
+    Q = rng.integers(-6, 7, size=(M, K))
+    Q[:, P] = 0
+    for i in range(M):
+        for g in range(K // 64):
+            cols = nonsal[(nonsal >= 64 * g) & (nonsal < 64 * g + 64)]
+            Q[i, rng.choice(cols)] = rng.choice([-7, 7])
+    Q8 = rng.integers(64, 128, size=(M, n_sal)) * rng.choice([-1, 1], size=(M, n_sal))
+    Q8[np.arange(M), rng.integers(0, n_sal, size=M)] = 127
+    W_rot = (Q.reshape(M, K // 64, 64) * s4[..., None]).reshape(M, K)
+    W_rot[:, P] = Q8 * s8[:, None]
+    return dict(P=P, Q=Q, s4=s4, Q8=Q8, s8=s8, W_rot=W_rot)
+
+
+def test_grid_round_trip_encode_and_forward():
+    # W = (Q s4 + scatter(Q8 s8)) H_K built with scipy's Hadamard: encode
+    # must return exactly the planted salient set, codes and scales, a zero
+    # residual, and forward must equal the dense W x (MiniCPM card §2 runtime
+    # equation; rotation invariance of §1) to fp64 rounding.
+    b, K, M = 256, 512, 8
+    pl = _planted_grid(3, M, K, b)
+    HK = _HK(K, b)
+    W = pl["W_rot"] @ HK
+    act = (1.0 + 0.5 * np.random.default_rng(4).random(K)).astype(np.float32)
+    enc = O.encode(W, act, b, 0, n_sal=64)
+    assert np.array_equal(enc["sal_idx"], pl["P"])
+    assert np.array_equal(enc["q"], pl["Q"])
+    assert np.array_equal(enc["s4"], pl["s4"])
+    assert np.array_equal(enc["q8"].astype(np.int64), pl["Q8"])
+    assert np.array_equal(enc["s8"], pl["s8"])
+    assert not np.any(enc["R"])                                  # residual exactly zero
+    rng = np.random.default_rng(5)
+    x = O.rn_bf16(rng.standard_normal((3, K)))
+    bias = O.rn_bf16(rng.standard_normal(M))
+    z = (np.zeros((M, 0)), np.zeros((0, K)))
+    y = O.forward(enc, x, bias, U=z[0], V=z[1])
+    ref = x @ W.T + bias
+    assert np.abs(y - ref).max() <= 1e-12 * np.abs(ref).max()
+    # the rank-r term acts on the rotated activations: W_eff = (W_rot + U V) H_K
+    U = O.rn_bf16(0.01 * rng.standard_normal((M, 4)))
+    V = O.rn_bf16(0.01 * rng.standard_normal((4, K)))
+    y = O.forward(enc, x, U=U, V=V)
+    ref = x @ ((pl["W_rot"] + U @ V) @ HK).T
+    assert np.abs(y - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_residual_excludes_salient_columns_and_is_the_rounding_error():
+    # Tier C: R = W_bg - What_bg, W_bg with the salient columns removed.  Off
+    # the grid, R at a salient column is 0 (neither W_bg nor What4 holds it)
+    # and elsewhere it is w - q s4 with q the brute-force nearest code.
+    b, K, M = 256, 512, 8
+    pl = _planted_grid(6, M, K, b)
+    rng = np.random.default_rng(7)
+    W_rot = pl["W_rot"].copy()
+    nonsal = np.setdiff1d(np.arange(K), pl["P"])
+    jitter = rng.uniform(-0.4, 0.4, size=(M, nonsal.size)) * np.repeat(pl["s4"], 64, axis=1)[:, nonsal]
+    W_rot[:, nonsal] += jitter                  # the +-7 anchors stay the group maxima
+    W = W_rot @ _HK(K, b)
+    enc = O.encode(W, np.ones(K, np.float32), b, 0, n_sal=64)
+    assert np.array_equal(enc["sal_idx"], pl["P"])
+    R = enc["R"]
+    assert not np.any(R[:, pl["P"]])
+    Wr = enc["W_rot"]
+    for i, j in ((0, nonsal[0]), (3, nonsal[100]), (7, nonsal[-1])):
+        s = enc["s4"][i, j // 64]
+        q = _rtn_brute(Wr[i, j], s, -8, 7)
+        assert R[i, j] == Wr[i, j] - q * s
+    assert np.abs(R[:, nonsal]).max() <= 0.5 * enc["s4"].max()
+
+
+def test_svd_recovers_planted_rank_r():
+    # Tier C / §2: a residual of exact rank r with distinct singular values
+    # sigma is returned as A B = R; the split is A = U sqrt(S), B = sqrt(S) V^T;
+    # truncation to r' < r keeps the planted leading terms.
+    rng = np.random.default_rng(31)
+    M, K, r = 40, 70, 4
+    U0, _ = np.linalg.qr(rng.standard_normal((M, r)))
+    V0, _ = np.linalg.qr(rng.standard_normal((K, r)))
+    sigma = np.array([5.0, 3.0, 2.0, 0.5])
+    R = U0 @ np.diag(sigma) @ V0.T
+    A, B, S = O.svd_factors(R, r, round_bf16=False)
+    assert np.allclose(S[:r], sigma, rtol=0, atol=1e-13)
+    assert np.all(S[r:] < 1e-13)
+    assert np.abs(A @ B - R).max() < 1e-13
+    assert np.allclose(np.linalg.norm(A, axis=0), np.sqrt(sigma), atol=1e-13)
+    assert np.allclose(np.linalg.norm(B, axis=1), np.sqrt(sigma), atol=1e-13)
+    A2, B2, _ = O.svd_factors(R, 2, round_bf16=False)
+    assert np.abs(A2 @ B2 - U0[:, :2] @ np.diag(sigma[:2]) @ V0[:, :2].T).max() < 1e-13
+
+
+def test_column_ssq_tree_on_exactly_summable_inputs():
+    # Where every partial sum is exact (small dyadic values), any summation
+    # order gives the same bits: the fixed tree equals a plain row-ascending
+    # sum and the exact integer sum.
+    rng = np.random.default_rng(37)
+    Wr = rng.integers(-20, 21, size=(333, 64)).astype(np.float64) / 8.0
+    tree = O.column_ssq(Wr)
+    seq = np.zeros(64)
+    for i in range(Wr.shape[0]):
+        seq = seq + Wr[i] * Wr[i]
+    exact = (np.rint(Wr * 8).astype(np.int64) ** 2).sum(axis=0) / 64.0
+    assert np.array_equal(tree, seq) and np.array_equal(tree, exact)
+
+
+@pytest.mark.parametrize("seed", [0, 4])
+def test_selection_valid_against_exact_scores_near_ties(seed):
+    # Planted exact ties whose squares straddle 16-row chunk boundaries: the
+    # fp64 rounding decides which tied columns make the top n_sal.  The
+    # oracle's fixed tree and a plain sequential sum both yield a valid
+    # top-n_sal set of the EXACT scores (rational arithmetic), though not the
+    # same set: the tree's shape is a reading (R3), not a fact of the pages.
+    import exact_topk as X
+    W, n_sal = X.near_tie_weight(seed)
+    Wf = O.torch_bf16_to_f64(W)
+    assert O.rotation_inexact_blocks(Wf, 256) == 0
+    act = np.ones(Wf.shape[1], np.float32)
+    Wr = O.rotate(Wf, 256)
+    score = O.salience(Wr, act)
+    sal = O.select_salient(score, n_sal)
+    info = X.check_selection_valid(Wr, act, sal, n_sal)
+    assert info["exact_ties"] == 16                 # the boundary sits in a 16-way tie
+    tied = np.argsort(-score, kind="stable")[8:24]
+    assert len(set(score[tied])) > 1                # ... which rounding splits
+    seq = np.zeros(Wr.shape[1])
+    for i in range(Wr.shape[0]):
+        seq = seq + Wr[i] * Wr[i]
+    sal_seq = O.select_salient(np.sqrt(seq), n_sal)
+    X.check_selection_valid(Wr, act, sal_seq, n_sal)
+    assert not np.array_equal(sal, sal_seq)
