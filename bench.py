@@ -601,6 +601,135 @@ class StackChainStep(StackStep):
     fused = False
 
 
+class ForwardLeg:
+    """Forwards of one synthetic layer at fixed token counts, on rotating
+    pre-encoded copies whose total size exceeds L2 (decode GEMV for T <= 16,
+    the tensor-core GEMM above).  Unit: GB/s of packed bytes per forward for
+    the decode path, TFLOP/s (2 T M K + 2 T r (K + M)) for the GEMM path."""
+
+    def __init__(self, dv, synth, torch, rank_id, device, wl_name, tokens, n_copies):
+        self.dv, self.torch = dv, torch
+        wl = synth.WORKLOADS[wl_name]
+        self.wl, self.tokens, self.n_copies = wl, tuple(tokens), n_copies
+        M, K, r, n = wl.M, wl.K, wl.rank, wl.n_sal
+        self.M, self.K, self.r, self.n = M, K, r, n
+        self.shape = dv.Shape.make(M, K, wl.block, r, n)
+        self.name = f"{wl_name}_{M}x{K}_r{r}_fwd_T" + "+".join(str(t) for t in tokens)
+        self.unit = "TFLOP/s" if min(tokens) > 16 else "GB/s"
+        ws = torch.empty(dv.dvssq_encode_workspace_size(self.shape), dtype=torch.uint8,
+                         device=device)
+        self.copies = []
+        for c in range(n_copies):
+            off = 1000 * rank_id + c
+            U, V = synth.lowrank_factors(M, K, r, seed=wl.seed + 7 + off)
+            packed = dv.PackedWeights.empty(self.shape, device, U=U.to(device), V=V.to(device))
+            dv.dvssq_encode(self.shape, wl.weight(seed_offset=off).to(device),
+                            wl.act_scale(seed_offset=off).to(device), packed, workspace=ws)
+            self.copies.append(packed)
+        self.x = {T: wl.activations(T, seed_offset=rank_id).to(device) for T in tokens}
+        self.ws = {T: torch.empty(max(1, dv.dvssq_forward_workspace_size(self.shape, T)),
+                                  dtype=torch.uint8, device=device) for T in tokens}
+        self.y = {T: torch.empty((T, M), dtype=torch.float32, device=device) for T in tokens}
+        self.i = 0
+
+    @property
+    def graph_slots(self):
+        return self.n_copies
+
+    def step_slot(self, i):
+        packed = self.copies[i % self.n_copies]
+        for T in self.tokens:
+            self.dv.dvssq_linear_forward(self.shape, packed, self.x[T], y=self.y[T],
+                                         workspace=self.ws[T])
+
+    def step(self):
+        self.step_slot(self.i)
+        self.i += 1
+
+    def bytes_per_step(self):
+        return len(self.tokens) * packed_bytes(self.M, self.K, self.r, self.n)
+
+    def work_per_step(self):
+        M, K, r = self.M, self.K, self.r
+        return sum(2.0 * T * M * K + 2.0 * T * r * (K + M) for T in self.tokens)
+
+    def kernel_work(self, name):
+        if name == "pre_gemm":
+            return self.work_per_step()
+        T = max(self.tokens)
+        salp = (self.n + 63) // 64 * 64
+        kc = self.K + salp + 64
+        if name == "pre_act":
+            return T * self.K * 2 + T * kc * 2
+        if name == "pre_mat":
+            return packed_bytes(self.M, self.K, self.r, self.n) + self.M * kc * 2
+        return kernel_bytes(name, self.M, self.K, self.r, self.n, T)
+
+    def config(self):
+        mb = packed_bytes(self.M, self.K, self.r, self.n) / 1e6
+        return {"workload": self.name, "M": self.M, "K": self.K, "block": self.wl.block,
+                "rank": self.r, "n_sal": self.n, "tokens": list(self.tokens),
+                "l2": f"{self.n_copies} rotating encoded layers (~{self.n_copies * mb:.0f} MB) "
+                      "> 126 MB L2",
+                "lowrank_factors": "seeded synthetic U, V (values do not change the work)"}
+
+
+class MaterializeLeg:
+    """dvssq_materialize of the Spark down_proj (2560 x 10240, r = 16): the
+    dense BF16 W_eff in the original domain, on rotating packed copies.
+    Unit: GB/s of packed bytes read + BF16 bytes written."""
+
+    name = "spark_down_proj_2560x10240_r16_materialize"
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv = dv
+        self.fw = ForwardLeg(dv, synth, torch, rank_id, device, "spark_down", (1,), 8)
+        self.M, self.K, self.r, self.n = self.fw.M, self.fw.K, self.fw.r, self.fw.n
+        self.W = torch.empty((self.M, self.K), dtype=torch.bfloat16, device=device)
+        self.i = 0
+
+    graph_slots = 8
+
+    def step_slot(self, i):
+        self.dv.dvssq_materialize(self.fw.shape, self.fw.copies[i % 8], out=self.W)
+
+    def step(self):
+        self.step_slot(self.i)
+        self.i += 1
+
+    def bytes_per_step(self):
+        return packed_bytes(self.M, self.K, self.r, self.n) + self.M * self.K * 2
+
+    def kernel_work(self, name):
+        return self.bytes_per_step() if name == "materialize" else None
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "K": self.K, "block": 256, "rank": self.r,
+                "n_sal": self.n, "l2": "8 rotating packed layers (141 MB) > 126 MB L2; the "
+                "52 MB BF16 output is rewritten every step"}
+
+
+# Legs of the metric timed in the default single-GPU run besides the headline:
+# (name, constructor).  Each is built, timed and freed in turn.
+def leg_specs():
+    def fwd(wl, tokens, copies):
+        return lambda dv, synth, torch, r, d: ForwardLeg(dv, synth, torch, r, d, wl, tokens, copies)
+    return [
+        ("decode_T1", fwd("spark_down", (1,), 8)),
+        ("decode_T16", fwd("spark_down", (16,), 8)),
+        ("stack", StackStep),
+        ("prefill", PrefillStep),
+        ("bulk_encode", BulkEncodeStep),
+        ("materialize", MaterializeLeg),
+        ("minicpm_k_T1", fwd("minicpm_k", (1,), 192)),
+        ("minicpm_k_T8", fwd("minicpm_k", (8,), 192)),
+        ("minicpm_k_T64", fwd("minicpm_k", (64,), 192)),
+        ("minicpm_up_T1", fwd("minicpm_up", (1,), 16)),
+        ("minicpm_up_T8", fwd("minicpm_up", (8,), 16)),
+        ("minicpm_up_T64", fwd("minicpm_up", (64,), 16)),
+    ]
+
+
 WORKLOADS = {"spark_down": SparkDownStep, "decode": DecodeStep, "prefill": PrefillStep,
              "bulk_encode": BulkEncodeStep, "stack": StackStep, "stack_chain": StackChainStep}
 
@@ -645,6 +774,157 @@ def job_throughput(world, units_per_rank_step, ms_step, scale):
     return world * units_per_rank_step / (ms_step * 1e-3) / scale
 
 
+def cpu_info():
+    """(logical CPUs of the host, CPU model name)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def measure(work, dv, torch, steps, warmup, world, device, local, key, use_graphs=True):
+    """Time one workload: W warm-up steps, K timed steps (CUDA graph replay
+    when the workload has graph slots) bracketed by a barrier and a device
+    synchronize, clocks sampled meanwhile; then the same K steps eagerly with
+    per-launch CUDA events for the per-kernel times and the roofline of the
+    dominant kernel."""
+    unit = getattr(work, "unit", "GB/s")
+    W = max(3, warmup)
+    for _ in range(W):
+        work.step()
+    torch.cuda.synchronize()
+    dv.dvssq_device_error(clear=True)
+
+    # one CUDA graph per rotation slot: the timed region replays the same
+    # launches without the host in the loop
+    graphs = []
+    n_slots = getattr(work, "graph_slots", 0)
+    if n_slots and use_graphs:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for slot in range(n_slots):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    work.step_slot(slot)
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(side)
+        for i in range(W):
+            graphs[i % n_slots].replay()
+        torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(steps):
+            if graphs:
+                graphs[i % n_slots].replay()
+            else:
+                work.step()
+        stop.record(stream)
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(stop), world, device)
+    err = dv.dvssq_device_error(clear=True)
+    del graphs
+    ms_step = ms / steps
+    if unit == "TFLOP/s":
+        bytes_step = None
+        value = job_throughput(world, work.work_per_step(), ms_step, 1e12)
+    else:
+        bytes_step = work.bytes_per_step()
+        value = job_throughput(world, bytes_step, ms_step, 1e9)
+
+    # per-kernel device times: the same K steps again with events around each launch
+    dv.dvssq_profile_reset()
+    dv.dvssq_profile_enable(True)
+    for _ in range(steps):
+        work.step()
+    torch.cuda.synchronize()
+    dv.dvssq_profile_collect()
+    dv.dvssq_profile_enable(False)
+    prof = dv.dvssq_profile_read()
+    launches_measured = sum(c for c, _ in prof.values())
+    pk, pk_kind = peaks()
+    # a kernel timed within a run of milliseconds runs at the burst tensor rate
+    tpk = pk["bf16_tflops"]
+    kernels = {}
+    tot_ms = sum(v[1] for v in prof.values())
+    kb_fn = getattr(work, "kernel_work", None) or (
+        lambda name: kernel_bytes(name, work.M, work.K, work.r, work.n, 16))
+    for name, (cnt, kms) in prof.items():
+        avg = kms / cnt
+        ent = {"launches": cnt, "avg_us": round(avg * 1e3, 3), "share": round(kms / tot_ms, 4)}
+        b = kb_fn(name)
+        if b is not None:
+            if name == "pre_gemm":
+                tfs = b / (avg * 1e-3) / 1e12
+                ent.update(flops=b, tflops=round(tfs, 1), frac=round(tfs / tpk, 4))
+            else:
+                gbs = b / (avg * 1e-3) / 1e9
+                ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
+        kernels[name] = ent
+    # dominant kernel among those with an algorithmic work count
+    dom = max((kv for kv in prof.items() if kb_fn(kv[0]) is not None), key=lambda kv: kv[1][1])[0]
+    db = kb_fn(dom)
+    dom_avg_ms = prof[dom][1] / prof[dom][0]
+    if dom == "pre_gemm":
+        achieved = db / (dom_avg_ms * 1e-3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
+                    "peak": tpk,
+                    "peak_source": pk_kind + " bf16 burst (a kernel timed within a short run; "
+                                             "f16 has the same dense rate)",
+                    "unit": "TFLOP/s", "frac": round(achieved / tpk, 4),
+                    "traffic": dram_traffic(dom, key),
+                    "algorithmic_flops_per_launch": db}
+    else:
+        achieved = db / (dom_avg_ms * 1e-3) / 1e9
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                    "peak": pk["hbm_gbs"], "peak_source": pk_kind, "unit": "GB/s",
+                    "frac": round(achieved / pk["hbm_gbs"], 4),
+                    "traffic": dram_traffic(dom, key),
+                    "algorithmic_bytes_per_launch": db}
+    return dict(ms_step=ms_step, value=value, unit=unit, bytes_step=bytes_step, kernels=kernels,
+                roofline=roofline, launches=launches_measured, err=err, clocks=clk.summary(),
+                W=W, barrier=barrier, stream=stream)
+
+
+def run_legs(dv, synth, torch, rank, device, local, steps, warmup, only=()):
+    """Every leg of the metric besides the headline, each timed on its own."""
+    legs = {}
+    for name, ctor in leg_specs():
+        if only and name not in only:
+            continue
+        work = ctor(dv, synth, torch, rank, device)
+        n = steps if name not in ("bulk_encode", "stack") else max(5, steps // 3)
+        r = measure(work, dv, torch, n, warmup, 1, device, local, name)
+        ent = {"workload": work.config()["workload"], "value": round(r["value"], 2),
+               "unit": r["unit"], "ms_per_step": round(r["ms_step"], 5), "steps": n,
+               "warmup": r["W"], "roofline": r["roofline"], "kernels": r["kernels"],
+               "gpu_launches": r["launches"], "device_error_word": r["err"],
+               "clocks": r["clocks"], "l2": work.config().get("l2")}
+        if r["unit"] == "GB/s":
+            ent["frac_of_hbm"] = round(r["value"] / peaks()[0]["hbm_gbs"], 4)
+        legs[name] = ent
+        del work
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return legs
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -655,6 +935,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the other legs of the metric (timed by default on one GPU)")
+    ap.add_argument("--legs", default="",
+                    help="comma-separated subset of the legs to time (default: all)")
     ap.add_argument("--layers", type=int, default=36,
                     help="blocks of the stack workloads (36 is the full model; fewer for profiling)")
     args = ap.parse_args()
@@ -680,108 +964,12 @@ def main():
                                 device_id=torch.device(device))
     StackStep.n_layers = args.layers
     work = WORKLOADS[args.workload](dv, synth, torch, rank, device)
-    unit = getattr(work, "unit", "GB/s")
-    W = max(3, args.warmup)
-    for _ in range(W):
-        work.step()
-    torch.cuda.synchronize()
-    dv.dvssq_device_error(clear=True)
-
-    # one CUDA graph per rotation slot: the timed region replays the same
-    # launches without the host in the loop
-    graphs = []
-    n_slots = getattr(work, "graph_slots", 0)
-    if n_slots and not args.no_graphs:
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            for slot in range(n_slots):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=side):
-                    work.step_slot(slot)
-                graphs.append(g)
-        torch.cuda.current_stream().wait_stream(side)
-        for i in range(W):
-            graphs[i % n_slots].replay()
-        torch.cuda.synchronize()
-
-    def timed_step(i):
-        if graphs:
-            graphs[i % n_slots].replay()
-        else:
-            work.step()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    stream = torch.cuda.current_stream()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    with ClockSampler(local) as clk:
-        start.record(stream)
-        for i in range(args.steps):
-            timed_step(i)
-        stop.record(stream)
-        barrier()
-    ms = max_over_ranks(start.elapsed_time(stop), world, device)
-    err = dv.dvssq_device_error(clear=True)
-    ms_step = ms / args.steps
-    if unit == "TFLOP/s":
-        bytes_step = None
-        value = job_throughput(world, work.work_per_step(), ms_step, 1e12)
-    else:
-        bytes_step = work.bytes_per_step()
-        value = job_throughput(world, bytes_step, ms_step, 1e9)
-
-    # per-kernel device times: the same K steps again with events around each launch
-    dv.dvssq_profile_reset()
-    dv.dvssq_profile_enable(True)
-    for _ in range(args.steps):
-        work.step()
-    torch.cuda.synchronize()
-    dv.dvssq_profile_collect()
-    dv.dvssq_profile_enable(False)
-    prof = dv.dvssq_profile_read()
-    launches_measured = sum(c for c, _ in prof.values())
-    pk, pk_kind = peaks()
-    kernels = {}
-    tot_ms = sum(v[1] for v in prof.values())
-    kb_fn = getattr(work, "kernel_work", None) or (
-        lambda name: kernel_bytes(name, work.M, work.K, work.r, work.n, 16))
-    for name, (cnt, kms) in prof.items():
-        avg = kms / cnt
-        ent = {"launches": cnt, "avg_us": round(avg * 1e3, 3), "share": round(kms / tot_ms, 4)}
-        b = kb_fn(name)
-        if b is not None:
-            if name == "pre_gemm":
-                tfs = b / (avg * 1e-3) / 1e12
-                ent.update(flops=b, tflops=round(tfs, 1),
-                           frac=round(tfs / pk["bf16_tflops_sustained"], 4))
-            else:
-                gbs = b / (avg * 1e-3) / 1e9
-                ent.update(bytes=b, gbs=round(gbs, 1), frac=round(gbs / pk["hbm_gbs"], 4))
-        kernels[name] = ent
-    # dominant kernel among those with an algorithmic work count
-    dom = max((kv for kv in prof.items() if kb_fn(kv[0]) is not None), key=lambda kv: kv[1][1])[0]
-    db = kb_fn(dom)
-    dom_avg_ms = prof[dom][1] / prof[dom][0]
-    if dom == "pre_gemm":
-        achieved = db / (dom_avg_ms * 1e-3) / 1e12
-        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1),
-                    "peak": pk["bf16_tflops_sustained"],
-                    "peak_source": pk_kind + " (bf16 sustained; f16 has the same dense rate)",
-                    "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
-                    "traffic": dram_traffic(dom, args.workload),
-                    "algorithmic_flops_per_launch": db}
-    else:
-        achieved = db / (dom_avg_ms * 1e-3) / 1e9
-        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
-                    "peak": pk["hbm_gbs"], "peak_source": pk_kind, "unit": "GB/s",
-                    "frac": round(achieved / pk["hbm_gbs"], 4),
-                    "traffic": dram_traffic(dom, args.workload),
-                    "algorithmic_bytes_per_launch": db}
+    r = measure(work, dv, torch, args.steps, args.warmup, world, device, local, args.workload,
+                use_graphs=not args.no_graphs)
+    unit, value, ms_step, bytes_step = r["unit"], r["value"], r["ms_step"], r["bytes_step"]
+    kernels = r["kernels"]
+    cfg = work.config()
+    barrier, stream = r["barrier"], r["stream"]
     # the decode GEMV's own roofline (the headline HBM-bound kernel)
     dm = kernels.get("dec_row") or kernels.get("dec_main") or kernels.get("mlp_stack")
 
@@ -812,18 +1000,29 @@ def main():
         sample_bytes = getattr(work, "_oracle_bytes", None) or bytes_step
         what = getattr(work, "oracle_what", "full step(s) of the same workload "
                                             "(encode without SVD + 2 forwards)")
+        nproc, model = cpu_info()
         cpu = {"value": round(sample_bytes * nst / dt / 1e9, 4), "unit": "GB/s",
-               "cores": threads_used(), "kind": "oracle",
-               "sample": f"{nst} {what} on the host, {dt:.1f} s"}
+               "cores": threads_used(), "nproc": nproc, "cpu_model": model, "kind": "oracle",
+               "sample": f"{nst} {what} on the host, {dt:.1f} s; numpy fp64 with "
+                         f"{threads_used()} BLAS threads for the matrix products, "
+                         "single-threaded Python loops for the sums of squares"}
+
+    legs = None
+    if world == 1 and args.workload == "spark_down" and not args.no_legs:
+        del work
+        torch.cuda.empty_cache()
+        only = tuple(x for x in args.legs.split(",") if x)
+        legs = run_legs(dv, synth, torch, rank, device, local, args.steps, args.warmup, only)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": W, "ms_per_step": round(ms_step, 4),
+            "steps": args.steps, "warmup": r["W"], "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp16",
             "data": "synthetic (seeded N(0,0.02) weights with outlier columns, N(0,1) tokens)",
-            "config": work.config(), "roofline": roofline, "kernels": kernels,
-            "decode_gemv": dm, "gpu_launches": launches_measured,
-            "e2e": e2e, "cpu_baseline": cpu, "device_error_word": err,
-            "clocks": clk.summary()}
+            "config": cfg,
+            "roofline": r["roofline"], "kernels": kernels,
+            "decode_gemv": dm, "gpu_launches": r["launches"],
+            "e2e": e2e, "cpu_baseline": cpu, "device_error_word": r["err"],
+            "clocks": r["clocks"], "legs": legs}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

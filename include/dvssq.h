@@ -35,6 +35,10 @@
  * - A workspace must not be shared by calls that may run concurrently.
  * - Kernels never wait without a bound: a wait that runs out sets a device
  *   error word that dvssq_device_error() reads and clears.
+ * - Per-device set-up (kernel attributes, constant tables, the address of
+ *   the static scratch array) runs on the first call on a device and is kept
+ *   for the life of the process: do not use the library across a
+ *   cudaDeviceReset of a device it has run on.
  */
 #ifndef DVSSQ_H
 #define DVSSQ_H
@@ -106,9 +110,10 @@ typedef struct {
 /* Diagnostics of one encode (host struct, filled when non-NULL). */
 typedef struct {
   /* row-blocks whose +-1 Hadamard sums are not provably exact in fp64
-     (BF16 exponent spread above 45 - log2(b) bits); codes of such blocks
-     may differ from an exact-arithmetic encoder in the last rounding.  The
-     test runs only in calls that ask for this struct.                    */
+     (BF16 exponent spread above 45 - log2(b) bits).  The encoder sums
+     these blocks exactly in integers and rounds each sum once, so their
+     codes equal an exact-arithmetic encoder's; blocks holding Inf or NaN
+     keep the fp64 butterfly's (non-finite) values.  A diagnostic count.  */
   int64_t inexact_rotation_blocks;
   /* INT4 groups with a nonzero scale outside [2^-17, 8188] and rows with a
      nonzero INT8 scale outside [2^-17, 511]: the prefill path stages q*s
@@ -166,8 +171,10 @@ DVSSQ_API dvssq_status dvssq_gelu_mul(const void *gate, const void *up, void *h,
 DVSSQ_API dvssq_status dvssq_encode_workspace_size(const dvssq_shape *shape, size_t *bytes);
 
 /* Encoder (Spark card, Tiers A and B; MiniCPM card §1-§2):
- *   1. W_rot = W . H_K in fp64; each +-1 sum is exact whenever
- *      inexact_rotation_blocks is 0, the scale 1/sqrt(b) is applied once.
+ *   1. W_rot = W . H_K: each +-1 sum is computed exactly and rounded once
+ *      to fp64 (fp64 butterflies where the block's exponent spread makes
+ *      them exact, integer sums elsewhere); the scale 1/sqrt(b) is applied
+ *      once.
  *   2. score_j = act_scale_j * sqrt(sum_i W_rot[i,j]^2); the sum runs over
  *      rows in chunks of 16 (within a chunk acc = acc + w*w, each operation
  *      rounded), the chunk sums in groups of 8 consecutive chunks (each group
@@ -226,6 +233,23 @@ DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvss
                                   void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* Dense effective weights of a packed layer, in the original (unrotated)
+ * domain: the library's counterpart of the Spark card's materialize_weights()
+ * ("Spark-X2.5-4B-Hadamard-GSQ", "Quickstart & Inference Guide": the
+ * quantised weights materialised as plain BF16):
+ *   W_eff = RN_bf16( (What4 + scatter(What8) + U V) . H_K ),
+ *   What4[i][j] = q4_ij s4_i,j/64,  What8[i][sal_k] = q8_ik s8_i,
+ * so that W_eff x equals the dvssq_linear_forward result up to rounding
+ * (H_K is symmetric and H_K^2 = I: MiniCPM card, Mathematical Foundations
+ * §1).  Evaluated in FP32 (U V on tensor cores with FP32 accumulation, the
+ * Walsh-Hadamard transform in FP32), then rounded once to BF16.
+ *   shape, w  as dvssq_linear_forward (w read only; U, V used when rank > 0)
+ *   W_eff     bf16 [M][K] (device, caller-owned, 16-byte aligned), written
+ * Stream-ordered and asynchronous; no workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, DEVICE, CUDA.        */
+DVSSQ_API dvssq_status dvssq_materialize(const dvssq_shape *shape, const dvssq_weights *w,
+                                         void *W_eff, void *stream);
+
 /* Allocation-free decode forward.  The paper has no counterpart: this entry
  * exists for callers that cannot obtain device memory for a workspace --
  * for example a host program that links only this library and has no device
@@ -240,9 +264,9 @@ DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvss
  *     DVSSQ_PATH_DECODE) exceeds DVSSQ_STATIC_SCRATCH_BYTES are rejected with
  *     DVSSQ_ERR_WORKSPACE before any launch; dvssq_last_error() then states
  *     the bytes needed and the limit.  T > 16 returns UNSUPPORTED_SHAPE.
- *   - The first call on a device looks up the array's device address
- *     (once per device, with that device current); make that first call
- *     before any stream capture.
+ *   - The first call on a device checks the device and looks up the array's
+ *     device address (once per device, with that device current, kept until
+ *     the process exits); make that first call before any stream capture.
  *   - All calls share the one array, which keeps the last call's contents
  *     (the kernels clear what must start at zero).  Calls that may overlap
  *     on the GPU -- concurrent streams, other host threads -- race on it
@@ -301,8 +325,27 @@ DVSSQ_API dvssq_status dvssq_mlp_stack_forward(const dvssq_mlp_layer *layers, in
                                                size_t workspace_bytes, void *stream);
 
 /* Reads (and clears when `clear` != 0) the device error word of the current
- * device; synchronises the device.  0 means no kernel gave up a wait.     */
+ * device; synchronises the device.  0 means no kernel gave up a wait; bit 0:
+ * an mbarrier wait ran out, bit 1: a tensor-memory accumulator wait, bit 2:
+ * a kernel saw an unsupported shape, bit 3: a grid-barrier wait.          */
 DVSSQ_API dvssq_status dvssq_device_error(uint32_t *word, int32_t clear);
+
+/* Wait limit of every bounded wait in the library's kernels, in SM clock
+ * cycles (default 4e9, about 2 s); cycles <= 0 restores the default.  Not
+ * part of the method: it lets a test shorten the limit so that a wait runs
+ * out quickly.  Applies to the current device; synchronises it.
+ * Errors: DEVICE, CUDA.                                                    */
+DVSSQ_API dvssq_status dvssq_set_wait_limit(int64_t cycles);
+
+/* Bounded-wait self-test (not part of the method): launches one warp that
+ * waits, through the kernels' own bounded-wait helpers, on something that
+ * is never signalled -- which = 0: an mbarrier expecting an arrival that
+ * never comes; which = 1: a grid-barrier counter nobody increments.  The
+ * wait gives up after the wait limit, sets bit 0 (mbarrier) or bit 3 (grid
+ * barrier) of the device error word, and the kernel returns; nothing
+ * faults, and the context stays usable.  Stream-ordered.
+ * Errors: INVALID_ARG, DEVICE, CUDA.                                       */
+DVSSQ_API dvssq_status dvssq_selftest_wait(int32_t which, void *stream);
 
 /* Per-kernel device timing.  While enabled, every launch is bracketed by
  * CUDA events on its own stream (and launched without programmatic

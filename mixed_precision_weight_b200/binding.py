@@ -26,10 +26,11 @@ __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
     "dvssq_fwht", "dvssq_gelu_mul", "dvssq_encode_workspace_size", "dvssq_encode",
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
-    "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
+    "dvssq_materialize", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
     "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
-    "dvssq_profile_reset", "Y_F32", "Y_BF16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
+    "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
+    "Y_F32", "Y_BF16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -50,11 +51,11 @@ EXPORTED_SYMBOLS = (
     "dvssq_abi_version", "dvssq_status_string", "dvssq_last_error", "dvssq_fwht",
     "dvssq_gelu_mul",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
-    "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_device_error",
-    "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
+    "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_materialize",
+    "dvssq_device_error", "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
-    "dvssq_profile_reset",
+    "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
 )
 
 
@@ -104,6 +105,7 @@ _sig = {
                                             _P, ctypes.c_size_t, _P]),
     "dvssq_linear_forward_static": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights),
                                                    _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
+    "dvssq_materialize": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights), _P, _P]),
     "dvssq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "dvssq_mlp_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32,
                                                       ctypes.POINTER(ctypes.c_size_t)]),
@@ -118,6 +120,8 @@ _sig = {
                                          ctypes.POINTER(ctypes.c_int64),
                                          ctypes.POINTER(ctypes.c_double)]),
     "dvssq_profile_reset": (ctypes.c_int, []),
+    "dvssq_set_wait_limit": (ctypes.c_int, [ctypes.c_int64]),
+    "dvssq_selftest_wait": (ctypes.c_int, [ctypes.c_int32, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(lib, _name)
@@ -287,6 +291,17 @@ def dvssq_linear_forward_static(shape: Shape, w: PackedWeights, x: torch.Tensor,
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
+def dvssq_materialize(shape: Shape, w: PackedWeights, out: torch.Tensor | None = None,
+                      stream=None):
+    """Dense BF16 W_eff [M][K] in the original domain (materialize_weights)."""
+    if out is None:
+        out = torch.empty((shape.M, shape.K), dtype=torch.bfloat16, device=w.q4.device)
+    wc = w._c(shape)
+    _check(lib.dvssq_materialize(ctypes.byref(shape), ctypes.byref(wc), _ptr(out),
+                                 _stream(stream)), "dvssq_materialize")
+    return out
+
+
 def _mlp_layers(layers) -> ctypes.Array:
     """[(gate, up, down)] of (Shape, PackedWeights) -> the C array of dvssq_mlp_layer."""
     arr = (_MlpLayer * len(layers))()
@@ -344,6 +359,16 @@ def dvssq_device_error(clear: bool = True) -> int:
     word = ctypes.c_uint32(0)
     _check(lib.dvssq_device_error(ctypes.byref(word), 1 if clear else 0), "dvssq_device_error")
     return word.value
+
+
+def dvssq_set_wait_limit(cycles: int = 0):
+    """Wait limit of the kernels' bounded waits (cycles; <= 0: the default)."""
+    _check(lib.dvssq_set_wait_limit(int(cycles)), "dvssq_set_wait_limit")
+
+
+def dvssq_selftest_wait(which: int, stream=None):
+    """One warp waits on something never signalled (0: mbarrier, 1: grid counter)."""
+    _check(lib.dvssq_selftest_wait(int(which), _stream(stream)), "dvssq_selftest_wait")
 
 
 def dvssq_profile_enable(on: bool = True):

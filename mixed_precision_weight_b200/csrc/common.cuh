@@ -3,8 +3,9 @@
 // PTX wrappers for mbarriers, bulk/tensor copies, programmatic dependent
 // launch, warp-level MMA and the 5th-generation tensor-core (tcgen05) ops,
 // plus exact format conversions.  Every wait is bounded: after
-// kWaitLimitCycles the waiter records an error code in g_dvssq_error and
-// gives up, so that no kernel can hang the device.
+// g_wait_limit cycles (kWaitLimitCycles unless the host shortened it) the
+// waiter records an error code in g_dvssq_error and gives up, so that no
+// kernel can hang the device.
 #pragma once
 
 #include <cuda.h>
@@ -30,6 +31,14 @@ __device__ __forceinline__ void set_error(uint32_t code) { atomicOr(&g_dvssq_err
 
 // ~2 s at 1.9 GHz: far beyond any legitimate wait, short enough to give up.
 constexpr long long kWaitLimitCycles = 4000000000LL;
+
+// The limit every bounded wait applies, in SM clock cycles.  The host sets
+// it through dvssq_set_wait_limit (a test shortens it to make a wait run out).
+__device__ long long g_wait_limit = kWaitLimitCycles;
+
+__device__ __forceinline__ long long wait_limit() {
+  return *(volatile long long *)&g_wait_limit;
+}
 
 // ------------------------------------------------------------ conversions -
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) {
@@ -134,17 +143,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait on phase `parity`; returns false (and flags the device error
-// word) if the phase did not complete within kWaitLimitCycles.
+// word) if the phase did not complete within the wait limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long t0 = clock64();
+  const long long t0 = clock64(), lim = wait_limit();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > lim) {
       set_error(kErrWaitMbarrier);
       return false;
     }
   }
   return true;
+}
+
+// Bounded wait, by one thread, until the global counter reaches `target`
+// (acquire).  Gives up, flags kErrWaitGrid and returns false when the wait
+// limit runs out or when the device error word changes from `err0` (another
+// CTA gave up first).
+__device__ __forceinline__ bool counter_wait(const unsigned int *ctr, unsigned int target,
+                                             uint32_t err0) {
+  const long long t0 = clock64(), lim = wait_limit();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (*(volatile uint32_t *)&g_dvssq_error != err0 || clock64() - t0 > lim) {
+      set_error(kErrWaitGrid);
+      return false;
+    }
+    __nanosleep(32);
+  }
 }
 
 // ------------------------------------------------------------ async copies -

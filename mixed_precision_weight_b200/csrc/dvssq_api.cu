@@ -81,6 +81,7 @@ dvssq_status ensure_device() {
   if ((e = prepare_encode_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_forward_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_stack_kernels()) != cudaSuccess) return cuda_fail(e);
+  if ((e = prepare_materialize_kernels()) != cudaSuccess) return cuda_fail(e);
   ready[dev] = 1;
   return DVSSQ_OK;
 }
@@ -285,6 +286,29 @@ dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvssq_weights 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = p == DVSSQ_PATH_DECODE ? launch_decode(a, st, launcher())
                                          : launch_prefill(a, st, launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
+dvssq_status dvssq_materialize(const dvssq_shape *shape, const dvssq_weights *w, void *W_eff,
+                               void *stream) {
+  dvssq_status s = check_shape(shape);
+  if (s != DVSSQ_OK) return s;
+  if (w == nullptr || W_eff == nullptr || w->q4 == nullptr || w->s4 == nullptr ||
+      w->s8 == nullptr)
+    return DVSSQ_ERR_INVALID_ARG;
+  if (shape->n_sal > 0 && (w->sal_idx == nullptr || w->q8 == nullptr)) return DVSSQ_ERR_INVALID_ARG;
+  if (shape->rank > 0 && (w->U == nullptr || w->V == nullptr)) return DVSSQ_ERR_INVALID_ARG;
+  const void *bufs[] = {W_eff, w->q4, w->s4, w->s8, w->sal_idx, w->q8, w->U, w->V};
+  for (const void *b : bufs)
+    if (b != nullptr && !aligned16(b)) return DVSSQ_ERR_MISALIGNED;
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
+  MaterializeArgs a;
+  a.M = shape->M; a.K = shape->K; a.block = shape->block; a.n_sal = shape->n_sal;
+  a.rank = shape->rank;
+  a.q4 = w->q4; a.s4 = w->s4; a.sal_idx = w->sal_idx; a.q8 = w->q8; a.s8 = w->s8;
+  a.U = w->U; a.V = w->V;
+  a.W = static_cast<uint16_t *>(W_eff);
+  const cudaError_t e = launch_materialize(a, static_cast<cudaStream_t>(stream), launcher());
   return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
 }
 

@@ -6,18 +6,23 @@
 //           one scale by 1/sqrt(b)); per-column sums of squares over fixed
 //           chunks of 16 rows, summed by the CTA into groups of 8 chunks; the
 //           last CTA of each column block adds the groups in order and writes
-//           score = a * sqrt(ssq).  Exactness check of every row-block.
+//           score = a * sqrt(ssq).  Every chunk is tested for exact fp64
+//           summation; a chunk that fails is recomputed row by row, its
+//           flagged row-blocks summed exactly in integers (exact_sum.cuh),
+//           and a per-(chunk, column block) row mask is written for pass 2.
 //   select  the n_sal largest scores (ties -> lower index) by an MSB-first
 //           radix select in one CTA that stops as soon as the boundary digit
 //           is taken whole; outputs sorted indices and per-32-column prefix
 //           counts.
 //   pass 2  whole rows per CTA (dynamic tile order): rotation again, salient
-//           values moved to a shared-memory stash and zeroed in place, INT4
+//           values (exact sums for the row-blocks pass 1 flagged) moved to a
+//           shared-memory stash and zeroed in place, INT4
 //           group RTN with BF16 scales, nibble packing, optional fp32
 //           residual; then the INT8 tier of the CTA's rows from the stash.
 #include <algorithm>
 
 #include "common.cuh"
+#include "exact_sum.cuh"
 #include "fwht_group.cuh"
 #include "kernels.h"
 
@@ -66,6 +71,13 @@ __device__ __forceinline__ uint16_t bf16_of_quotient(double a, double d, double 
   return f64_to_bf16_rn(q);
 }
 
+// Thread t's 16 outputs 16t .. 16t+15 of the exact +-1 sums of a row-block,
+// written to out[16t + j] (rare path: out of line, and through memory, so
+// that nothing of the caller's stays live across it).
+__device__ __noinline__ void exact_pm_sums16(const uint16_t *w, int b, int t, double *out) {
+  for (int j = 0; j < 16; ++j) out[16 * t + j] = exact_pm_sum(w, b, 16 * t + j);
+}
+
 // Per-halfword unsigned max / min of two pairs of 16-bit lanes.
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -102,13 +114,16 @@ __device__ __forceinline__ bool spread_exceeds(int emax, int emin1, int lg) {
 // CTA then forms the 8-chunk group sums (ascending chunks, from 0.0) in shared
 // memory, and the CTA that finishes a column block last adds that block's
 // group sums in ascending order and writes the scores.
-// STATS: also the exact-sum test behind info.inexact_rotation_blocks (only
-// when the caller asks for the diagnostics; the codes do not depend on it)
-template <int B, bool STATS>
+// Every chunk is tested for exact fp64 summation (BF16 exponent spread of the
+// whole chunk).  A chunk that fails is summed again row by row: a row whose
+// own spread exceeds the bound takes the exact integer sums, and its bit is
+// set in xmask[chunk * nkb + kb] (written for every chunk, 0 when it passes)
+// so that pass 2 takes the same path for that row-block.
+template <int B>
 __global__ void __launch_bounds__(128, 6) enc_pass1_kernel(
     const uint16_t *__restrict__ W, int M, int K, double c, const float *__restrict__ act_scale,
     double *__restrict__ gpart, double *__restrict__ score, unsigned int *__restrict__ done,
-    unsigned long long *__restrict__ info) {
+    unsigned long long *__restrict__ info, uint16_t *__restrict__ xmask) {
   constexpr int P = B / 16;
   constexpr int GPW = 32 / P;
   constexpr int NG = GPW * 4;
@@ -157,7 +172,7 @@ __global__ void __launch_bounds__(128, 6) enc_pass1_kernel(
     cp_async_wait<kStages - 1>();
     __syncwarp();
     const uint16_t *buf = ring[g][i % kStages];
-    if (STATS && i < nrows) {
+    if (i < nrows) {
       // this thread's 32 contiguous bytes of the row-block, for the exact-sum test
       const uint4 *wq = reinterpret_cast<const uint4 *>(buf) + 2 * t;
       const uint4 a = wq[0], b = wq[1];
@@ -183,9 +198,9 @@ __global__ void __launch_bounds__(128, 6) enc_pass1_kernel(
   cp_async_wait<0>();
 
   // Exact-sum test, first over the whole chunk: the chunk's spread bounds the
-  // spread of each of its row-blocks.  Only a chunk that fails it is checked
-  // row by row (from global memory).
-  if (STATS) {
+  // spread of each of its row-blocks.  Only a chunk that fails it is summed
+  // again row by row.
+  {
     const uint32_t mxh = max(mx & 0xFFFFu, mx >> 16), mnh = min(mn & 0xFFFFu, mn >> 16);
     const int emax = (int)(mxh >> 7);
     const int emin1 = mnh == 0xFFFFu ? 0xFFFF : max((int)((mnh + 1u) >> 7), 1);
@@ -195,28 +210,62 @@ __global__ void __launch_bounds__(128, 6) enc_pass1_kernel(
     for (int o = 1; o < P; o <<= 1) pk = vmax_u16x2(pk, __shfl_xor_sync(0xffffffffu, pk, o));
     const int gmax = (int)(pk >> 16), gmin1 = 0xFFFF - (int)(pk & 0xFFFFu);
     const bool fail = nrows > 0 && spread_exceeds(gmax, gmin1, lg);
+    uint32_t rowmask = 0u;
     // the warp's groups may differ: the whole warp runs the row loop (its
-    // shuffles need every lane), each group counting only its own rows
+    // shuffles and the rotation need every lane), each group keeping only
+    // its own rows
     if (__any_sync(0xffffffffu, fail)) {
       unsigned long long inexact = 0;
+      // a failing group sums its chunk again from zero; the other groups of
+      // the warp keep theirs (their rows are not re-added)
+      if (fail) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ssq[j] = 0.0;
+      }
+      uint16_t *buf = ring[g][0];
       for (int i = 0; i < kSsqChunk; ++i) {
         const bool row = fail && i < nrows;
-        uint32_t rx = 0u, rn = 0xFFFFFFFFu;
         if (row) {
-          const uint32_t *src =
-              reinterpret_cast<const uint32_t *>(W + (size_t)(r0 + i) * K + (size_t)kb * B);
-          for (int q = t; q < B / 2; q += P) exp_pair_stats(src[q], rx, rn);
+          const uint4 *src =
+              reinterpret_cast<const uint4 *>(W + (size_t)(r0 + i) * K + (size_t)kb * B);
+          for (int q = t; q < B / 8; q += P) reinterpret_cast<uint4 *>(buf)[q] = src[q];
         }
+        __syncwarp();
+        uint32_t rx = 0u, rn = 0xFFFFFFFFu;
+        if (row)
+          for (int q = t; q < B / 2; q += P)
+            exp_pair_stats(reinterpret_cast<const uint32_t *>(buf)[q], rx, rn);
         const uint32_t rxh = max(rx & 0xFFFFu, rx >> 16), rnh = min(rn & 0xFFFFu, rn >> 16);
         const int re = (int)(rxh >> 7);
         const int rm = rnh == 0xFFFFu ? 0xFFFF : max((int)((rnh + 1u) >> 7), 1);
         uint32_t rp = ((uint32_t)re << 16) | (uint32_t)(0xFFFF - rm);
 #pragma unroll
         for (int o = 1; o < P; o <<= 1) rp = vmax_u16x2(rp, __shfl_xor_sync(0xffffffffu, rp, o));
-        if (row) inexact += spread_exceeds((int)(rp >> 16), 0xFFFF - (int)(rp & 0xFFFFu), lg);
+        const bool exact_row =
+            row && spread_exceeds((int)(rp >> 16), 0xFFFF - (int)(rp & 0xFFFFu), lg);
+        double v[16];
+#pragma unroll
+        for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
+        fwht_group<B>(v, scratch[g], t);
+        if (exact_row && !block_has_nonfinite(buf, B)) {
+          exact_pm_sums16(buf, B, t, scratch[g]);   // the transpose scratch is free here
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = scratch[g][16 * t + j];
+        }
+        if (row) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const double w = B == 256 ? v[j] : __dmul_rn(v[j], c);
+            ssq[j] = __dadd_rn(ssq[j], __dmul_rn(w, w));
+          }
+        }
+        rowmask |= (uint32_t)exact_row << i;
+        inexact += exact_row;
+        __syncwarp();
       }
       if (t == 0 && inexact) atomicAdd(&info[0], inexact);
     }
+    if (t == 0 && chunk < nchunk) xmask[(size_t)chunk * nkb + kb] = (uint16_t)rowmask;
   }
 
   // chunk partials -> shared memory (the transpose scratch is free now)
@@ -531,6 +580,7 @@ struct Pass2Params {
   double *sv;
   unsigned int *tile_ctr;
   unsigned long long *info;
+  const uint16_t *xmask;   // pass 1's rows whose row-block takes the exact sums
 };
 
 // Staged outputs: thread t's 16 values at [16 t, 16 t + 16), the 16-byte
@@ -633,6 +683,17 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
 #pragma unroll
       for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
       fwht_group<B>(v, sgrp, t);
+      // row-blocks that pass 1 flagged: exact integer sums, rounded once (the
+      // mask was written by pass 1, which completed before the select kernel
+      // released this one; read from L2)
+      if (valid) {
+        const uint32_t mk = __ldcg(p.xmask + (size_t)(row >> 4) * (K / B) + kb);
+        if (((mk >> (row & 15)) & 1u) && !block_has_nonfinite(buf, B)) {
+          exact_pm_sums16(buf, B, t, sgrp);         // free until the staging below
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = sgrp[16 * t + j];
+        }
+      }
       // v holds the values the codes see: unscaled sums (b = 256) or w = c * sum
       if (!kPow2) {
 #pragma unroll
@@ -817,7 +878,7 @@ Pass2Plan pass2_plan(int M, int K, int B, int n_sal) {
 }
 
 struct EncodeLayout {
-  size_t info, ctr, done, zero_bytes, gpart, score, pref, sv, total;
+  size_t info, ctr, done, zero_bytes, gpart, score, pref, sv, xmask, total;
 };
 EncodeLayout encode_layout(int M, int K, int block, int n_sal) {
   const size_t nchunk = (size_t)(M + kSsqChunk - 1) / kSsqChunk;
@@ -841,6 +902,7 @@ EncodeLayout encode_layout(int M, int K, int block, int n_sal) {
   L.score = take((size_t)K * sizeof(double));
   L.pref = take((size_t)((K + 31) / 32) * sizeof(int32_t));
   L.sv = take(pl.smem ? 0 : (size_t)M * n_sal * sizeof(double));
+  L.xmask = take(nchunk * (size_t)(K / block) * sizeof(uint16_t));
   L.total = off;
   return L;
 }
@@ -878,6 +940,7 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
   auto *score = reinterpret_cast<double *>(ws + lay.score);
   auto *pref = reinterpret_cast<int32_t *>(ws + lay.pref);
   auto *sv = pl.smem ? nullptr : reinterpret_cast<double *>(ws + lay.sv);
+  auto *xmask = reinterpret_cast<uint16_t *>(ws + lay.xmask);
   const double c = sqrt(1.0 / (double)B);
 
   cudaError_t e = cudaMemsetAsync(info, 0, lay.zero_bytes, st);
@@ -885,11 +948,9 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
   const int nkb = K / B;
   const int NG = groups_per_cta(B);
   dim3 g1((unsigned)(((nchunk + NG - 1) / NG) * nkb));
-  const bool stats = a.info_host != nullptr;
-  auto p1 = B == 256 ? (stats ? enc_pass1_kernel<256, true> : enc_pass1_kernel<256, false>)
-                     : (stats ? enc_pass1_kernel<128, true> : enc_pass1_kernel<128, false>);
+  auto p1 = B == 256 ? enc_pass1_kernel<256> : enc_pass1_kernel<128>;
   e = L.launch("enc_pass1", p1, g1, dim3(128), 0, st, false, (const uint16_t *)a.W, M, K, c,
-               a.act_scale, gpart, score, done, info);
+               a.act_scale, gpart, score, done, info, xmask);
   if (e != cudaSuccess) return e;
   const size_t sel_smem = K <= kSelSmemKeys ? (size_t)K * sizeof(unsigned long long) : 0;
   e = L.launch("enc_select", enc_select_kernel, dim3(1), dim3(kSelThreads), sel_smem, st, true,
@@ -904,7 +965,7 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
   pp.c = c;
   pp.sal_idx = a.sal_idx; pp.sal_prefix = pref;
   pp.q4 = a.q4; pp.s4 = a.s4; pp.q8 = a.q8; pp.s8 = a.s8; pp.resid = a.resid;
-  pp.sv = sv; pp.tile_ctr = ctr; pp.info = info;
+  pp.sv = sv; pp.tile_ctr = ctr; pp.info = info; pp.xmask = xmask;
   if (B == 256)
     e = a.resid ? launch_pass2<256, true>(pp, pl.smem_bytes, st, L)
                 : launch_pass2<256, false>(pp, pl.smem_bytes, st, L);
@@ -928,8 +989,7 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L) {
 cudaError_t prepare_encode_kernels() {
   cudaError_t e;
   for (const void *f :
-       {(const void *)enc_pass1_kernel<256, true>, (const void *)enc_pass1_kernel<128, true>,
-        (const void *)enc_pass1_kernel<256, false>, (const void *)enc_pass1_kernel<128, false>})
+       {(const void *)enc_pass1_kernel<256>, (const void *)enc_pass1_kernel<128>})
     if ((e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;

@@ -181,6 +181,21 @@ cudaError_t prepare_forward_kernels();
 cudaError_t launch_decode(const ForwardArgs &a, cudaStream_t st, Launcher &L);
 cudaError_t launch_prefill(const ForwardArgs &a, cudaStream_t st, Launcher &L);
 
+// ------------------------------------------------------------ materialize -
+struct MaterializeArgs {
+  int M, K, block, n_sal, rank;
+  const uint8_t *q4;
+  const uint16_t *s4;
+  const int32_t *sal_idx;
+  const int8_t *q8;
+  const uint16_t *s8;
+  const uint16_t *U;
+  const uint16_t *V;
+  uint16_t *W;
+};
+cudaError_t launch_materialize(const MaterializeArgs &a, cudaStream_t st, Launcher &L);
+cudaError_t prepare_materialize_kernels();
+
 // Tensor-map encoder from the driver (resolved once through the runtime).
 CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,

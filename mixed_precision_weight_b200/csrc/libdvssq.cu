@@ -8,4 +8,6 @@
 #include "decode_row.cu"
 #include "prefill.cu"
 #include "stack.cu"
+#include "materialize.cu"
+#include "selftest.cu"
 #include "static_scratch.cu"

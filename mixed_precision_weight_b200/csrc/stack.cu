@@ -33,9 +33,9 @@
 //     phase; after the barrier the consumers of t sum the G shares in a fixed
 //     order.  No extra barrier is needed for it.
 //
-// Every wait is bounded (mbarriers via mbar_wait, the grid barrier by
-// kWaitLimitCycles); a timeout sets the device error word and every warp
-// leaves at its next wait.
+// Every wait is bounded (mbarriers and the grid barrier by the library's
+// wait limit); a timeout sets the device error word and every warp leaves at
+// its next wait.
 #include "common.cuh"
 #include "fwht_group.cuh"
 #include "kernels.h"
@@ -98,10 +98,10 @@ __device__ __forceinline__ uint32_t stk_splice(uint32_t a, uint32_t b, uint32_t 
 // waiting warp does not take issue slots from the warps that compute.
 __device__ __forceinline__ bool stk_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  const long long t0 = clock64(), lim = wait_limit();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > lim) {
       set_error(kErrWaitMbarrier);
       *abort = 1;
       return false;
@@ -247,20 +247,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     }
   };
   auto grid_wait = [&]() -> bool {
-    if (ctid == 0 && *abort == 0) {
-      const long long t0 = clock64();
-      while (true) {
-        unsigned int v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.gbar) : "memory");
-        if (v >= nbar * (unsigned int)G) break;
-        if (*(volatile uint32_t *)&g_dvssq_error != err0 || clock64() - t0 > kWaitLimitCycles) {
-          set_error(kErrWaitGrid);
-          *abort = 1;
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
+    if (ctid == 0 && *abort == 0 && !counter_wait(p.gbar, nbar * (unsigned int)G, err0))
+      *abort = 1;
     // one thread decides, so that every consumer warp takes the same branches
     if (ctid == 0) *s_live = *abort == 0;
     stk_consumer_sync();

@@ -18,7 +18,9 @@ namespace dvssq {
 static __device__ __align__(256) unsigned char g_static_scratch[DVSSQ_STATIC_SCRATCH_BYTES];
 
 // Device address of g_static_scratch on the current device, looked up once
-// per device with that device current.
+// per device with that device current and kept for the life of the process
+// (the library's other per-device set-up is kept the same way, so neither
+// survives a cudaDeviceReset).
 static cudaError_t static_scratch_ptr(void **out) {
   static std::mutex mu;
   static std::vector<void *> ptrs;
@@ -54,13 +56,17 @@ extern "C" dvssq_status dvssq_linear_forward_static(const dvssq_shape *shape,
                    "scratch of " + std::to_string((size_t)DVSSQ_STATIC_SCRATCH_BYTES) + " bytes");
     return DVSSQ_ERR_WORKSPACE;
   }
+  // the device check comes first: an unsupported device reports
+  // DVSSQ_ERR_DEVICE, not a failed symbol lookup
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
   void *scratch = nullptr;
   cudaError_t e = static_scratch_ptr(&scratch);
   if (e != cudaSuccess) {
     set_last_error(cudaGetErrorString(e));
     return DVSSQ_ERR_CUDA;
   }
-  // every other argument is validated here, on the host, before any launch
+  // dvssq_linear_forward validates the remaining arguments on the host
+  // before any launch
   return dvssq_linear_forward(shape, w, x, T, bias, y, y_dtype, DVSSQ_PATH_DECODE, scratch,
                               (size_t)DVSSQ_STATIC_SCRATCH_BYTES, stream);
 }

@@ -138,16 +138,38 @@ def test_encode_zero_rows_and_wide_exponent_spread(dv):
     Wn = synth.weight(M, K, seed=9).float()
     Wn[3] = 0.0                                         # all-zero row: s4 = s8 = 0
     Wn[7, 0] = 1.0
-    Wn[7, 1] = 2.0 ** -60                               # block not exactly summable
+    Wn[7, 1] = 2.0 ** -60                               # fp64 butterfly would round
+    Wn[20, 300] = 2.0 ** 40                             # a second chunk and block
+    Wn[20, 301] = -(2.0 ** -30)
+    Wn[20, 302] = 2.0 ** -120                           # BF16 subnormal-adjacent tail
+    Wn[40, 256:512] = 0.0
+    Wn[40, 260] = 3.0 * 2.0 ** -133                     # BF16 subnormals only
+    Wn[40, 261] = -(2.0 ** -130)
     W = Wn.to(torch.bfloat16)
     act = synth.act_scale(K, seed=2)
     enc = O.encode(f64(W), act.numpy(), 256, 0, with_svd=False)
-    shape, packed, info, _ = gpu_encode(dv, W, act, 256, 0)
-    assert info["inexact_rotation_blocks"] == enc["inexact_blocks"] >= 1
-    # rows with exactly summable blocks still match bit for bit
-    keep = [i for i in range(M) if i != 7]
-    assert np.array_equal(packed.q4.cpu().numpy()[keep], enc["q4"][keep])
+    assert enc["inexact_blocks"] >= 2
+    shape, packed, info, R = gpu_encode(dv, W, act, 256, 0, resid=True)
+    assert info["inexact_rotation_blocks"] == enc["inexact_blocks"]
+    # every row, the flagged ones included, bit for bit (codes, scales, salient
+    # set, residual)
+    check_codes(shape, packed, enc, R)
     assert np.all(packed.q4.cpu().numpy()[3] == 0) and bits16(packed.s8)[3] == 0
+
+
+@pytest.mark.parametrize("seed", [0, 4])
+def test_encode_near_ties_bit_exact_and_valid(dv, seed):
+    # exact ties across 16-row chunk boundaries, split by fp64 rounding: the
+    # GPU's salient set equals the oracle's (same summation tree) and is a
+    # valid top-n_sal set of the exact rational scores
+    import exact_topk as X
+    W, n_sal = X.near_tie_weight(seed)
+    act = torch.ones(W.shape[1], dtype=torch.float32)
+    enc = O.encode(f64(W), act.numpy(), 256, 0, n_sal=n_sal, with_svd=False)
+    shape, packed, info, R = gpu_encode(dv, W, act, 256, 0, n_sal, resid=True)
+    check_codes(shape, packed, enc, R)
+    got = packed.sal_idx[:n_sal].cpu().numpy()
+    X.check_selection_valid(enc["W_rot"], act.numpy(), got, n_sal)
 
 
 # ---------------------------------------------------------------- forward ---

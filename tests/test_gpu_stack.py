@@ -149,3 +149,49 @@ def test_stack_rejects_bad_layers(dv):
         dv.dvssq_mlp_stack_workspace_size(bad)
     with pytest.raises(dv.DvssqError):
         dv.dvssq_mlp_stack_workspace_size([])
+
+
+def _full_block(dv, l, r, base=7):
+    """One Spark-shaped block (hidden 2560, intermediate 10240, rank r), encoded
+    by the oracle and by the GPU (codes checked bit for bit); stand-in BF16
+    factors U, V shared by both sides."""
+    H, I = 2560, 10240
+    mats, encs = [], []
+    for which, (M, K) in enumerate(((I, H), (I, H), (H, I))):
+        seed = synth.layer_seed(base, l, which)
+        W = synth.weight(M, K, seed, n_outlier_cols=max(1, K // 1000), outlier_scale=15.0)
+        act = synth.act_scale(K, seed)
+        U, V = synth.lowrank_factors(M, K, r, seed=seed + 17)
+        enc = O.encode(f64(W), act.numpy(), 256, r, with_svd=False)
+        enc["U"], enc["V"] = f64(U), f64(V)
+        shape, packed, _, _ = gpu_encode(dv, W, act, 256, r, U=U.cuda().contiguous(),
+                                         V=V.cuda().contiguous())
+        check_codes(shape, packed, enc)
+        mats.append((shape, packed))
+        encs.append(enc)
+    return tuple(mats), encs
+
+
+def test_stack_full_spark_shapes_teacher_forced_oracle(dv):
+    # Each block of a two-layer Spark stack (rank 16, then 24) runs as a
+    # one-layer stack fed the ORACLE's input for that block, and its BF16
+    # output is held to the oracle's block (reading R10: BF16 after gate, up,
+    # the gated product and down).  The two computations round at the same
+    # four points; their pre-rounding values differ by the GPU's FP32 error,
+    # so a fraction of the BF16 values sit one step apart.
+    x = f64(synth.activations(1, 2560, seed=21, n_outlier=13, outlier_scale=25.0))
+    for l, r in enumerate((16, 24)):
+        mats, (eg, eu, ed) = _full_block(dv, l, r)
+        ref = O.mlp_block(eg, eu, ed, x)
+        xin = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda()
+        y = dv.MlpStack([mats]).forward(xin)
+        torch.cuda.synchronize()
+        assert dv.dvssq_device_error(clear=True) == 0
+        got = f64(y)[None, :]
+        rl = rel_l2(got, ref)
+        mx = float(np.abs(got - ref).max() / np.abs(ref).max())
+        eq = float(np.mean(got == ref))
+        print(f"block {l} r={r}: rel-L2 {rl:.3e}, max-abs/max|y| {mx:.3e}, equal {eq:.4f}")
+        assert rl <= 3e-3 and mx <= 1e-2, (rl, mx)
+        assert eq >= 0.80, eq
+        x = ref[0]                                       # teacher forcing: the oracle's output
