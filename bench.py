@@ -709,6 +709,50 @@ class MaterializeLeg:
                 "52 MB BF16 output is rewritten every step"}
 
 
+class LowrankLeg:
+    """dvssq_lowrank of the Spark down_proj residual (2560 x 10240 FP32, rank
+    16, 4 power iterations): the truncated SVD of the encoder on the GPU.
+    Unit: GB/s of residual bytes read by the products with R (each launch of
+    lr_mul reads R once: 2 (iters + 1) + 1 = 11 reads per call)."""
+
+    name = "spark_down_proj_2560x10240_lowrank_r16_q4"
+    iters = 4
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv = dv
+        wl = synth.WORKLOADS["spark_down"]
+        self.M, self.K, self.r = wl.M, wl.K, 16
+        shape = dv.Shape.make(wl.M, wl.K, wl.block, 0)
+        packed = dv.PackedWeights.empty(shape, device)
+        self.R = torch.empty((wl.M, wl.K), dtype=torch.float32, device=device)
+        dv.dvssq_encode(shape, wl.weight(seed_offset=rank_id).to(device),
+                        wl.act_scale(seed_offset=rank_id).to(device), packed, resid=self.R)
+        self.U = torch.empty((wl.M, 16), dtype=torch.bfloat16, device=device)
+        self.V = torch.empty((16, wl.K), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(dv.dvssq_lowrank_workspace_size(wl.M, wl.K, 16), dtype=torch.uint8,
+                              device=device)
+
+    graph_slots = 1
+
+    def step_slot(self, i):
+        self.dv.dvssq_lowrank(self.R, 16, iters=self.iters, seed=5, U=self.U, V=self.V,
+                              workspace=self.ws)
+
+    def step(self):
+        self.step_slot(0)
+
+    def bytes_per_step(self):
+        return (2 * (self.iters + 1) + 1) * self.M * self.K * 4
+
+    def kernel_work(self, name):
+        return self.M * self.K * 4 if name == "lr_mul" else None
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "K": self.K, "rank": 16,
+                "iters": self.iters, "oversampling": 16,
+                "l2": "the 105 MB FP32 residual is read 11 times per call; partly from L2"}
+
+
 # Legs of the metric timed in the default single-GPU run besides the headline:
 # (name, constructor).  Each is built, timed and freed in turn.
 def leg_specs():
@@ -721,6 +765,7 @@ def leg_specs():
         ("prefill", PrefillStep),
         ("bulk_encode", BulkEncodeStep),
         ("materialize", MaterializeLeg),
+        ("lowrank", LowrankLeg),
         ("minicpm_k_T1", fwd("minicpm_k", (1,), 192)),
         ("minicpm_k_T8", fwd("minicpm_k", (8,), 192)),
         ("minicpm_k_T64", fwd("minicpm_k", (64,), 192)),

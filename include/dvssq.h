@@ -250,6 +250,36 @@ DVSSQ_API dvssq_status dvssq_linear_forward(const dvssq_shape *shape, const dvss
 DVSSQ_API dvssq_status dvssq_materialize(const dvssq_shape *shape, const dvssq_weights *w,
                                          void *W_eff, void *stream);
 
+/* Bytes of workspace dvssq_lowrank needs (host only). */
+DVSSQ_API dvssq_status dvssq_lowrank_workspace_size(int32_t M, int32_t K, int32_t rank,
+                                                    size_t *bytes);
+
+/* Rank-r factors of the INT4 residual on the GPU (Spark card, Tier C,
+ * "Truncated SVD Low-Rank Residual Compensation": R ~= U_r S_r V_r^T;
+ * MiniCPM card, Mathematical Foundations §2: A = U_r sqrt(S_r),
+ * B = sqrt(S_r) V_r^T), by randomised subspace iteration: a Gaussian test
+ * matrix of p = rank + 16 columns (a counter-based generator keyed by
+ * `seed`), `iters` power iterations R R^T with CholeskyQR
+ * re-orthonormalisation, then the exact eigen-decomposition (Jacobi, fp64)
+ * of the p x p projected Gram matrix.  The truncation error approaches the
+ * Eckart-Young optimum sum_{k>r} sigma_k^2 as `iters` grows; the products
+ * with R run in FP32, the small problems in fp64, every reduction in a fixed
+ * order (deterministic for a given seed).
+ *   R      fp32 [M][K] (device): the residual dvssq_encode writes (`resid`)
+ *   rank   8 <= rank <= 64, rank % 8 == 0, rank + 16 <= min(M, K)
+ *   iters  power iterations, 0..64 (4 is a good default)
+ *   U      bf16 [M][rank] (device), written: A = U_r sqrt(S_r)
+ *   V      bf16 [rank][K] (device), written: B = sqrt(S_r) V_r^T
+ *   sigma  fp32 [rank] (device) or NULL: the estimated singular values
+ *   workspace  device scratch of dvssq_lowrank_workspace_size bytes
+ * Stream-ordered and asynchronous.  U and V are the inputs U and V of
+ * dvssq_weights for the forward.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_lowrank(const float *R, int32_t M, int32_t K, int32_t rank,
+                                     int32_t iters, uint64_t seed, uint16_t *U, uint16_t *V,
+                                     float *sigma, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
 /* Allocation-free decode forward.  The paper has no counterpart: this entry
  * exists for callers that cannot obtain device memory for a workspace --
  * for example a host program that links only this library and has no device

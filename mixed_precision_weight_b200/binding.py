@@ -26,7 +26,7 @@ __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
     "dvssq_fwht", "dvssq_gelu_mul", "dvssq_encode_workspace_size", "dvssq_encode",
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
-    "dvssq_materialize", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
+    "dvssq_materialize", "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
     "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
@@ -52,7 +52,7 @@ EXPORTED_SYMBOLS = (
     "dvssq_gelu_mul",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
     "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_materialize",
-    "dvssq_device_error", "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
+    "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_device_error", "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
@@ -106,6 +106,11 @@ _sig = {
     "dvssq_linear_forward_static": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights),
                                                    _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "dvssq_materialize": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights), _P, _P]),
+    "dvssq_lowrank_workspace_size": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                    ctypes.POINTER(ctypes.c_size_t)]),
+    "dvssq_lowrank": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.c_uint64, _P, _P, _P, _P,
+                                     ctypes.c_size_t, _P]),
     "dvssq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "dvssq_mlp_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32,
                                                       ctypes.POINTER(ctypes.c_size_t)]),
@@ -289,6 +294,34 @@ def dvssq_linear_forward_static(shape: Shape, w: PackedWeights, x: torch.Tensor,
 
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def dvssq_lowrank_workspace_size(M: int, K: int, rank: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.dvssq_lowrank_workspace_size(M, K, rank, ctypes.byref(n)),
+           "dvssq_lowrank_workspace_size")
+    return n.value
+
+
+def dvssq_lowrank(R: torch.Tensor, rank: int, iters: int = 4, seed: int = 0,
+                  U: torch.Tensor | None = None, V: torch.Tensor | None = None,
+                  sigma: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  stream=None):
+    """BF16 rank-r factors (U [M][r], V [r][K]) of the FP32 residual R [M][K]."""
+    if R.dtype != torch.float32 or R.dim() != 2:
+        raise TypeError("R must be a float32 matrix")
+    M, K = R.shape
+    if U is None:
+        U = torch.empty((M, rank), dtype=torch.bfloat16, device=R.device)
+    if V is None:
+        V = torch.empty((rank, K), dtype=torch.bfloat16, device=R.device)
+    if workspace is None:
+        workspace = torch.empty(dvssq_lowrank_workspace_size(M, K, rank), dtype=torch.uint8,
+                                device=R.device)
+    _check(lib.dvssq_lowrank(_ptr(R), M, K, rank, iters, seed & (2 ** 64 - 1), _ptr(U), _ptr(V),
+                             _ptr(sigma), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dvssq_lowrank")
+    return U, V
 
 
 def dvssq_materialize(shape: Shape, w: PackedWeights, out: torch.Tensor | None = None,

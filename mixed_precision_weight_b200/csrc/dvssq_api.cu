@@ -82,6 +82,7 @@ dvssq_status ensure_device() {
   if ((e = prepare_forward_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_stack_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_materialize_kernels()) != cudaSuccess) return cuda_fail(e);
+  if ((e = prepare_lowrank_kernels()) != cudaSuccess) return cuda_fail(e);
   ready[dev] = 1;
   return DVSSQ_OK;
 }
@@ -309,6 +310,42 @@ dvssq_status dvssq_materialize(const dvssq_shape *shape, const dvssq_weights *w,
   a.U = w->U; a.V = w->V;
   a.W = static_cast<uint16_t *>(W_eff);
   const cudaError_t e = launch_materialize(a, static_cast<cudaStream_t>(stream), launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
+static dvssq_status lowrank_shape(int32_t M, int32_t K, int32_t rank) {
+  if (M < 1 || K < 1 || M > (1 << 24) || K > 65536) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  if (rank < 8 || rank > 64 || rank % 8 != 0) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  if (rank + 16 > M || rank + 16 > K) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  return DVSSQ_OK;
+}
+
+dvssq_status dvssq_lowrank_workspace_size(int32_t M, int32_t K, int32_t rank, size_t *bytes) {
+  if (bytes == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  const dvssq_status s = lowrank_shape(M, K, rank);
+  if (s != DVSSQ_OK) return s;
+  *bytes = lowrank_workspace_bytes(M, K, rank);
+  return DVSSQ_OK;
+}
+
+dvssq_status dvssq_lowrank(const float *R, int32_t M, int32_t K, int32_t rank, int32_t iters,
+                           uint64_t seed, uint16_t *U, uint16_t *V, float *sigma,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+  dvssq_status s = lowrank_shape(M, K, rank);
+  if (s != DVSSQ_OK) return s;
+  if (R == nullptr || U == nullptr || V == nullptr || workspace == nullptr || iters < 0 ||
+      iters > 64)
+    return DVSSQ_ERR_INVALID_ARG;
+  const void *bufs[] = {R, U, V, sigma};
+  for (const void *b : bufs)
+    if (b != nullptr && !aligned16(b)) return DVSSQ_ERR_MISALIGNED;
+  if (!aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
+  if (workspace_bytes < lowrank_workspace_bytes(M, K, rank)) return DVSSQ_ERR_WORKSPACE;
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
+  LowrankArgs a;
+  a.R = R; a.M = M; a.K = K; a.rank = rank; a.iters = iters; a.seed = seed;
+  a.U = U; a.V = V; a.sigma = sigma; a.workspace = workspace;
+  const cudaError_t e = launch_lowrank(a, static_cast<cudaStream_t>(stream), launcher());
   return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
 }
 

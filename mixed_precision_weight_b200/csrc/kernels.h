@@ -196,6 +196,19 @@ struct MaterializeArgs {
 cudaError_t launch_materialize(const MaterializeArgs &a, cudaStream_t st, Launcher &L);
 cudaError_t prepare_materialize_kernels();
 
+// ---------------------------------------------------------------- lowrank -
+struct LowrankArgs {
+  const float *R;
+  int M, K, rank, iters;
+  uint64_t seed;
+  uint16_t *U, *V;
+  float *sigma;
+  void *workspace;
+};
+size_t lowrank_workspace_bytes(int M, int K, int rank);
+cudaError_t launch_lowrank(const LowrankArgs &a, cudaStream_t st, Launcher &L);
+cudaError_t prepare_lowrank_kernels();
+
 // Tensor-map encoder from the driver (resolved once through the runtime).
 CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,

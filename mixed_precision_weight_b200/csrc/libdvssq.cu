@@ -9,5 +9,6 @@
 #include "prefill.cu"
 #include "stack.cu"
 #include "materialize.cu"
+#include "lowrank.cu"
 #include "selftest.cu"
 #include "static_scratch.cu"
