@@ -753,6 +753,57 @@ class LowrankLeg:
                 "l2": "the 105 MB FP32 residual is read 11 times per call; partly from L2"}
 
 
+class BssAttentionLeg:
+    """KV-BSS decode attention of the Spark attention shape: 16 query heads, 4
+    KV heads, head_dim 256, one query token per sequence over a 32768-token
+    BF16 KV cache, batch 4 (K + V = 537 MB > L2).  Seeded N(0, 1) tensors,
+    so the truncation drops few keys and every V row is read.
+    Unit: GB/s of K and V bytes."""
+
+    name = "spark_attention_kv_bss_B4_Hq16_Hkv4_d256_L32768"
+
+    def __init__(self, dv, synth, torch, rank_id, device):
+        self.dv = dv
+        self.B, self.Hq, self.Hkv, self.d, self.L = 4, 16, 4, 256, 32768
+        gen = torch.Generator(device=device)
+        gen.manual_seed(1234 + rank_id)
+        mk = lambda *s: torch.randn(s, generator=gen, device=device).to(torch.bfloat16)
+        self.q = mk(self.B, self.Hq, self.d)
+        self.k = mk(self.B, self.Hkv, self.L, self.d)
+        self.v = mk(self.B, self.Hkv, self.L, self.d)
+        self.out = torch.empty((self.B, self.Hq, self.d), dtype=torch.float32, device=device)
+        shape = dv.AttnShape(self.B, self.Hq, self.Hkv, self.d, self.L, 1.10, 12.0)
+        self.ws = torch.empty(dv.dvssq_bss_attention_workspace_size(shape), dtype=torch.uint8,
+                              device=device)
+
+    graph_slots = 1
+
+    def step_slot(self, i):
+        self.dv.dvssq_bss_attention(self.q, self.k, self.v, out=self.out, workspace=self.ws)
+
+    def step(self):
+        self.step_slot(0)
+
+    def kv_bytes(self):
+        return self.B * self.Hkv * self.L * self.d * 2
+
+    def bytes_per_step(self):
+        return 2 * self.kv_bytes()
+
+    def kernel_work(self, name):
+        logits = self.B * self.Hq * self.L * 4
+        if name == "bss_logits":
+            return self.kv_bytes() + logits
+        if name == "bss_pv":
+            return self.kv_bytes() + logits
+        return None
+
+    def config(self):
+        return {"workload": self.name, "batch": self.B, "q_heads": self.Hq,
+                "kv_heads": self.Hkv, "head_dim": self.d, "ctx": self.L, "tau": 1.10,
+                "haze": 12.0, "l2": "537 MB of K and V per step > 126 MB L2"}
+
+
 # Legs of the metric timed in the default single-GPU run besides the headline:
 # (name, constructor).  Each is built, timed and freed in turn.
 def leg_specs():
@@ -766,6 +817,7 @@ def leg_specs():
         ("bulk_encode", BulkEncodeStep),
         ("materialize", MaterializeLeg),
         ("lowrank", LowrankLeg),
+        ("bss_attention", BssAttentionLeg),
         ("minicpm_k_T1", fwd("minicpm_k", (1,), 192)),
         ("minicpm_k_T8", fwd("minicpm_k", (8,), 192)),
         ("minicpm_k_T64", fwd("minicpm_k", (64,), 192)),

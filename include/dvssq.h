@@ -280,6 +280,46 @@ DVSSQ_API dvssq_status dvssq_lowrank(const float *R, int32_t M, int32_t K, int32
                                      float *sigma, void *workspace, size_t workspace_bytes,
                                      void *stream);
 
+/* KV-BSS attention for decode: one query token per sequence over its whole
+ * context ("Spark-X2.5-4B-Hadamard-GSQ", "2. KV-BSS: Key-Value Binding
+ * Softmax Sharpening": focus factor scaling and attention haze truncation).
+ * Per query head h (KV head h / (q_heads / kv_heads), grouped-query):
+ *   s_l = (q_h . k_l) tau / sqrt(head_dim),  m = max_l s_l,
+ *   s_l -> -inf where s_l < m - haze  (haze <= 0 disables the truncation),
+ *   out_h = softmax(s) . V
+ * Logits, the mask decision, the exponentials and the sums are FP32.
+ *   batch, q_heads, kv_heads  q_heads % kv_heads == 0; the group size
+ *       q_heads / kv_heads is 2, 4 or 8 for head_dim 128 and 2 or 4 for 256
+ *   head_dim  128 or 256;  ctx  context length L >= 1
+ *   tau, haze the focus factor and the truncation depth (the pages: 1.10, 12)
+ */
+typedef struct {
+  int32_t batch;
+  int32_t q_heads;
+  int32_t kv_heads;
+  int32_t head_dim;
+  int32_t ctx;
+  float tau;
+  float haze;
+} dvssq_attn_shape;
+
+/* Bytes of workspace dvssq_bss_attention needs (host only). */
+DVSSQ_API dvssq_status dvssq_bss_attention_workspace_size(const dvssq_attn_shape *shape,
+                                                          size_t *bytes);
+
+/*   q    bf16 [batch][q_heads][head_dim] (device)
+ *   k, v bf16 [batch][kv_heads][ctx][head_dim] (device; the KV cache)
+ *   out  fp32 [batch][q_heads][head_dim] (device), written
+ *   workspace  device scratch of dvssq_bss_attention_workspace_size bytes
+ * Three stream-ordered launches (logits and per-chunk maxima; masked
+ * weights and partial P V, skipping V rows masked for every head of a
+ * group; the fixed-order merge): results are deterministic.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, DEVICE, CUDA. */
+DVSSQ_API dvssq_status dvssq_bss_attention(const dvssq_attn_shape *shape, const void *q,
+                                           const void *k, const void *v, float *out,
+                                           void *workspace, size_t workspace_bytes,
+                                           void *stream);
+
 /* Allocation-free decode forward.  The paper has no counterpart: this entry
  * exists for callers that cannot obtain device memory for a workspace --
  * for example a host program that links only this library and has no device

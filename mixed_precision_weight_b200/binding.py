@@ -26,7 +26,8 @@ __all__ = [
     "DvssqError", "Shape", "PackedWeights", "DvssqLinear", "lib", "library_path",
     "dvssq_fwht", "dvssq_gelu_mul", "dvssq_encode_workspace_size", "dvssq_encode",
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
-    "dvssq_materialize", "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
+    "dvssq_materialize", "dvssq_lowrank_workspace_size", "dvssq_lowrank", "AttnShape",
+    "dvssq_bss_attention_workspace_size", "dvssq_bss_attention", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
     "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
@@ -52,7 +53,9 @@ EXPORTED_SYMBOLS = (
     "dvssq_gelu_mul",
     "dvssq_encode_workspace_size", "dvssq_encode", "dvssq_forward_workspace_size",
     "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_materialize",
-    "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_device_error", "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
+    "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_bss_attention_workspace_size",
+    "dvssq_bss_attention", "dvssq_device_error", "dvssq_mlp_stack_workspace_size",
+    "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
@@ -82,6 +85,12 @@ class _MlpLayer(ctypes.Structure):
     _fields_ = [("shape", Shape * 3), ("w", _Weights * 3)]
 
 
+class AttnShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("q_heads", ctypes.c_int32),
+                ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ctx", ctypes.c_int32), ("tau", ctypes.c_float), ("haze", ctypes.c_float)]
+
+
 class _EncodeInfo(ctypes.Structure):
     _fields_ = [("inexact_rotation_blocks", ctypes.c_int64),
                 ("fp16_unsafe_scales", ctypes.c_int64),
@@ -106,6 +115,10 @@ _sig = {
     "dvssq_linear_forward_static": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights),
                                                    _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "dvssq_materialize": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.POINTER(_Weights), _P, _P]),
+    "dvssq_bss_attention_workspace_size": (ctypes.c_int, [ctypes.POINTER(AttnShape),
+                                                          ctypes.POINTER(ctypes.c_size_t)]),
+    "dvssq_bss_attention": (ctypes.c_int, [ctypes.POINTER(AttnShape), _P, _P, _P, _P, _P,
+                                           ctypes.c_size_t, _P]),
     "dvssq_lowrank_workspace_size": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                     ctypes.POINTER(ctypes.c_size_t)]),
     "dvssq_lowrank": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -294,6 +307,31 @@ def dvssq_linear_forward_static(shape: Shape, w: PackedWeights, x: torch.Tensor,
 
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
+
+
+def dvssq_bss_attention_workspace_size(shape: AttnShape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.dvssq_bss_attention_workspace_size(ctypes.byref(shape), ctypes.byref(n)),
+           "dvssq_bss_attention_workspace_size")
+    return n.value
+
+
+def dvssq_bss_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float = 1.10,
+                        haze: float = 12.0, out: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, stream=None):
+    """KV-BSS decode attention: q [B][Hq][d], k/v [B][Hkv][L][d] (BF16) -> FP32 [B][Hq][d]."""
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    shape = AttnShape(B, Hq, Hkv, d, L, tau, haze)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(dvssq_bss_attention_workspace_size(shape), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib.dvssq_bss_attention(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dvssq_bss_attention")
+    return out
 
 
 def dvssq_lowrank_workspace_size(M: int, K: int, rank: int) -> int:

@@ -349,6 +349,56 @@ dvssq_status dvssq_lowrank(const float *R, int32_t M, int32_t K, int32_t rank, i
   return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
 }
 
+static dvssq_status bss_shape(const dvssq_attn_shape *s) {
+  if (s == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->q_heads < 1 || s->kv_heads < 1 || s->ctx < 1)
+    return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  if (s->q_heads % s->kv_heads != 0) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  const int G = s->q_heads / s->kv_heads;
+  const bool ok = (s->head_dim == 256 && (G == 2 || G == 4)) ||
+                  (s->head_dim == 128 && (G == 2 || G == 4 || G == 8));
+  if (!ok) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)s->batch * s->q_heads > 65535 || s->ctx > (1 << 24))
+    return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  if (!(s->tau > 0.f) || s->haze != s->haze) return DVSSQ_ERR_INVALID_ARG;
+  return DVSSQ_OK;
+}
+
+dvssq_status dvssq_bss_attention_workspace_size(const dvssq_attn_shape *shape, size_t *bytes) {
+  if (bytes == nullptr) return DVSSQ_ERR_INVALID_ARG;
+  const dvssq_status s = bss_shape(shape);
+  if (s != DVSSQ_OK) return s;
+  *bytes = bss_workspace_bytes(shape->batch, shape->q_heads, shape->ctx, shape->head_dim);
+  return DVSSQ_OK;
+}
+
+dvssq_status dvssq_bss_attention(const dvssq_attn_shape *shape, const void *q, const void *k,
+                                 const void *v, float *out, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+  dvssq_status s = bss_shape(shape);
+  if (s != DVSSQ_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || workspace == nullptr)
+    return DVSSQ_ERR_INVALID_ARG;
+  const void *bufs[] = {q, k, v, out};
+  for (const void *b : bufs)
+    if (!aligned16(b)) return DVSSQ_ERR_MISALIGNED;
+  if (!aligned256(workspace)) return DVSSQ_ERR_MISALIGNED;
+  if (workspace_bytes < bss_workspace_bytes(shape->batch, shape->q_heads, shape->ctx,
+                                            shape->head_dim))
+    return DVSSQ_ERR_WORKSPACE;
+  if ((s = ensure_device()) != DVSSQ_OK) return s;
+  BssArgs a;
+  a.q = static_cast<const uint16_t *>(q);
+  a.k = static_cast<const uint16_t *>(k);
+  a.v = static_cast<const uint16_t *>(v);
+  a.out = out;
+  a.B = shape->batch; a.Hq = shape->q_heads; a.Hkv = shape->kv_heads; a.L = shape->ctx;
+  a.D = shape->head_dim; a.tau = shape->tau; a.haze = shape->haze;
+  a.workspace = workspace;
+  const cudaError_t e = launch_bss_attention(a, static_cast<cudaStream_t>(stream), launcher());
+  return e == cudaSuccess ? DVSSQ_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------- MLP stack ---
 namespace {
 // Host-side checks of a stack and its flattening into matrix descriptors.

@@ -209,6 +209,17 @@ size_t lowrank_workspace_bytes(int M, int K, int rank);
 cudaError_t launch_lowrank(const LowrankArgs &a, cudaStream_t st, Launcher &L);
 cudaError_t prepare_lowrank_kernels();
 
+// -------------------------------------------------------- KV-BSS attention -
+struct BssArgs {
+  const uint16_t *q, *k, *v;
+  float *out;
+  int B, Hq, Hkv, L, D;
+  float tau, haze;
+  void *workspace;
+};
+size_t bss_workspace_bytes(int B, int Hq, int L, int D);
+cudaError_t launch_bss_attention(const BssArgs &a, cudaStream_t st, Launcher &L);
+
 // Tensor-map encoder from the driver (resolved once through the runtime).
 CUresult encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                         uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,

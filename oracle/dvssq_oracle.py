@@ -54,6 +54,9 @@ R10 MLP block of the Spark shape ("Myric/Spark-X2.5-4B-GGUF", "The model":
     ffn_gate / ffn_up / ffn_down): x_next = down(GELU(gate x) * up x) with
     the exact erf GELU, no norm or residual, and hidden states rounded to
     BF16 after every projection and after the gated product.
+R11 KV-BSS attention ([Spark] "2. KV-BSS"): logits q.k tau / sqrt(d), tau =
+    1.10; a logit more than `haze` = 12 nats below the query's largest logit
+    (over the keys it attends) is masked to -inf before the softmax.
 """
 from __future__ import annotations
 
@@ -479,3 +482,46 @@ def mlp_block(enc_gate: dict, enc_up: dict, enc_down: dict, x: np.ndarray) -> np
     u = rn_bf16(forward(enc_up, x))
     h = gelu_mul(g, u)
     return rn_bf16(forward(enc_down, h))
+
+
+# ---------------------------------------------------------------------------
+# KV-BSS attention ([Spark] "2. KV-BSS: Key-Value Binding Softmax
+# Sharpening"; forum post "Architectural Proposal: KV-BSS", implementation
+# notes): focus factor and attention haze truncation
+# ---------------------------------------------------------------------------
+
+
+def bss_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, tau: float = 1.10,
+                  haze: float = 12.0) -> np.ndarray:
+    """Attention of the query tokens over their whole context with KV-BSS.
+
+    q [B][Hq][d], k and v [B][Hkv][L][d] (BF16 values as fp64), Hq a multiple
+    of Hkv (grouped-query attention: query head h reads KV head h // (Hq/Hkv)).
+    Per query head, in fp64:
+      s_l = (q . k_l) * tau / sqrt(d)           (focus factor scaling)
+      s_l -> -inf where s_l < max_l s_l - haze  (attention haze truncation;
+                                                 haze <= 0 or inf disables it)
+      p = softmax(s),  out = sum_l p_l v_l.
+    Reading R11: the threshold is taken on the scaled logits over the keys the
+    query attends (the whole context here), as the implementation notes apply
+    it to attn_weights before the softmax.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    grp = Hq // Hkv
+    out = np.empty((B, Hq, d))
+    scale = tau / math.sqrt(d)
+    for b in range(B):
+        for h in range(Hq):
+            kh = h // grp
+            s = (k[b, kh] @ q[b, h]) * scale
+            m = s.max()
+            keep = np.ones_like(s, dtype=bool)
+            if 0 < haze < np.inf:
+                keep = s >= m - haze
+            p = np.where(keep, np.exp(s - m), 0.0)
+            out[b, h] = (p @ v[b, kh]) / p.sum()
+    return out

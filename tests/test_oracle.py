@@ -627,3 +627,63 @@ def test_selection_valid_against_exact_scores_near_ties(seed):
     sal_seq = O.select_salient(np.sqrt(seq), n_sal)
     X.check_selection_valid(Wr, act, sal_seq, n_sal)
     assert not np.array_equal(sal, sal_seq)
+
+
+# ------------------------------------------------------------- R11 KV-BSS ---
+
+def test_bss_reduces_to_plain_softmax_attention():
+    # tau = 1 and the haze truncation off: standard scaled dot-product
+    # attention, checked against scipy's softmax
+    from scipy.special import softmax
+    rng = np.random.default_rng(8)
+    B, Hq, Hkv, L, d = 2, 4, 2, 37, 16
+    q, k, v = (rng.standard_normal(s) for s in ((B, Hq, d), (B, Hkv, L, d), (B, Hkv, L, d)))
+    out = O.bss_attention(q, k, v, tau=1.0, haze=0.0)
+    for b in range(B):
+        for h in range(Hq):
+            p = softmax(k[b, h // 2] @ q[b, h] / 4.0)
+            assert np.allclose(out[b, h], p @ v[b, h // 2], rtol=0, atol=1e-13)
+
+
+def test_bss_focus_factor_scales_the_logits():
+    # tau multiplies the logits: tau = 2 equals tau = 1 on a doubled query
+    rng = np.random.default_rng(9)
+    q, k, v = rng.standard_normal((1, 2, 8)), rng.standard_normal((1, 1, 20, 8)), \
+        rng.standard_normal((1, 1, 20, 8))
+    assert np.allclose(O.bss_attention(q, k, v, tau=2.0, haze=0.0),
+                       O.bss_attention(2.0 * q, k, v, tau=1.0, haze=0.0), atol=1e-14)
+
+
+def test_bss_haze_truncation_planted():
+    # logits (after scaling) planted at 0, -5, -11.9, -12.1 and -30 nats below
+    # the maximum: the last two are masked, the rest keep exp(-gap) weights;
+    # exp(-12) = 6.14e-6 (the pages' figure)
+    assert abs(math.exp(-12.0) - 6.14e-6) < 0.01e-6
+    d = 4
+    gaps = np.array([0.0, 5.0, 11.9, 12.1, 30.0])
+    q = np.zeros((1, 1, d)); q[0, 0, 0] = 1.0
+    tau = 1.10
+    k = np.zeros((1, 1, 5, d))
+    k[0, 0, :, 0] = (20.0 - gaps) * math.sqrt(d) / tau        # logits 20 - gap
+    v = np.zeros((1, 1, 5, d)); v[0, 0, :, 1] = np.arange(5) + 1.0
+    out = O.bss_attention(q, k, v, tau=tau, haze=12.0)[0, 0]
+    w = np.exp(-gaps[:3])
+    assert abs(out[1] - (w @ (np.arange(3) + 1.0)) / w.sum()) < 1e-14
+    # without the truncation the two far keys count
+    full = O.bss_attention(q, k, v, tau=tau, haze=0.0)[0, 0]
+    w5 = np.exp(-gaps)
+    assert abs(full[1] - (w5 @ (np.arange(5) + 1.0)) / w5.sum()) < 1e-14
+    assert out[1] != full[1]
+
+
+def test_bss_single_dominant_binding_returns_its_value():
+    # one key 13 nats above every other: all others are truncated and the
+    # output is exactly that key's value
+    rng = np.random.default_rng(10)
+    d, L = 8, 50
+    q = rng.standard_normal((1, 1, d))
+    k = 0.01 * rng.standard_normal((1, 1, L, d))
+    k[0, 0, 17] = q[0, 0] * (13.5 * math.sqrt(d) / 1.10 / (q[0, 0] @ q[0, 0]))
+    v = rng.standard_normal((1, 1, L, d))
+    out = O.bss_attention(q, k, v)
+    assert np.array_equal(out[0, 0], v[0, 0, 17])
