@@ -344,83 +344,144 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     const int K = ph.K, nrows = ph.b - ph.a;
     // input vector and t: the G shares of each (matrix, k), NP parts per
     // pair summed in parallel, then the parts in order
-    for (int i = ctid; i < K / 8; i += kStkConsThreads)
-      reinterpret_cast<uint4 *>(xi)[i] = __ldcg(reinterpret_cast<const uint4 *>(ph.src) + i);
-    const int r0m = ph.m[0].r, npair = r0m + (ph.nm > 1 ? ph.m[1].r : 0);
-    const int NP = npair > 0 ? max(1, min(16, kStkConsThreads / npair)) : 1;
-    const int Gp = (G + NP - 1) / NP;
-    for (int tau = ctid; tau < npair * NP; tau += kStkConsThreads) {
-      const int q = tau / NP, j = tau - q * NP;
-      const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
-      const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * G;
-      const int c0 = j * Gp, c1 = min(G, c0 + Gp);
-      float s = 0.0f;
-      for (int i0 = c0; i0 < c1; i0 += 16) {
-        float v[16];
+    // the input vector, four 16-byte loads per thread in flight at once (its
+    // producers are other CTAs: the loads go to L2 after the grid barrier)
+    for (int i0 = ctid; i0 < K / 8; i0 += 4 * kStkConsThreads) {
+      uint4 xv[4];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = i0 + u < c1 ? __ldcg(src + i0 + u) : 0.0f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) s += v[u];
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kStkConsThreads;
+        if (i < K / 8) xv[u] = __ldcg(reinterpret_cast<const uint4 *>(ph.src) + i);
       }
-      tq[tau] = s;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kStkConsThreads;
+        if (i < K / 8) reinterpret_cast<uint4 *>(xi)[i] = xv[u];
+      }
+    }
+    // t = the sum of the G CTAs' shares of each (matrix, rank index) pair.
+    // A warp takes up to four pairs (q = cw + 15 i); its lanes read the
+    // shares at lane + 32 u (coalesced, every load in flight at once), add
+    // them in u order and then by a fixed shuffle tree: deterministic.
+    const int r0m = ph.m[0].r, npair = r0m + (ph.nm > 1 ? ph.m[1].r : 0);
+    {
+      constexpr int QW = (2 * kStkMaxRank + kStkCons - 1) / kStkCons;   // pairs per warp
+      constexpr int UW = 8;                                              // G <= 256
+      float v[QW][UW];
+#pragma unroll
+      for (int i = 0; i < QW; ++i) {
+        const int q = cw + kStkCons * i;
+        const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
+        const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * G;
+#pragma unroll
+        for (int u = 0; u < UW; ++u) {
+          const int j = lane + 32 * u;
+          v[i][u] = (q < npair && j < G) ? __ldcg(src + j) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < QW; ++i) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int u = 0; u < UW; ++u) sum += v[i][u];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const int q = cw + kStkCons * i;
+        if (lane == 0 && q < npair) {
+          const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
+          tv[mi * kStkMaxRank + k] = sum;
+        }
+      }
     }
     stk_cp_async_wait_all();             // this phase's prefetched s8 and salient indices
     stk_consumer_sync();
-    for (int q = ctid; q < npair; q += kStkConsThreads) {
-      float s = 0.0f;
-      for (int j = 0; j < NP; ++j) s += tq[q * NP + j];
-      const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
-      tv[mi * kStkMaxRank + k] = s;
-    }
 
-    // rotate x: BF16 in, int16 (unit/chunk layout) with one scale per 64 columns
+    // rotate x: BF16 in, int16 (unit/chunk layout) with one scale per 64
+    // columns.  One warp per Hadamard block: lane l holds the E = B/32
+    // consecutive columns [E l, E l + E); the butterflies inside a lane run
+    // in registers, the ones across lanes (index bits log2 E and up) by
+    // shuffles.  The block is read whole before its int16 form is written
+    // back in place (both stay inside the block).
     {
-      constexpr int P = B / 16;
+      constexpr int E = B / 32;                // columns per lane: 8 or 4
+      constexpr int LPG = 64 / E;              // lanes per 64-column group: 8 or 16
+      constexpr int LPU = 32 / E;              // lanes per 32-column unit: 4 or 8
       const int nblk = K / B;
-      const int grp = ctid / P, t = ctid % P;
       const float cb = B == 256 ? 0.0625f : 0.08838834764831845f;
-      if (grp < kStkFwhtGroups)
-        for (int kb0 = 0; kb0 < nblk; kb0 += kStkFwhtGroups) {
-          const int kb = kb0 + grp;
-          const bool in = kb < nblk;
-          const uint16_t *blk = xi + (size_t)(in ? kb : 0) * B;
-          float v[16];
+      for (int kb = cw; kb < nblk; kb += kStkCons) {
+        const uint16_t *blk = xi + (size_t)kb * B + E * lane;
+        float v[E];
+        if constexpr (E == 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(blk);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int a = 0; a < 16; ++a) v[a] = in ? bf16_bits_to_f32(blk[P * a + t]) : 0.0f;
-          fwht_group<B>(v, scr + grp * GroupScratch<B>::kElems, t);
-          float mx = 0.0f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v[j] *= cb;
-            mx = fmaxf(mx, fabsf(v[j]));
+          for (int i = 0; i < 4; ++i) {
+            v[2 * i] = bf16_bits_to_f32(ww[i] & 0xFFFFu);
+            v[2 * i + 1] = bf16_bits_to_f32(ww[i] >> 16);
           }
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));   // 64 columns = 4 threads
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
-          int q[16], sum = 0;
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2 *>(blk);
+          v[0] = bf16_bits_to_f32(w.x & 0xFFFFu);
+          v[1] = bf16_bits_to_f32(w.x >> 16);
+          v[2] = bf16_bits_to_f32(w.y & 0xFFFFu);
+          v[3] = bf16_bits_to_f32(w.y >> 16);
+        }
+        __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            q[j] = max(-32767, min(32767, __float2int_rn(v[j] * inv)));
-            sum += q[j];
-          }
-          sum += __shfl_xor_sync(0xffffffffu, sum, 1);           // 32-column unit = 2 threads
-          if (in) {
-            const int col0 = kb * B + 16 * t, vu = col0 >> 5;
-            uint4 w[2];
+        for (int h = 1; h < E; h <<= 1)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int *qq = q + 8 * hh;
-              w[hh].x = (uint32_t)(qq[0] & 0xFFFF) | ((uint32_t)qq[2] << 16);
-              w[hh].y = (uint32_t)(qq[4] & 0xFFFF) | ((uint32_t)qq[6] << 16);
-              w[hh].z = (uint32_t)(qq[1] & 0xFFFF) | ((uint32_t)qq[3] << 16);
-              w[hh].w = (uint32_t)(qq[5] & 0xFFFF) | ((uint32_t)qq[7] << 16);
-              const int ci = ((col0 >> 3) & 3) + hh;
-              *reinterpret_cast<uint4 *>(xi + 32 * vu + 8 * stk_chunk(vu, ci)) = w[hh];
+          for (int i = 0; i < E; ++i)
+            if (!(i & h)) {
+              const float a = v[i], b2 = v[i + h];
+              v[i] = a + b2;
+              v[i + h] = a - b2;
             }
-            if ((t & 3) == 0) xsc[col0 >> 6] = mx * (1.0f / 32767.0f);
-            if ((t & 1) == 0) xsu[vu] = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const bool upper = (lane & o) != 0;
+#pragma unroll
+          for (int i = 0; i < E; ++i) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[i], o);
+            v[i] = upper ? other - v[i] : v[i] + other;
           }
         }
+        float mx = 0.0f;
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          v[j] *= cb;
+          mx = fmaxf(mx, fabsf(v[j]));
+        }
+#pragma unroll
+        for (int o = 1; o < LPG; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
+        int q[E], sum = 0;
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          q[j] = max(-32767, min(32767, __float2int_rn(v[j] * inv)));
+          sum += q[j];
+        }
+#pragma unroll
+        for (int o = 1; o < LPU; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const int col0 = kb * B + E * lane, vu = col0 >> 5, ci = (col0 >> 3) & 3;
+        uint16_t *chunk = xi + 32 * vu + 8 * stk_chunk(vu, ci);
+        // DP2A order inside the 8-column chunk: {0, 2, 4, 6, 1, 3, 5, 7}
+        if constexpr (E == 8) {
+          uint4 w;
+          w.x = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[2] << 16);
+          w.y = (uint32_t)(q[4] & 0xFFFF) | ((uint32_t)q[6] << 16);
+          w.z = (uint32_t)(q[1] & 0xFFFF) | ((uint32_t)q[3] << 16);
+          w.w = (uint32_t)(q[5] & 0xFFFF) | ((uint32_t)q[7] << 16);
+          *reinterpret_cast<uint4 *>(chunk) = w;
+        } else {
+          // this lane holds columns 0..3 (lane even) or 4..7 (lane odd) of
+          // the chunk: words x, z or y, w of it
+          uint32_t *cw32 = reinterpret_cast<uint32_t *>(chunk) + (lane & 1);
+          cw32[0] = (uint32_t)(q[0] & 0xFFFF) | ((uint32_t)q[2] << 16);
+          cw32[2] = (uint32_t)(q[1] & 0xFFFF) | ((uint32_t)q[3] << 16);
+        }
+        if (lane % LPG == 0) xsc[col0 >> 6] = mx * (1.0f / 32767.0f);
+        if (lane % LPU == 0) xsu[vu] = sum;
+      }
     }
     stk_consumer_sync();
 
@@ -683,6 +744,7 @@ StkWs stk_ws_layout(const StackShapeInfo &si, int L, int G) {
 }
 
 bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &p) {
+  if (G < 1 || G > 256) return false;        // the t-share sums read at most 256 shares
   const int L = (int)Ls.size();
   p.L = L;
   p.H = Ls[0].m[2].M;
