@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kBssThreads) bss_logits_kernel(const BssParams
 
 // Masked weights and the partial p . V of one chunk.
 template <int D, int G>
-__global__ void __launch_bounds__(kBssThreads) bss_pv_kernel(const BssParams p) {
+__global__ void __launch_bounds__(kBssThreads, 3) bss_pv_kernel(const BssParams p) {
   constexpr int DL = D / 32;
   __shared__ float pw[G][kBssChunk];
   __shared__ float s_m[G];
@@ -190,15 +190,15 @@ __global__ void __launch_bounds__(kBssThreads) bss_pv_kernel(const BssParams p) 
 #pragma unroll
   for (int g = 0; g < G; ++g) lw[g] = 0.f;
   const uint16_t *vbase = p.v + ((size_t)b * p.Hkv + kh) * (size_t)L * D + lane * DL;
-  // warp w: keys w, w + 8, ... of the chunk, four at a time; a key dropped
+  // warp w: keys w, w + 8, ... of the chunk, two at a time; a key dropped
   // for every head is skipped without reading its V row
 #pragma unroll 1
-  for (int kk0 = warp; kk0 < kBssChunk; kk0 += 4 * kBssWarps) {
-    float vf[4][DL];
-    float wt[4][G];
-    bool any[4];
+  for (int kk0 = warp; kk0 < kBssChunk; kk0 += 2 * kBssWarps) {
+    float vf[2][DL];
+    float wt[2][G];
+    bool any[2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int kk = kk0 + u * kBssWarps;
       any[u] = false;
 #pragma unroll
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kBssThreads) bss_pv_kernel(const BssParams p) 
       if (any[u]) bss_load_row<DL>(vbase + (size_t)(key0 + kk) * D, vf[u]);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 2; ++u)
       if (any[u]) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -241,21 +241,24 @@ __global__ void __launch_bounds__(kBssThreads) bss_pv_kernel(const BssParams p) 
   }
 }
 
-// out[b][h][:] = sum_c pacc / sum_c psum, chunks in order.
+// out[b][h][:] = sum_c pacc / sum_c psum, chunks in order: thread (j, dd)
+// sums the j-th quarter of the chunks for dimension dd (loads in batches
+// of 16 in flight), and the quarters are added in order.
 template <int D>
-__global__ void __launch_bounds__(D) bss_merge_kernel(const BssParams p) {
-  const int h = blockIdx.x, b = blockIdx.y, dd = threadIdx.x;
+__global__ void __launch_bounds__(4 * D) bss_merge_kernel(const BssParams p) {
+  __shared__ float ps[4][D], ls[4];
+  const int h = blockIdx.x, b = blockIdx.y, dd = threadIdx.x % D, j = threadIdx.x / D;
   pdl_wait();
   const size_t row = (size_t)b * p.Hq + h;
+  const int c0 = (j * p.nc) / 4, c1 = ((j + 1) * p.nc) / 4;
   float l = 0.f, s = 0.f;
-  // chunks in order; the loads of a batch of 16 are issued together
-  for (int c0 = 0; c0 < p.nc; c0 += 16) {
+  for (int cb = c0; cb < c1; cb += 16) {
     float lv[16], sv[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-      const bool in = c0 + u < p.nc;
-      lv[u] = in ? p.psum[row * p.nc + c0 + u] : 0.f;
-      sv[u] = in ? p.pacc[(row * p.nc + c0 + u) * D + dd] : 0.f;
+      const bool in = cb + u < c1;
+      lv[u] = in && dd == 0 ? p.psum[row * p.nc + cb + u] : 0.f;
+      sv[u] = in ? p.pacc[(row * p.nc + cb + u) * D + dd] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
@@ -263,7 +266,13 @@ __global__ void __launch_bounds__(D) bss_merge_kernel(const BssParams p) {
       s += sv[u];
     }
   }
-  p.out[row * D + dd] = s / l;
+  ps[j][dd] = s;
+  if (dd == 0) ls[j] = l;
+  __syncthreads();
+  if (j == 0) {
+    const float lt = ((ls[0] + ls[1]) + ls[2]) + ls[3];
+    p.out[row * D + dd] = (((ps[0][dd] + ps[1][dd]) + ps[2][dd]) + ps[3][dd]) / lt;
+  }
 }
 
 namespace {
@@ -295,8 +304,8 @@ cudaError_t bss_run(const BssParams &p, cudaStream_t st, Launcher &L) {
   if (e != cudaSuccess) return e;
   e = L.launch("bss_pv", bss_pv_kernel<D, G>, grid, dim3(kBssThreads), 0, st, true, p);
   if (e != cudaSuccess) return e;
-  return L.launch("bss_merge", bss_merge_kernel<D>, dim3((unsigned)p.Hq, (unsigned)p.B), dim3(D), 0,
-                  st, true, p);
+  return L.launch("bss_merge", bss_merge_kernel<D>, dim3((unsigned)p.Hq, (unsigned)p.B),
+                  dim3(4 * D), 0, st, true, p);
 }
 }  // namespace
 

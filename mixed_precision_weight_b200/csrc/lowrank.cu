@@ -207,6 +207,39 @@ __device__ __forceinline__ double lr_sum_parts(const double *__restrict__ part, 
   return s;
 }
 
+// M[a][b] (row stride P + 1) = sum_b part[b][a][b] in ascending b for all
+// P x P entries: each thread's entries with a batch of partials each in
+// flight together (32 loads at most), the adds in order.
+template <int P>
+__device__ __forceinline__ void lr_fill_sums(const double *__restrict__ part, int nparts,
+                                             double *M) {
+  constexpr int EPT = (P * P + kLrThreads - 1) / kLrThreads;
+  constexpr int KB = EPT >= 32 ? 1 : 32 / EPT;      // partials per batch: <= 32 loads in flight
+  double acc[EPT];
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) acc[u] = 0.0;
+  for (int b0 = 0; b0 < nparts; b0 += KB) {
+    double v[EPT][KB];
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) {
+      const int e = threadIdx.x + u * kLrThreads;
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+        v[u][k] = (e < P * P && b0 + k < nparts) ? part[(size_t)(b0 + k) * P * P + e] : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < EPT; ++u)
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+        if (b0 + k < nparts) acc[u] += v[u][k];
+  }
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const int e = threadIdx.x + u * kLrThreads;
+    if (e < P * P) M[(e / P) * (P + 1) + e % P] = acc[u];
+  }
+}
+
 // One CTA: G = sum of the partials (in block order), shifted Cholesky
 // G + s I = L L^T, s = 1e-12 trace(G), and Linv = L^-1 (lower triangular).
 template <int P>
@@ -217,10 +250,8 @@ __global__ void __launch_bounds__(kLrThreads) lr_chol_kernel(const double *__res
   double(*L)[P + 1] = reinterpret_cast<double(*)[P + 1]>(lr_dyn + P * (P + 1));
   __shared__ double s_shift;
   const int tid = threadIdx.x;
-  for (int e = tid; e < P * P; e += kLrThreads) {
-    G[e / P][e % P] = lr_sum_parts(part, nparts, e, P * P);
-    L[e / P][e % P] = 0.0;
-  }
+  lr_fill_sums<P>(part, nparts, &G[0][0]);
+  for (int e = tid; e < P * P; e += kLrThreads) L[e / P][e % P] = 0.0;
   __syncthreads();
   if (tid == 0) {
     double tr = 0.0;
@@ -246,16 +277,18 @@ __global__ void __launch_bounds__(kLrThreads) lr_chol_kernel(const double *__res
     }
     __syncthreads();
   }
-  // Linv column by column: L x = e_c, forward substitution (one thread per column)
-  for (int c = tid; c < P; c += kLrThreads) {
-    double x[P];
+  // Linv column by column, L x = e_c by forward substitution: thread c owns
+  // column c of Li (in place of G, which is no longer read)
+  __syncthreads();
+  double(*Li)[P + 1] = G;
+  for (int cc = tid; cc < P; cc += kLrThreads)
     for (int i = 0; i < P; ++i) {
-      double v = i == c ? 1.0 : 0.0;
-      for (int k = c; k < i; ++k) v -= L[i][k] * x[k];
-      x[i] = i < c ? 0.0 : v / L[i][i];
+      double v = i == cc ? 1.0 : 0.0;
+      for (int k = cc; k < i; ++k) v -= L[i][k] * Li[k][cc];
+      Li[i][cc] = i < cc ? 0.0 : v / L[i][i];
     }
-    for (int i = 0; i < P; ++i) Linv[i * P + c] = x[i];
-  }
+  __syncthreads();
+  for (int e = tid; e < P * P; e += kLrThreads) Linv[e] = Li[e / P][e % P];
 }
 
 // Y[n][p] <- Y Linv^T (row y -> Linv y), in place: a CTA stages 32 rows in
@@ -307,10 +340,8 @@ __global__ void __launch_bounds__(kLrThreads) lr_eig_kernel(const double *__rest
   __shared__ double rowoff[P], rowdia[P];
   __shared__ double s_off;
   const int tid = threadIdx.x;
-  for (int e = tid; e < P * P; e += kLrThreads) {
-    A[e / P][e % P] = lr_sum_parts(part, nparts, e, P * P);
-    W[e / P][e % P] = (e / P == e % P) ? 1.0 : 0.0;
-  }
+  lr_fill_sums<P>(part, nparts, &A[0][0]);
+  for (int e = tid; e < P * P; e += kLrThreads) W[e / P][e % P] = (e / P == e % P) ? 1.0 : 0.0;
   if (tid < P) perm[tid] = tid;
   __syncthreads();
   for (int sweep = 0; sweep < 30; ++sweep) {
