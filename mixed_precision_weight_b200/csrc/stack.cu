@@ -45,7 +45,7 @@
 
 namespace dvssq {
 
-constexpr int kStkWarps = 16;
+constexpr int kStkWarps = 12;
 constexpr int kStkThreads = 32 * kStkWarps;
 constexpr int kStkCons = kStkWarps - 1;           // consumer warps (warp 0 streams weights)
 constexpr int kStkConsThreads = 32 * kStkCons;
@@ -147,6 +147,124 @@ __device__ __forceinline__ void stk_cp_async_commit() {
 }
 __device__ __forceinline__ void stk_cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// One tile's items for one consumer warp: RG rows x RR rounds per item,
+// straight-line; rows past the tile repeat its last row and are masked when
+// written.  Every operand comes in by value (no closure): the hot loop keeps
+// them in registers.
+struct StkTileArgs {
+  const uint8_t *q4s, *s4s, *q8s;
+  const uint16_t *us, *xi, *xsm, *s8m;
+  const int *xsu;
+  const float *xsc, *xssm, *tvm;
+  float *red;
+  int kq, ks, nsal, nu4, nu8, rk, nr, nrg, items, it0, ra, mi, rows_max, rounds_max;
+};
+
+template <int RGc>
+__device__ __forceinline__ void stk_tile_items(const StkTileArgs a, int lane) {
+  constexpr int RRc = 8 / RGc;
+  const uint8_t *__restrict__ q4s = a.q4s;
+  const uint8_t *__restrict__ s4s = a.s4s;
+  const uint8_t *__restrict__ q8s = a.q8s;
+  const uint16_t *__restrict__ us = a.us;
+  const uint16_t *__restrict__ xi = a.xi;
+  const uint16_t *__restrict__ xsm = a.xsm;
+  const uint16_t *__restrict__ s8m = a.s8m;
+  const int *__restrict__ xsu = a.xsu;
+  const float *__restrict__ xsc = a.xsc;
+  const float *__restrict__ xssm = a.xssm;
+  const float *__restrict__ tvm = a.tvm;
+  const int kq = a.kq, ks = a.ks, nsal = a.nsal, nu4 = a.nu4, nu8 = a.nu8, rk = a.rk;
+  const int nr = a.nr, nrg = a.nrg, items = a.items;
+  for (int it = a.it0; it < items; it += kStkCons) {
+    const int gi = it / nrg, rq = it - gi * nrg;
+    const int r0 = gi * RGc;
+    int rl[RGc];
+    float acc[RGc];
+#pragma unroll
+    for (int ri = 0; ri < RGc; ++ri) {
+      rl[ri] = min(r0 + ri, nr - 1);
+      acc[ri] = 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < RRc; ++u) {
+      const int task = 32 * (rq * RRc + u) + lane;
+      float f[RGc];
+      if (task < nu4) {
+        const int v = task, g = v >> 1;
+        uint4 xa[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
+        const int bias = 8 * xsu[v];
+        const float sc = xsc[g];
+#pragma unroll
+        for (int ri = 0; ri < RGc; ++ri) {
+          const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
+          const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+          int d[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
+            const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+            d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
+            d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
+            d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
+            d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
+          }
+          const float s4v =
+              bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
+          f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
+        }
+      } else if (task < nu4 + nu8) {
+        const int j = task - nu4;
+        uint4 xa[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
+        const float sc = xssm[j];
+#pragma unroll
+        for (int ri = 0; ri < RGc; ++ri) {
+          const uint8_t *qr = q8s + (size_t)rl[ri] * nsal + 32 * j;
+          const uint4 qa = *reinterpret_cast<const uint4 *>(qr);
+          const uint4 qb = *reinterpret_cast<const uint4 *>(qr + 16);
+          const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+          int d[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            d[i] = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d[i]);
+            d[i] = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d[i]);
+            d[i] = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d[i]);
+            d[i] = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d[i]);
+          }
+          f[ri] = bf16_bits_to_f32(s8m[a.ra + rl[ri]]) * sc * (float)((d[0] + d[1]) + (d[2] + d[3]));
+        }
+      } else {
+#pragma unroll
+        for (int ri = 0; ri < RGc; ++ri) f[ri] = 0.0f;
+      }
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri) acc[ri] += f[ri];
+    }
+    if (rq == 0 && lane < rk) {
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri)
+        acc[ri] = fmaf(bf16_bits_to_f32(us[rl[ri] * rk + lane]), tvm[lane], acc[ri]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri) acc[ri] += __shfl_xor_sync(0xffffffffu, acc[ri], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri)
+        if (r0 + ri < nr)
+          a.red[((size_t)a.mi * a.rows_max + a.ra + r0 + ri) * a.rounds_max + rq] = acc[ri];
+    }
+  }
 }
 
 template <int B>
@@ -528,102 +646,15 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         const uint8_t *s4s = q4s + nr * kq, *q8s = s4s + nr * ks;
         const uint16_t *us = reinterpret_cast<const uint16_t *>(q8s + nr * nsal);
         const int items = ngr * nrg;
-        // RG rows x RR rounds per item, straight-line: rows past the tile
-        // repeat its last row and are masked when accumulated
-        auto run_items = [&](auto rg_tag) {
-          constexpr int RGc = decltype(rg_tag)::value, RRc = 8 / RGc;
-          for (int it = (cw - rot + kStkCons * 64) % kStkCons; got && it < items; it += kStkCons) {
-            const int gi = it / nrg, rq = it - gi * nrg;
-            const int r0 = gi * RGc;
-            int rl[RGc];
-            float acc[RGc];
-#pragma unroll
-            for (int ri = 0; ri < RGc; ++ri) {
-              rl[ri] = min(r0 + ri, nr - 1);
-              acc[ri] = 0.0f;
-            }
-#pragma unroll
-            for (int u = 0; u < RRc; ++u) {
-              const int task = 32 * (rq * RRc + u) + lane;
-              float f[RGc];
-              if (task < nu4) {
-                const int v = task, g = v >> 1;
-                uint4 xa[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
-                const int bias = 8 * xsu[v];
-                const float sc = xsc[g];
-#pragma unroll
-                for (int ri = 0; ri < RGc; ++ri) {
-                  const uint4 w4 =
-                      *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
-                  const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-                  int d[4] = {0, 0, 0, 0};
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
-                    const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
-                    d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
-                    d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
-                    d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
-                    d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
-                  }
-                  const float s4v = bf16_bits_to_f32(
-                      reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
-                  f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
-                }
-              } else if (task < nu4 + nu8) {
-                const int j = task - nu4;
-                uint4 xa[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                  xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
-                const float sc = xssm[j];
-#pragma unroll
-                for (int ri = 0; ri < RGc; ++ri) {
-                  const uint8_t *qr = q8s + (size_t)rl[ri] * nsal + 32 * j;
-                  const uint4 qa = *reinterpret_cast<const uint4 *>(qr);
-                  const uint4 qb = *reinterpret_cast<const uint4 *>(qr + 16);
-                  const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-                  int d[4] = {0, 0, 0, 0};
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    d[i] = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d[i]);
-                    d[i] = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d[i]);
-                    d[i] = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d[i]);
-                    d[i] = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d[i]);
-                  }
-                  f[ri] = bf16_bits_to_f32(s8m[(i0 - ph.a) + rl[ri]]) * sc *
-                          (float)((d[0] + d[1]) + (d[2] + d[3]));
-                }
-              } else {
-#pragma unroll
-                for (int ri = 0; ri < RGc; ++ri) f[ri] = 0.0f;
-              }
-#pragma unroll
-              for (int ri = 0; ri < RGc; ++ri) acc[ri] += f[ri];
-            }
-            if (rq == 0 && lane < rk) {
-#pragma unroll
-              for (int ri = 0; ri < RGc; ++ri)
-                acc[ri] = fmaf(bf16_bits_to_f32(us[rl[ri] * rk + lane]), tvm[lane], acc[ri]);
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-#pragma unroll
-              for (int ri = 0; ri < RGc; ++ri) acc[ri] += __shfl_xor_sync(0xffffffffu, acc[ri], o);
-            }
-            if (lane == 0) {
-#pragma unroll
-              for (int ri = 0; ri < RGc; ++ri)
-                if (r0 + ri < nr)
-                  red[((size_t)mi * rows_max + (i0 - ph.a) + r0 + ri) * rounds_max + rq] = acc[ri];
-            }
-          }
-        };
-        if (RG == 4) run_items(std::integral_constant<int, 4>{});
-        else run_items(std::integral_constant<int, 2>{});
+        StkTileArgs ta;
+        ta.q4s = q4s; ta.s4s = s4s; ta.q8s = q8s; ta.us = us; ta.xi = xi; ta.xsm = xsm;
+        ta.s8m = s8m; ta.xsu = xsu; ta.xsc = xsc; ta.xssm = xssm; ta.tvm = tvm; ta.red = red;
+        ta.kq = kq; ta.ks = ks; ta.nsal = nsal; ta.nu4 = nu4; ta.nu8 = nu8; ta.rk = rk;
+        ta.nr = nr; ta.nrg = nrg; ta.items = got ? items : 0;
+        ta.it0 = (cw - rot + kStkCons * 64) % kStkCons;
+        ta.ra = i0 - ph.a; ta.mi = mi; ta.rows_max = rows_max; ta.rounds_max = rounds_max;
+        if (RG == 4) stk_tile_items<4>(ta, lane);
+        else stk_tile_items<2>(ta, lane);
         rot = (rot + items) % kStkCons;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
