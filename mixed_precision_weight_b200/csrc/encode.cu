@@ -670,24 +670,25 @@ __global__ void __launch_bounds__(128, 5) enc_pass2_kernel(const Pass2Params p) 
     if (tid == 0) s_tile[2 + (k & 1)] = (int)atomicAdd(p.tile_ctr, 1u);   // the tile after nxt
     double *const stash = p.stash_smem ? stash_s : nullptr;
     for (int ii = 0; ii < ipg; ++ii, ++pos) {
-      const int ia = ii + kP2Stages - 1;
-      issue(ia < ipg ? src_of(cur, ia) : src_of(nxt, ia - ipg), (pos + kP2Stages - 1) % kP2Stages);
-      cp_async_wait<kP2Stages - 1>();
-      __syncwarp();
       const int item = item0 + ii;
       const int kb = item >> rshift, r = item - (kb << rshift);
       const int row = (cur << rshift) + r;
       const bool valid = row < M;
+      // the exact-path mask of this row-block (written by pass 1, which
+      // completed before the select kernel released this one; read from L2),
+      // loaded first so that its latency overlaps the ring wait and the rotation
+      const uint32_t mk = valid ? __ldcg(p.xmask + (size_t)(row >> 4) * (K / B) + kb) : 0u;
+      const int ia = ii + kP2Stages - 1;
+      issue(ia < ipg ? src_of(cur, ia) : src_of(nxt, ia - ipg), (pos + kP2Stages - 1) % kP2Stages);
+      cp_async_wait<kP2Stages - 1>();
+      __syncwarp();
       const uint16_t *buf = ring[g][pos % kP2Stages];
       double v[16];
 #pragma unroll
       for (int a = 0; a < 16; ++a) v[a] = bf16_bits_to_f64(buf[P * a + t]);
       fwht_group<B>(v, sgrp, t);
-      // row-blocks that pass 1 flagged: exact integer sums, rounded once (the
-      // mask was written by pass 1, which completed before the select kernel
-      // released this one; read from L2)
+      // row-blocks that pass 1 flagged: exact integer sums, rounded once
       if (valid) {
-        const uint32_t mk = __ldcg(p.xmask + (size_t)(row >> 4) * (K / B) + kb);
         if (((mk >> (row & 15)) & 1u) && !block_has_nonfinite(buf, B)) {
           exact_pm_sums16(buf, B, t, sgrp);         // free until the staging below
 #pragma unroll

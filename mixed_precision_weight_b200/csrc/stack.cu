@@ -37,7 +37,6 @@
 // wait limit); a timeout sets the device error word and every warp leaves at
 // its next wait.
 #include "common.cuh"
-#include "fwht_group.cuh"
 #include "kernels.h"
 
 #include <algorithm>
@@ -49,7 +48,6 @@ constexpr int kStkWarps = 12;
 constexpr int kStkThreads = 32 * kStkWarps;
 constexpr int kStkCons = kStkWarps - 1;           // consumer warps (warp 0 streams weights)
 constexpr int kStkConsThreads = 32 * kStkCons;
-constexpr int kStkFwhtGroups = 20;                // 16-thread FWHT groups (10 warps)
 constexpr int kStkMaxRank = 32;                   // rank <= 32: one U t term per lane
 constexpr int kStkMaxSlots = 24;
 
@@ -63,7 +61,6 @@ struct StackParams {
   int tr_gu, tr_d;                // rows per tile of gate/up and of down
   int slot_bytes, nslots;
   int max_rank, max_nsal, rows_max, rounds_max;
-  int rg_gu, rg_d;                // rows per item of gate/up and of down
   const uint16_t *x;              // BF16 [H]
   uint16_t *y;                    // BF16 [H]: the running hidden state, then the output
   uint16_t *h;                    // BF16 [I]
@@ -71,7 +68,7 @@ struct StackParams {
   unsigned int *gbar;             // grid barrier counter, zero at launch
   // shared-memory offsets from the 1024-aligned base
   int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
-      o_scr, o_flag, o_tq, o_vhs, smem_total;
+      o_flag, o_grab, o_vhs, smem_total;
 };
 
 // Entries per matrix of the BF16 s8 staging: the own rows plus the partial
@@ -124,7 +121,7 @@ __device__ __forceinline__ int stk_xpos(int col) {
 struct StkPhase {
   int nm;                   // matrices of the phase (2: gate and up; 1: down)
   StackMatDesc m[2];
-  int K, a, b, tr, rg;      // input length, own rows [a, b), rows per tile, rows per item
+  int K, a, b, tr;          // input length, own rows [a, b), rows per tile (even)
   const uint16_t *src;      // input vector (BF16 [K])
   int tslot[2];             // t-share slot of each matrix
   // the matrices that consume this phase's output: their (V H) columns [a, b)
@@ -149,22 +146,23 @@ __device__ __forceinline__ void stk_cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// One tile's items for one consumer warp: RG rows x RR rounds per item,
-// straight-line; rows past the tile repeat its last row and are masked when
-// written.  Every operand comes in by value (no closure): the hot loop keeps
-// them in registers.
+// One item of a tile for one consumer warp: rows [2 gi, 2 gi + 2) of the tile
+// x rounds [RR rq, RR rq + RR), straight-line; a row past the tile repeats
+// its last row and is masked when written.  Every operand comes in by value
+// (no closure): the hot code keeps them in registers.
+constexpr int kStkRG = 2;                         // rows per item
 struct StkTileArgs {
   const uint8_t *q4s, *s4s, *q8s;
   const uint16_t *us, *xi, *xsm, *s8m;
   const int *xsu;
   const float *xsc, *xssm, *tvm;
   float *red;
-  int kq, ks, nsal, nu4, nu8, rk, nr, nrg, items, it0, ra, mi, rows_max, rounds_max;
+  int kq, ks, nsal, nu4, nu8, rk, nr, nrg, ra, mi, rows_max, rounds_max;
 };
 
-template <int RGc>
-__device__ __forceinline__ void stk_tile_items(const StkTileArgs a, int lane) {
-  constexpr int RRc = 8 / RGc;
+template <int RRc>
+__device__ __forceinline__ void stk_item(const StkTileArgs a, int it, int lane) {
+  constexpr int RGc = kStkRG;
   const uint8_t *__restrict__ q4s = a.q4s;
   const uint8_t *__restrict__ s4s = a.s4s;
   const uint8_t *__restrict__ q8s = a.q8s;
@@ -177,94 +175,99 @@ __device__ __forceinline__ void stk_tile_items(const StkTileArgs a, int lane) {
   const float *__restrict__ xssm = a.xssm;
   const float *__restrict__ tvm = a.tvm;
   const int kq = a.kq, ks = a.ks, nsal = a.nsal, nu4 = a.nu4, nu8 = a.nu8, rk = a.rk;
-  const int nr = a.nr, nrg = a.nrg, items = a.items;
-  for (int it = a.it0; it < items; it += kStkCons) {
-    const int gi = it / nrg, rq = it - gi * nrg;
-    const int r0 = gi * RGc;
-    int rl[RGc];
-    float acc[RGc];
+  const int nr = a.nr, nrg = a.nrg;
+  const int gi = it / nrg, rq = it - gi * nrg;
+  const int r0 = gi * RGc;
+  int rl[RGc];
+  float acc[RGc];
 #pragma unroll
-    for (int ri = 0; ri < RGc; ++ri) {
-      rl[ri] = min(r0 + ri, nr - 1);
-      acc[ri] = 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < RRc; ++u) {
-      const int task = 32 * (rq * RRc + u) + lane;
-      float f[RGc];
-      if (task < nu4) {
-        const int v = task, g = v >> 1;
-        uint4 xa[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
-        const int bias = 8 * xsu[v];
-        const float sc = xsc[g];
-#pragma unroll
-        for (int ri = 0; ri < RGc; ++ri) {
-          const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
-          const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-          int d[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
-            const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
-            d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
-            d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
-            d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
-            d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
-          }
-          const float s4v =
-              bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
-          f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
-        }
-      } else if (task < nu4 + nu8) {
-        const int j = task - nu4;
-        uint4 xa[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
-        const float sc = xssm[j];
-#pragma unroll
-        for (int ri = 0; ri < RGc; ++ri) {
-          const uint8_t *qr = q8s + (size_t)rl[ri] * nsal + 32 * j;
-          const uint4 qa = *reinterpret_cast<const uint4 *>(qr);
-          const uint4 qb = *reinterpret_cast<const uint4 *>(qr + 16);
-          const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-          int d[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            d[i] = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d[i]);
-            d[i] = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d[i]);
-            d[i] = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d[i]);
-            d[i] = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d[i]);
-          }
-          f[ri] = bf16_bits_to_f32(s8m[a.ra + rl[ri]]) * sc * (float)((d[0] + d[1]) + (d[2] + d[3]));
-        }
-      } else {
-#pragma unroll
-        for (int ri = 0; ri < RGc; ++ri) f[ri] = 0.0f;
-      }
-#pragma unroll
-      for (int ri = 0; ri < RGc; ++ri) acc[ri] += f[ri];
-    }
-    if (rq == 0 && lane < rk) {
-#pragma unroll
-      for (int ri = 0; ri < RGc; ++ri)
-        acc[ri] = fmaf(bf16_bits_to_f32(us[rl[ri] * rk + lane]), tvm[lane], acc[ri]);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-#pragma unroll
-      for (int ri = 0; ri < RGc; ++ri) acc[ri] += __shfl_xor_sync(0xffffffffu, acc[ri], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int ri = 0; ri < RGc; ++ri)
-        if (r0 + ri < nr)
-          a.red[((size_t)a.mi * a.rows_max + a.ra + r0 + ri) * a.rounds_max + rq] = acc[ri];
-    }
+  for (int ri = 0; ri < RGc; ++ri) {
+    rl[ri] = min(r0 + ri, nr - 1);
+    acc[ri] = 0.0f;
   }
+#pragma unroll
+  for (int u = 0; u < RRc; ++u) {
+    const int task = 32 * (rq * RRc + u) + lane;
+    float f[RGc];
+    if (task < nu4) {
+      const int v = task, g = v >> 1;
+      uint4 xa[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        xa[i] = *reinterpret_cast<const uint4 *>(xi + 32 * v + 8 * stk_chunk(v, i));
+      const int bias = 8 * xsu[v];
+      const float sc = xsc[g];
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri) {
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
+        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+        int d[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
+          const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+          d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
+          d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
+          d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
+          d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
+        }
+        const float s4v =
+            bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
+        f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
+      }
+    } else if (task < nu4 + nu8) {
+      const int j = task - nu4;
+      uint4 xa[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        xa[i] = *reinterpret_cast<const uint4 *>(xsm + 32 * j + 8 * stk_chunk(j, i));
+      const float sc = xssm[j];
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri) {
+        const uint8_t *qr = q8s + (size_t)rl[ri] * nsal + 32 * j;
+        const uint4 qa = *reinterpret_cast<const uint4 *>(qr);
+        const uint4 qb = *reinterpret_cast<const uint4 *>(qr + 16);
+        const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        int d[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d[i] = __dp2a_lo((int)xa[i].x, (int)qw[2 * i], d[i]);
+          d[i] = __dp2a_hi((int)xa[i].y, (int)qw[2 * i], d[i]);
+          d[i] = __dp2a_lo((int)xa[i].z, (int)qw[2 * i + 1], d[i]);
+          d[i] = __dp2a_hi((int)xa[i].w, (int)qw[2 * i + 1], d[i]);
+        }
+        f[ri] = bf16_bits_to_f32(s8m[a.ra + rl[ri]]) * sc * (float)((d[0] + d[1]) + (d[2] + d[3]));
+      }
+    } else {
+#pragma unroll
+      for (int ri = 0; ri < RGc; ++ri) f[ri] = 0.0f;
+    }
+#pragma unroll
+    for (int ri = 0; ri < RGc; ++ri) acc[ri] += f[ri];
+  }
+  if (rq == 0 && lane < rk) {
+#pragma unroll
+    for (int ri = 0; ri < RGc; ++ri)
+      acc[ri] = fmaf(bf16_bits_to_f32(us[rl[ri] * rk + lane]), tvm[lane], acc[ri]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+#pragma unroll
+    for (int ri = 0; ri < RGc; ++ri) acc[ri] += __shfl_xor_sync(0xffffffffu, acc[ri], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int ri = 0; ri < RGc; ++ri)
+      if (r0 + ri < nr)
+        a.red[((size_t)a.mi * a.rows_max + a.ra + r0 + ri) * a.rounds_max + rq] = acc[ri];
+  }
+}
+
+// Rounds per item for a matrix of `rounds` 32-task rounds: at most four, as
+// even as possible (3 for 3 rounds, 4 for 12, 3 for 9).
+__host__ __device__ __forceinline__ int stk_rr(int rounds) {
+  const int n = (rounds + 3) / 4;
+  return (rounds + n - 1) / n;
 }
 
 template <int B>
@@ -284,8 +287,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   uint16_t *s8c = reinterpret_cast<uint16_t *>(base + p.o_s8);  // [2][s8_stride] BF16
   float *red = reinterpret_cast<float *>(base + p.o_yv);        // [2][rows_max][rounds_max]
   float *vals = reinterpret_cast<float *>(base + p.o_vh);       // [rows_max] produced values
-  float *scr = reinterpret_cast<float *>(base + p.o_scr);
   volatile int *abort = reinterpret_cast<volatile int *>(base + p.o_flag);
+  int *s_grab = reinterpret_cast<int *>(base + p.o_grab);        // next item of the phase
+  int *s_done = s_grab + 1;                                       // [nslots] items done per slot
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = p.G;
@@ -295,10 +299,12 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kStkCons);
+      mbar_init(&empty[s], 1);
+      s_done[s] = 0;
     }
     fence_mbarrier_init();
     *abort = 0;
+    *s_grab = 0;
   }
   __syncthreads();
 
@@ -345,13 +351,11 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   const unsigned int err0 = *(volatile uint32_t *)&g_dvssq_error;
   uint32_t seq = 0;            // ring position, in step with the producer
   unsigned int nbar = 0;       // grid barriers passed
-  int rot = 0;                 // item -> warp rotation
   const int rows_max = p.rows_max, rounds_max = p.rounds_max;
   // per-matrix BF16 staging of s8: 16-byte words covering the own rows, so a
   // multiple of 8 entries (each slice starts 16-byte aligned)
   const int s8_stride = stk_s8_stride(rows_max);
   volatile int *s_live = abort + 1;
-  float *tq = reinterpret_cast<float *>(base + p.o_tq);         // t-share partial sums
   float *vhs = reinterpret_cast<float *>(base + p.o_vhs);       // (V H) columns of own outputs
 
   // Split grid barrier: a CTA arrives as soon as its outputs are written,
@@ -385,7 +389,6 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       ph.a = gu_a;
       ph.b = gu_b;
       ph.tr = p.tr_gu;
-      ph.rg = p.rg_gu;
       ph.src = l == 0 ? p.x : p.y;
       ph.tslot[0] = 0;
       ph.tslot[1] = 1;
@@ -401,7 +404,6 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       ph.a = d_a;
       ph.b = d_b;
       ph.tr = p.tr_d;
-      ph.rg = p.rg_d;
       ph.src = p.h;
       ph.tslot[0] = 2;
       ph.nout = l + 1 < p.L ? 2 : 0;
@@ -460,6 +462,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   // ---- one phase: activations in, the CTA's rows of one or two matrices out
   auto run_phase = [&](const StkPhase &ph) {
     const int K = ph.K, nrows = ph.b - ph.a;
+    if (ctid == 0) *s_grab = 0;    // the previous phase's rows ended before its last barrier
     // input vector and t: the G shares of each (matrix, k), NP parts per
     // pair summed in parallel, then the parts in order
     // the input vector, four 16-byte loads per thread in flight at once (its
@@ -623,48 +626,85 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     stk_consumer_sync();
 
     // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
-    // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
-    // RR rounds (RG RR = 8 independent dot products per lane); the items of
-    // a tile go round-robin over the consumer warps.
-    for (int mi = 0; mi < ph.nm; ++mi) {
-      const StackMatDesc &m = ph.m[mi];
-      const int nsal = m.n_sal, rk = m.r;
-      const int kq = m.K / 2, ks = m.K / 32, nu4 = m.K / 32, nu8 = nsal / 32;
-      const int rounds = (nu4 + nu8 + 31) / 32;
-      const int RG = ph.rg, RR = 8 / RG;
-      const int nrg = (rounds + RR - 1) / RR;
-      const float *tvm = tv + mi * kStkMaxRank;
-      const uint16_t *xsm = xsal + mi * p.max_nsal;
-      const float *xssm = xss + mi * (p.max_nsal / 32);
-      const uint16_t *s8m = s8c + mi * s8_stride + (ph.a & 7);
-      for (int i0 = ph.a; i0 < ph.b; i0 += ph.tr, ++seq) {
-        const int nr = min(ph.tr, ph.b - i0), ngr = (nr + RG - 1) / RG;
-        const int s = (int)(seq % (uint32_t)NS);
+    // q8) of one row; a round is 32 consecutive tasks.  An item is 2 rows x
+    // RR rounds of one tile.  The consumer warps take items from a shared
+    // counter in (matrix, tile, item) order, which is the ring's order; the
+    // warp that completes a tile's last item frees its ring slot.  With at
+    // least as many slots as consumer warps, a warp never takes an item of a
+    // tile whose slot still holds the tile one ring turn earlier (the items
+    // of the slots in between would need more warps than there are).
+    {
+      int nsal_[2], rk_[2], K_[2], nrg_[2], rr_[2], ntl_[2], ipt_[2], tot_[2];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        const bool on = mi < ph.nm;
+        nsal_[mi] = on ? ph.m[mi].n_sal : 0;
+        rk_[mi] = on ? ph.m[mi].r : 0;
+        K_[mi] = on ? ph.m[mi].K : 32;
+        const int rounds = (K_[mi] / 32 + nsal_[mi] / 32 + 31) / 32;
+        rr_[mi] = stk_rr(rounds);
+        nrg_[mi] = (rounds + rr_[mi] - 1) / rr_[mi];
+        ntl_[mi] = on ? (nrows + ph.tr - 1) / ph.tr : 0;
+        ipt_[mi] = (ph.tr / kStkRG) * nrg_[mi];
+        const int nl = nrows - (ntl_[mi] - 1) * ph.tr;
+        tot_[mi] = on ? (ntl_[mi] - 1) * ipt_[mi] + ((nl + kStkRG - 1) / kStkRG) * nrg_[mi] : 0;
+      }
+      const int total = tot_[0] + tot_[1];
+      for (;;) {
+        int gx = 0;
+        if (lane == 0) gx = atomicAdd(s_grab, 1);
+        gx = __shfl_sync(0xffffffffu, gx, 0);
+        if (gx >= total) break;
+        const int mi = gx < tot_[0] ? 0 : 1;
+        const int g = gx - (mi ? tot_[0] : 0);
+        const int ipt = mi ? ipt_[1] : ipt_[0];
+        const int tile = g / ipt, it = g - tile * ipt;
+        const uint32_t tseq = seq + (uint32_t)((mi ? ntl_[0] : 0) + tile);
+        const int s = (int)(tseq % (uint32_t)NS);
         const bool got =
-            __all_sync(0xffffffffu, stk_wait(&full[s], (seq / (uint32_t)NS) & 1u, abort));
+            __all_sync(0xffffffffu, stk_wait(&full[s], (tseq / (uint32_t)NS) & 1u, abort));
+        const int i0 = ph.a + tile * ph.tr;
+        const int nr = min(ph.tr, ph.b - i0);
+        const int nsal = mi ? nsal_[1] : nsal_[0], Km = mi ? K_[1] : K_[0];
+        const int nrg = mi ? nrg_[1] : nrg_[0], rr = mi ? rr_[1] : rr_[0];
+        const int kq = Km / 2, ks = Km / 32;
         const uint8_t *q4s = ring + (size_t)s * p.slot_bytes;
         const uint8_t *s4s = q4s + nr * kq, *q8s = s4s + nr * ks;
-        const uint16_t *us = reinterpret_cast<const uint16_t *>(q8s + nr * nsal);
-        const int items = ngr * nrg;
         StkTileArgs ta;
-        ta.q4s = q4s; ta.s4s = s4s; ta.q8s = q8s; ta.us = us; ta.xi = xi; ta.xsm = xsm;
-        ta.s8m = s8m; ta.xsu = xsu; ta.xsc = xsc; ta.xssm = xssm; ta.tvm = tvm; ta.red = red;
-        ta.kq = kq; ta.ks = ks; ta.nsal = nsal; ta.nu4 = nu4; ta.nu8 = nu8; ta.rk = rk;
-        ta.nr = nr; ta.nrg = nrg; ta.items = got ? items : 0;
-        ta.it0 = (cw - rot + kStkCons * 64) % kStkCons;
-        ta.ra = i0 - ph.a; ta.mi = mi; ta.rows_max = rows_max; ta.rounds_max = rounds_max;
-        if (RG == 4) stk_tile_items<4>(ta, lane);
-        else stk_tile_items<2>(ta, lane);
-        rot = (rot + items) % kStkCons;
+        ta.q4s = q4s; ta.s4s = s4s; ta.q8s = q8s;
+        ta.us = reinterpret_cast<const uint16_t *>(q8s + nr * nsal);
+        ta.xi = xi; ta.xsm = xsal + mi * p.max_nsal;
+        ta.s8m = s8c + mi * s8_stride + (ph.a & 7);
+        ta.xsu = xsu; ta.xsc = xsc; ta.xssm = xss + mi * (p.max_nsal / 32);
+        ta.tvm = tv + mi * kStkMaxRank; ta.red = red;
+        ta.kq = kq; ta.ks = ks; ta.nsal = nsal; ta.nu4 = Km / 32; ta.nu8 = nsal / 32;
+        ta.rk = mi ? rk_[1] : rk_[0];
+        ta.nr = nr; ta.nrg = nrg; ta.ra = i0 - ph.a; ta.mi = mi;
+        ta.rows_max = rows_max; ta.rounds_max = rounds_max;
+        if (got) {
+          switch (rr) {
+            case 1: stk_item<1>(ta, it, lane); break;
+            case 2: stk_item<2>(ta, it, lane); break;
+            case 3: stk_item<3>(ta, it, lane); break;
+            default: stk_item<4>(ta, it, lane); break;
+          }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0) {
+          const int nit = ((nr + kStkRG - 1) / kStkRG) * nrg;
+          if (atomicAdd(&s_done[s], 1) == nit - 1) {
+            atomicExch(&s_done[s], 0);
+            mbar_arrive(&empty[s]);
+          }
+        }
       }
+      seq += (uint32_t)(ntl_[0] + ntl_[1]);
     }
     stk_consumer_sync();
     // row results (round groups in order) back into red[mi][row][0]
     for (int mi = 0; mi < ph.nm; ++mi) {
       const int rounds = (ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32;
-      const int nrg = (rounds + 8 / ph.rg - 1) / (8 / ph.rg);
+      const int nrg = (rounds + stk_rr(rounds) - 1) / stk_rr(rounds);
       for (int i = ctid; i < nrows; i += kStkConsThreads) {
         float *rw = red + ((size_t)mi * rows_max + i) * rounds_max;
         float sum = rw[0];
@@ -774,7 +814,7 @@ StkWs stk_ws_layout(const StackShapeInfo &si, int L, int G) {
   return w;
 }
 
-bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &p) {
+bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
   if (G < 1 || G > 256) return false;        // the t-share sums read at most 256 shares
   const int L = (int)Ls.size();
   p.L = L;
@@ -793,8 +833,6 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &
     }
   p.tr_gu = std::max(2, (kStkSlotTarget / rb_gu) & ~1);
   p.tr_d = std::max(2, (kStkSlotTarget / rb_d) & ~1);
-  p.rg_gu = p.tr_gu >= 4 ? 4 : 2;
-  p.rg_d = p.tr_d >= 4 ? 4 : 2;
   p.slot_bytes = (std::max(p.tr_gu * rb_gu, p.tr_d * rb_d) + 127) & ~127;
   p.max_rank = max_rank;
   p.max_nsal = std::max(max_nsal, 32);
@@ -817,17 +855,18 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, int B, StackParams &
   p.o_s8 = take(2 * stk_s8_stride(p.rows_max) * 2);
   p.o_yv = take(2 * p.rows_max * p.rounds_max * 4);
   p.o_vh = take(p.rows_max * 4);
-  p.o_tq = take(kStkConsThreads * 4);
   {
     const int rg = (p.I + G - 1) / G, rd = (p.H + G - 1) / G;
     p.o_vhs = take(std::max(max_rank * rg, 2 * max_rank * rd) * 4);
   }
-  p.o_scr = take(kStkFwhtGroups * (B == 256 ? GroupScratch<256>::kElems : GroupScratch<128>::kElems) * 4);
   p.o_flag = take(16);
+  p.o_grab = take((1 + kStkMaxSlots) * 4);
   const int fixed = off;
   const int room = kStkSmemLimit - 1024 - fixed - 2 * kStkMaxSlots * 8 - 128;
   p.nslots = std::min(kStkMaxSlots, room / p.slot_bytes);
-  if (p.nslots < 2) return false;
+  // the consumer warps take items from a shared counter: a slot per warp at
+  // least keeps every taken item on the ring turn it waits for
+  if (p.nslots < kStkCons) return false;
   p.o_full = take(p.nslots * 8);
   p.o_empty = take(p.nslots * 8);
   off = (off + 1023) & ~1023;
@@ -899,7 +938,7 @@ cudaError_t launch_mlp_stack(const StackMatDesc *mats, int L, const StackShapeIn
   for (int l = 0; l < L; ++l)
     for (int mi = 0; mi < 3; ++mi) Ls[(size_t)l].m[mi] = mats[3 * l + mi];
   StackParams p{};
-  if (!stk_plan(Ls, G, si.block, p)) return cudaErrorNotSupported;
+  if (!stk_plan(Ls, G, p)) return cudaErrorNotSupported;
   const StkWs w = stk_ws_layout(si, L, G);
   char *base = static_cast<char *>(ws);
   p.layers = reinterpret_cast<const StackLayerDesc *>(base + w.desc);
