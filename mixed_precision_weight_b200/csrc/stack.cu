@@ -22,11 +22,13 @@
 //     runs ahead across layer boundaries while the consumers wait.
 //   * The 15 consumer warps run two phases per block, each ending in a grid
 //     barrier: gate+up (x -> h) and down (h -> x).  After a barrier every CTA
-//     reads the whole input vector, rotates it (16-thread Kronecker FWHT,
-//     FP32) into int16 with one scale per 64 columns, requantises the
-//     salient entries per 64-entry chunk, and runs its rows as exact int32
-//     dot products (DP2A on bytes u = q + 8, minus 8 times the segment sums),
-//     scaled per group in FP32.
+//     reads the whole input vector, rotates it (one warp per Hadamard block,
+//     FP32 butterflies in registers and shuffles) into int16 with one scale
+//     per 64 columns, requantises the salient entries per 32-entry chunk, and
+//     runs its rows as exact int32 dot products by DP2A: even columns as
+//     bytes q + 8 (minus 8 times the unit's even-column activation sum), odd
+//     columns as the high nibble masked in place, a signed byte equal to
+//     16 q (the sum divided by 16 exactly); scaled per group in FP32.
 //   * The rank-r term needs t = V (H x) = (V H) x for all of x.  With
 //     (V H) precomputed once in FP32, each CTA adds the share of the entries
 //     it produced, t_c = (V H)[:, own] x[own], at the end of the producing
@@ -68,7 +70,7 @@ struct StackParams {
   unsigned int *gbar;             // grid barrier counter, zero at launch
   // shared-memory offsets from the 1024-aligned base
   int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
-      o_flag, o_grab, o_vhs, smem_total;
+      o_flag, o_grab, o_ph, o_vhs, smem_total;
 };
 
 // Entries per matrix of the BF16 s8 staging: the own rows plus the partial
@@ -146,11 +148,10 @@ __device__ __forceinline__ void stk_cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// One item of a tile for one consumer warp: rows [2 gi, 2 gi + 2) of the tile
-// x rounds [RR rq, RR rq + RR), straight-line; a row past the tile repeats
-// its last row and is masked when written.  Every operand comes in by value
-// (no closure): the hot code keeps them in registers.
-constexpr int kStkRG = 2;                         // rows per item
+// One item of a tile for one consumer warp: rows [RG gi, RG gi + RG) of the
+// tile x rounds [RR rq, RR rq + RR), straight-line; a row past the tile
+// repeats its last row and is masked when written.  Every operand comes in by
+// value (no closure): the hot code keeps them in registers.
 struct StkTileArgs {
   const uint8_t *q4s, *s4s, *q8s;
   const uint16_t *us, *xi, *xsm, *s8m;
@@ -160,9 +161,8 @@ struct StkTileArgs {
   int kq, ks, nsal, nu4, nu8, rk, nr, nrg, ra, mi, rows_max, rounds_max;
 };
 
-template <int RRc>
+template <int RGc, int RRc>
 __device__ __forceinline__ void stk_item(const StkTileArgs a, int it, int lane) {
-  constexpr int RGc = kStkRG;
   const uint8_t *__restrict__ q4s = a.q4s;
   const uint8_t *__restrict__ s4s = a.s4s;
   const uint8_t *__restrict__ q8s = a.q8s;
@@ -201,19 +201,21 @@ __device__ __forceinline__ void stk_item(const StkTileArgs a, int it, int lane) 
       for (int ri = 0; ri < RGc; ++ri) {
         const uint4 w4 = *reinterpret_cast<const uint4 *>(q4s + (size_t)rl[ri] * kq + 16 * v);
         const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-        int d[4] = {0, 0, 0, 0};
+        // even columns (low nibbles) as bytes q + 8; odd columns (high
+        // nibbles) masked in place, which as signed bytes are exactly 16 q
+        int de[2] = {0, 0}, dd[2] = {0, 0};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t L = stk_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
-          const uint32_t Hh = stk_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
-          d[i] = __dp2a_lo((int)xa[i].x, (int)L, d[i]);
-          d[i] = __dp2a_hi((int)xa[i].y, (int)L, d[i]);
-          d[i] = __dp2a_lo((int)xa[i].z, (int)Hh, d[i]);
-          d[i] = __dp2a_hi((int)xa[i].w, (int)Hh, d[i]);
+          const uint32_t Hs = wd[i] & 0xF0F0F0F0u;
+          de[i & 1] = __dp2a_lo((int)xa[i].x, (int)L, de[i & 1]);
+          de[i & 1] = __dp2a_hi((int)xa[i].y, (int)L, de[i & 1]);
+          dd[i & 1] = __dp2a_lo((int)xa[i].z, (int)Hs, dd[i & 1]);
+          dd[i & 1] = __dp2a_hi((int)xa[i].w, (int)Hs, dd[i & 1]);
         }
         const float s4v =
             bf16_bits_to_f32(reinterpret_cast<const uint16_t *>(s4s + (size_t)rl[ri] * ks)[g]);
-        f[ri] = s4v * sc * (float)((d[0] + d[1]) + (d[2] + d[3]) - bias);
+        f[ri] = s4v * sc * (float)((de[0] + de[1] - bias) + ((dd[0] + dd[1]) >> 4));
       }
     } else if (task < nu4 + nu8) {
       const int j = task - nu4;
@@ -289,6 +291,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   float *vals = reinterpret_cast<float *>(base + p.o_vh);       // [rows_max] produced values
   volatile int *abort = reinterpret_cast<volatile int *>(base + p.o_flag);
   int *s_grab = reinterpret_cast<int *>(base + p.o_grab);        // next item of the phase
+  StkPhase *sph = reinterpret_cast<StkPhase *>(base + p.o_ph);  // the current phase
   int *s_done = s_grab + 1;                                       // [nslots] items done per slot
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -377,44 +380,49 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     return *s_live != 0;
   };
 
-  // phase descriptors: layer l, kind 0 = gate and up (x -> h), 1 = down (h -> x)
-  auto make_phase = [&](int l, int kind) {
-    StkPhase ph;
-    const StackLayerDesc *Ld = p.layers + l;
-    if (kind == 0) {
-      ph.nm = 2;
-      ph.m[0] = Ld->m[0];
-      ph.m[1] = Ld->m[1];
-      ph.K = p.H;
-      ph.a = gu_a;
-      ph.b = gu_b;
-      ph.tr = p.tr_gu;
-      ph.src = l == 0 ? p.x : p.y;
-      ph.tslot[0] = 0;
-      ph.tslot[1] = 1;
-      ph.nout = 1;
-      ph.ovh[0] = Ld->m[2].vh;
-      ph.oK[0] = Ld->m[2].K;
-      ph.orank[0] = Ld->m[2].r;
-      ph.oslot[0] = 2;
-    } else {
-      ph.nm = 1;
-      ph.m[0] = Ld->m[2];
-      ph.K = p.I;
-      ph.a = d_a;
-      ph.b = d_b;
-      ph.tr = p.tr_d;
-      ph.src = p.h;
-      ph.tslot[0] = 2;
-      ph.nout = l + 1 < p.L ? 2 : 0;
-      for (int j = 0; j < ph.nout; ++j) {
-        ph.ovh[j] = Ld[1].m[j].vh;
-        ph.oK[j] = Ld[1].m[j].K;
-        ph.orank[j] = Ld[1].m[j].r;
-        ph.oslot[j] = j;
+  // phase descriptors: layer l, kind 0 = gate and up (x -> h), 1 = down (h -> x).
+  // One thread writes the descriptor to shared memory and the consumers read
+  // it there: a per-thread copy would live in local memory, whose lines the
+  // small L1 (shared memory takes the rest) loses to L2 between uses.
+  auto set_phase = [&](int l, int kind) {
+    if (ctid == 0) {
+      StkPhase &ph = *sph;
+      const StackLayerDesc *Ld = p.layers + l;
+      if (kind == 0) {
+        ph.nm = 2;
+        ph.m[0] = Ld->m[0];
+        ph.m[1] = Ld->m[1];
+        ph.K = p.H;
+        ph.a = gu_a;
+        ph.b = gu_b;
+        ph.tr = p.tr_gu;
+        ph.src = l == 0 ? p.x : p.y;
+        ph.tslot[0] = 0;
+        ph.tslot[1] = 1;
+        ph.nout = 1;
+        ph.ovh[0] = Ld->m[2].vh;
+        ph.oK[0] = Ld->m[2].K;
+        ph.orank[0] = Ld->m[2].r;
+        ph.oslot[0] = 2;
+      } else {
+        ph.nm = 1;
+        ph.m[0] = Ld->m[2];
+        ph.K = p.I;
+        ph.a = d_a;
+        ph.b = d_b;
+        ph.tr = p.tr_d;
+        ph.src = p.h;
+        ph.tslot[0] = 2;
+        ph.nout = l + 1 < p.L ? 2 : 0;
+        for (int j = 0; j < ph.nout; ++j) {
+          ph.ovh[j] = Ld[1].m[j].vh;
+          ph.oK[j] = Ld[1].m[j].K;
+          ph.orank[j] = Ld[1].m[j].r;
+          ph.oslot[j] = j;
+        }
       }
     }
-    return ph;
+    stk_consumer_sync();
   };
 
   // weight-side data of a phase, loaded while the grid barrier is pending:
@@ -575,11 +583,11 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
 #pragma unroll
         for (int o = 1; o < LPG; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
-        int q[E], sum = 0;
+        int q[E], sum = 0;      // sum over the even columns (their codes carry the +8)
 #pragma unroll
         for (int j = 0; j < E; ++j) {
           q[j] = max(-32767, min(32767, __float2int_rn(v[j] * inv)));
-          sum += q[j];
+          if (!(j & 1)) sum += q[j];
         }
 #pragma unroll
         for (int o = 1; o < LPU; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -626,14 +634,15 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     stk_consumer_sync();
 
     // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
-    // q8) of one row; a round is 32 consecutive tasks.  An item is 2 rows x
-    // RR rounds of one tile.  The consumer warps take items from a shared
+    // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
+    // RR rounds of one tile (RG = 4 when the tile's rows allow it, else 2).  The consumer warps take items from a shared
     // counter in (matrix, tile, item) order, which is the ring's order; the
     // warp that completes a tile's last item frees its ring slot.  With at
     // least as many slots as consumer warps, a warp never takes an item of a
     // tile whose slot still holds the tile one ring turn earlier (the items
     // of the slots in between would need more warps than there are).
     {
+      const int RG = ph.tr % 4 == 0 ? 4 : 2;
       int nsal_[2], rk_[2], K_[2], nrg_[2], rr_[2], ntl_[2], ipt_[2], tot_[2];
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi) {
@@ -645,9 +654,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         rr_[mi] = stk_rr(rounds);
         nrg_[mi] = (rounds + rr_[mi] - 1) / rr_[mi];
         ntl_[mi] = on ? (nrows + ph.tr - 1) / ph.tr : 0;
-        ipt_[mi] = (ph.tr / kStkRG) * nrg_[mi];
+        ipt_[mi] = (ph.tr / RG) * nrg_[mi];
         const int nl = nrows - (ntl_[mi] - 1) * ph.tr;
-        tot_[mi] = on ? (ntl_[mi] - 1) * ipt_[mi] + ((nl + kStkRG - 1) / kStkRG) * nrg_[mi] : 0;
+        tot_[mi] = on ? (ntl_[mi] - 1) * ipt_[mi] + ((nl + RG - 1) / RG) * nrg_[mi] : 0;
       }
       const int total = tot_[0] + tot_[1];
       for (;;) {
@@ -682,16 +691,21 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         ta.nr = nr; ta.nrg = nrg; ta.ra = i0 - ph.a; ta.mi = mi;
         ta.rows_max = rows_max; ta.rounds_max = rounds_max;
         if (got) {
-          switch (rr) {
-            case 1: stk_item<1>(ta, it, lane); break;
-            case 2: stk_item<2>(ta, it, lane); break;
-            case 3: stk_item<3>(ta, it, lane); break;
-            default: stk_item<4>(ta, it, lane); break;
+          if (RG == 4) {
+            if (rr == 3) stk_item<4, 3>(ta, it, lane);
+            else if (rr == 4) stk_item<4, 4>(ta, it, lane);
+            else if (rr == 2) stk_item<4, 2>(ta, it, lane);
+            else stk_item<4, 1>(ta, it, lane);
+          } else {
+            if (rr == 3) stk_item<2, 3>(ta, it, lane);
+            else if (rr == 4) stk_item<2, 4>(ta, it, lane);
+            else if (rr == 2) stk_item<2, 2>(ta, it, lane);
+            else stk_item<2, 1>(ta, it, lane);
           }
         }
         __syncwarp();
         if (lane == 0) {
-          const int nit = ((nr + kStkRG - 1) / kStkRG) * nrg;
+          const int nit = ((nr + RG - 1) / RG) * nrg;
           if (atomicAdd(&s_done[s], 1) == nit - 1) {
             atomicExch(&s_done[s], 0);
             mbar_arrive(&empty[s]);
@@ -716,7 +730,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   };
 
   // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
-  StkPhase ph = make_phase(0, 0);
+  set_phase(0, 0);
+  const StkPhase &ph = *sph;
   prefetch(ph);
   {
     const int n = d_b - d_a;
@@ -755,7 +770,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       stk_consumer_sync();
       if (live) t_share_out(ph);
       grid_arrive();
-      ph = make_phase(l, 1);
+      set_phase(l, 1);
       prefetch(ph);
       live = grid_wait() && live;
     }
@@ -772,7 +787,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       if (l + 1 < p.L) {
         if (live) t_share_out(ph);
         grid_arrive();
-        ph = make_phase(l + 1, 0);
+        set_phase(l + 1, 0);
         prefetch(ph);
         live = grid_wait() && live;
       }
@@ -861,6 +876,7 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
   }
   p.o_flag = take(16);
   p.o_grab = take((1 + kStkMaxSlots) * 4);
+  p.o_ph = take((int)sizeof(StkPhase));
   const int fixed = off;
   const int room = kStkSmemLimit - 1024 - fixed - 2 * kStkMaxSlots * 8 - 128;
   p.nslots = std::min(kStkMaxSlots, room / p.slot_bytes);
