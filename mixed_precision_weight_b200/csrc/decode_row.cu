@@ -8,10 +8,13 @@
 // path keeps the contraction in 32-bit integers instead:
 //   * the rotated activations x_rot = H x are held as int16 with one FP32
 //     scale per 64-column group (|x| <= 32767 * scale, relative step 2^-15);
-//   * each nibble becomes the byte u = q + 8 in [0, 15] with one LOP3 per
-//     four nibbles, and DP2A multiplies two int16 activations by two bytes;
-//   * a 64-column group sum is exact in int32; subtracting 8 * (sum of the
-//     group's int16 activations) gives sum q * x_int exactly, and the group
+//   * an even column's nibble becomes the byte u = q + 8 in [0, 15] (one
+//     LOP3 per four nibbles); an odd column's nibble, masked in place, is a
+//     signed byte equal to 16 q (one AND per four); DP2A multiplies two int16
+//     activations by two bytes;
+//   * a 64-column group sum is exact in int32: the even-column sum minus
+//     8 * (sum of the group's even-column int16 activations), plus the
+//     odd-column sum divided by 16 (exactly), is sum q * x_int, and the group
 //     result s4 * scale * sum is accumulated in FP32.
 // The salient INT8 columns run the same way (signed bytes, no bias), with
 // the salient activations requantised per 128-entry chunk.
@@ -334,11 +337,11 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float inv = mx > 0.0f ? 32767.0f / mx : 0.0f;
-      int q[16], sum = 0;
+      int q[16], sum = 0;      // sum over the even columns (their codes carry the +8)
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         q[j] = max(-32767, min(32767, __float2int_rn(v[j] * inv)));
-        sum += q[j];
+        if (!(j & 1)) sum += q[j];
       }
       sum += __shfl_xor_sync(0xffffffffu, sum, 1);
       sum += __shfl_xor_sync(0xffffffffu, sum, 2);
@@ -505,11 +508,13 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
         const uint4 wa = *reinterpret_cast<const uint4 *>(row + ((c0 ^ (r & 7)) << 4));
         const uint4 wb = *reinterpret_cast<const uint4 *>(row + (((c0 + 1) ^ (r & 7)) << 4));
         const uint32_t wd[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        // even columns (low nibbles) as bytes q + 8; odd columns (high
+        // nibbles) masked in place, which as signed bytes are exactly 16 q
         uint32_t L[8], H[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           L[i] = lop3_splice(wd[i], 0x0F0F0F0Fu, 0x08080808u);
-          H[i] = lop3_splice(wd[i] >> 4, 0x0F0F0F0Fu, 0x08080808u);
+          H[i] = wd[i] & 0xF0F0F0F0u;
         }
         const float s4v = bf16_bits_to_f32(sb[gi]);
 #pragma unroll
@@ -524,7 +529,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) dec_row_kernel(
             d1 = dp2a_lo(sg.z, H[i], d1);
             d1 = dp2a_hi(sg.w, H[i], d1);
           }
-          const int dq = d0 + d1 - 8 * xsum[tok * KG + gcol];
+          const int dq = d0 - 8 * xsum[tok * KG + gcol] + (d1 >> 4);
           acc[tok] = fmaf(s4v * xsc[tok * KG + gcol], (float)dq, acc[tok]);
         }
       }
