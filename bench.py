@@ -82,8 +82,8 @@ def kernel_bytes(name, M, K, rank, n_sal, T):
 # The source files each kernel is built from: a recorded DRAM count stays valid
 # while these files are unchanged.
 KERNEL_SOURCES = {
-    "enc_pass1": ("encode.cu", "fwht_group.cuh"),
-    "enc_pass2": ("encode.cu", "fwht_group.cuh"),
+    "enc_pass1": ("encode.cu", "fwht_group.cuh", "exact_sum.cuh"),
+    "enc_pass2": ("encode.cu", "fwht_group.cuh", "exact_sum.cuh"),
     "enc_select": ("encode.cu",),
     "dec_row": ("decode_row.cu", "fwht_group.cuh"),
     "dec_main": ("decode.cu", "fwht_group.cuh"),
@@ -91,7 +91,11 @@ KERNEL_SOURCES = {
     "pre_act": ("prefill.cu", "fwht_group.cuh"),
     "pre_mat": ("prefill.cu",),
     "pre_gemm": ("prefill.cu", "common.cuh"),
-    "mlp_stack": ("stack.cu", "fwht_group.cuh"),
+    "mlp_stack": ("stack.cu", "common.cuh"),
+    "materialize": ("materialize.cu",),
+    "lr_mul": ("lowrank.cu",),
+    "bss_logits": ("attention.cu",),
+    "bss_pv": ("attention.cu",),
 }
 
 
