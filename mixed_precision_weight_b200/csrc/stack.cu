@@ -265,11 +265,13 @@ __device__ __forceinline__ void stk_item(const StkTileArgs a, int it, int lane) 
   }
 }
 
-// Rounds per item for a matrix of `rounds` 32-task rounds: at most four, as
-// even as possible (3 for 3 rounds, 4 for 12, 3 for 9).
+// Rounds per item for a matrix of `rounds` 32-task rounds: three or four,
+// as even as possible (3 for 3 rounds, 4 for 12, 3 for 9; 3 for one or two
+// rounds, whose missing rounds are idle).  Two item shapes per row count
+// keep the kernel's code small.
 __host__ __device__ __forceinline__ int stk_rr(int rounds) {
   const int n = (rounds + 3) / 4;
-  return (rounds + n - 1) / n;
+  return max(3, (rounds + n - 1) / n);
 }
 
 template <int B>
@@ -635,14 +637,19 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
 
     // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
     // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
-    // RR rounds of one tile (RG = 4 when the tile's rows allow it, else 2).  The consumer warps take items from a shared
+    // RR rounds of one tile (RG = 4 for three-round items when the tile's rows
+    // allow it, else 2).  The consumer warps take items from a shared
     // counter in (matrix, tile, item) order, which is the ring's order; the
     // warp that completes a tile's last item frees its ring slot.  With at
     // least as many slots as consumer warps, a warp never takes an item of a
     // tile whose slot still holds the tile one ring turn earlier (the items
     // of the slots in between would need more warps than there are).
     {
-      const int RG = ph.tr % 4 == 0 ? 4 : 2;
+      // four-row items where the tile's rows allow it and every matrix of the
+      // phase takes three-round items (three item shapes in all)
+      int RG = ph.tr % 4 == 0 ? 4 : 2;
+      for (int mi = 0; mi < ph.nm; ++mi)
+        if (stk_rr((ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32) != 3) RG = 2;
       int nsal_[2], rk_[2], K_[2], nrg_[2], rr_[2], ntl_[2], ipt_[2], tot_[2];
 #pragma unroll
       for (int mi = 0; mi < 2; ++mi) {
@@ -692,15 +699,10 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         ta.rows_max = rows_max; ta.rounds_max = rounds_max;
         if (got) {
           if (RG == 4) {
-            if (rr == 3) stk_item<4, 3>(ta, it, lane);
-            else if (rr == 4) stk_item<4, 4>(ta, it, lane);
-            else if (rr == 2) stk_item<4, 2>(ta, it, lane);
-            else stk_item<4, 1>(ta, it, lane);
+            stk_item<4, 3>(ta, it, lane);
           } else {
             if (rr == 3) stk_item<2, 3>(ta, it, lane);
-            else if (rr == 4) stk_item<2, 4>(ta, it, lane);
-            else if (rr == 2) stk_item<2, 2>(ta, it, lane);
-            else stk_item<2, 1>(ta, it, lane);
+            else stk_item<2, 4>(ta, it, lane);
           }
         }
         __syncwarp();
@@ -715,10 +717,14 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       seq += (uint32_t)(ntl_[0] + ntl_[1]);
     }
     stk_consumer_sync();
-    // row results (round groups in order) back into red[mi][row][0]
+    // row results (round groups in order) back into red[mi][row][0]; a
+    // matrix whose items span all rounds of a row has nothing to add
+    bool more = false;
     for (int mi = 0; mi < ph.nm; ++mi) {
       const int rounds = (ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32;
       const int nrg = (rounds + stk_rr(rounds) - 1) / stk_rr(rounds);
+      if (nrg == 1) continue;
+      more = true;
       for (int i = ctid; i < nrows; i += kStkConsThreads) {
         float *rw = red + ((size_t)mi * rows_max + i) * rounds_max;
         float sum = rw[0];
@@ -726,7 +732,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         rw[0] = sum;
       }
     }
-    stk_consumer_sync();
+    if (more) stk_consumer_sync();
   };
 
   // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
@@ -752,10 +758,14 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   grid_arrive();
   bool live = grid_wait();
 
-  // ---- the blocks: gate+up (x -> h), then down (h -> x)
-  for (int l = 0; l < p.L; ++l) {
-    {
-      if (live) run_phase(ph);
+  // ---- the blocks: gate+up (x -> h), then down (h -> x).  One loop over the
+  // 2 L phases with a single call site per step, so that the phase's code
+  // exists once in the kernel (it is executed once per phase and must stay
+  // within the instruction caches).
+  for (int step = 0; step < 2 * p.L; ++step) {
+    const int l = step >> 1, kind = step & 1;
+    if (live) run_phase(ph);
+    if (kind == 0) {
       // h = RN_bf16(gelu(g) u), g and u rounded to BF16 first
       const int n = gu_b - gu_a;
       for (int i = ctid; i < n && live; i += kStkConsThreads) {
@@ -766,32 +776,22 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         p.h[gu_a + i] = hb;
         vals[i] = bf16_bits_to_f32(hb);
       }
-      stk_cp_async_wait_all();
-      stk_consumer_sync();
-      if (live) t_share_out(ph);
-      grid_arrive();
-      set_phase(l, 1);
-      prefetch(ph);
-      live = grid_wait() && live;
-    }
-    {
-      if (live) run_phase(ph);
+    } else {
       const int n = d_b - d_a;
       for (int i = ctid; i < n && live; i += kStkConsThreads) {
         const uint16_t xb = f32_to_bf16_rn_bits(red[(size_t)i * rounds_max]);
         p.y[d_a + i] = xb;
         vals[i] = bf16_bits_to_f32(xb);
       }
-      stk_cp_async_wait_all();
-      stk_consumer_sync();
-      if (l + 1 < p.L) {
-        if (live) t_share_out(ph);
-        grid_arrive();
-        set_phase(l + 1, 0);
-        prefetch(ph);
-        live = grid_wait() && live;
-      }
     }
+    stk_cp_async_wait_all();
+    stk_consumer_sync();
+    if (step + 1 == 2 * p.L) break;     // the last block's output needs no t shares
+    if (live) t_share_out(ph);
+    grid_arrive();
+    set_phase(kind == 0 ? l : l + 1, kind ^ 1);
+    prefetch(ph);
+    live = grid_wait() && live;
   }
 }
 
