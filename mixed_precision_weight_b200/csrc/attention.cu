@@ -20,6 +20,8 @@
 //               key that the haze mask drops for all G heads is never read;
 //   bss_merge   out = sum over chunks of the partials / sum of the weights,
 //               in chunk order (deterministic).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -190,34 +192,68 @@ __global__ void __launch_bounds__(kBssThreads, 3) bss_pv_kernel(const BssParams 
 #pragma unroll
   for (int g = 0; g < G; ++g) lw[g] = 0.f;
   const uint16_t *vbase = p.v + ((size_t)b * p.Hkv + kh) * (size_t)L * D + lane * DL;
-  // warp w: keys w, w + 8, ... of the chunk, two at a time; a key dropped
-  // for every head is skipped without reading its V row
-#pragma unroll 1
-  for (int kk0 = warp; kk0 < kBssChunk; kk0 += 2 * kBssWarps) {
-    float vf[2][DL];
-    float wt[2][G];
-    bool any[2];
+  // warp w: keys w + 8 j of the chunk in groups of KG, software-pipelined:
+  // the raw V rows of the next group are in flight while the current group
+  // is weighted and added.  A key dropped for every head is skipped without
+  // reading its V row.
+  using Raw = typename std::conditional<DL == 8, uint4, uint2>::type;
+  constexpr int KG = 2;                                    // keys per group
+  constexpr int NGRP = kBssChunk / (kBssWarps * KG);       // groups per warp
+  Raw raw[2][KG];
+  auto issue = [&](int grp, Raw *dst) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int kk = kk0 + u * kBssWarps;
-      any[u] = false;
+    for (int u = 0; u < KG; ++u) {
+      const int kk = warp + kBssWarps * (KG * grp + u);
+      bool any = false;
+#pragma unroll
+      for (int g = 0; g < G; ++g) any |= pw[g][kk] != 0.f;
+      if (any) dst[u] = *reinterpret_cast<const Raw *>(vbase + (size_t)(key0 + kk) * D);
+    }
+  };
+  auto consume = [&](int grp, const Raw *src) {
+#pragma unroll
+    for (int u = 0; u < KG; ++u) {
+      const int kk = warp + kBssWarps * (KG * grp + u);
+      float wt[G];
+      bool any = false;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        wt[u][g] = kk < kBssChunk ? pw[g][kk] : 0.f;
-        any[u] |= wt[u][g] != 0.f;
+        wt[g] = pw[g][kk];
+        any |= wt[g] != 0.f;
       }
-      if (any[u]) bss_load_row<DL>(vbase + (size_t)(key0 + kk) * D, vf[u]);
-    }
+      if (!any) continue;
+      float vf[DL];
+      if constexpr (DL == 8) {
+        const uint32_t w[4] = {src[u].x, src[u].y, src[u].z, src[u].w};
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (any[u]) {
+        for (int i = 0; i < 4; ++i) {
+          vf[2 * i] = __uint_as_float(w[i] << 16);
+          vf[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+      } else {
+        const uint32_t w[2] = {src[u].x, src[u].y};
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          lw[g] += wt[u][g];
-#pragma unroll
-          for (int i = 0; i < DL; ++i) acc[g][i] = fmaf(wt[u][g], vf[u][i], acc[g][i]);
+        for (int i = 0; i < 2; ++i) {
+          vf[2 * i] = __uint_as_float(w[i] << 16);
+          vf[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
       }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        lw[g] += wt[g];
+#pragma unroll
+        for (int i = 0; i < DL; ++i) acc[g][i] = fmaf(wt[g], vf[i], acc[g][i]);
+      }
+    }
+  };
+  static_assert(NGRP % 2 == 0, "groups go in pairs (double buffer)");
+  issue(0, raw[0]);
+#pragma unroll 1
+  for (int grp = 0; grp < NGRP; grp += 2) {
+    issue(grp + 1, raw[1]);
+    consume(grp, raw[0]);
+    if (grp + 2 < NGRP) issue(grp + 2, raw[0]);
+    consume(grp + 1, raw[1]);
   }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
