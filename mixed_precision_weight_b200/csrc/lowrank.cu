@@ -210,10 +210,10 @@ __device__ __forceinline__ double lr_sum_parts(const double *__restrict__ part, 
 // M[a][b] (row stride P + 1) = sum_b part[b][a][b] in ascending b for all
 // P x P entries: each thread's entries with a batch of partials each in
 // flight together (32 loads at most), the adds in order.
-template <int P>
+template <int P, int NT = kLrThreads>
 __device__ __forceinline__ void lr_fill_sums(const double *__restrict__ part, int nparts,
                                              double *M) {
-  constexpr int EPT = (P * P + kLrThreads - 1) / kLrThreads;
+  constexpr int EPT = (P * P + NT - 1) / NT;
   constexpr int KB = EPT >= 32 ? 1 : 32 / EPT;      // partials per batch: <= 32 loads in flight
   double acc[EPT];
 #pragma unroll
@@ -222,7 +222,7 @@ __device__ __forceinline__ void lr_fill_sums(const double *__restrict__ part, in
     double v[EPT][KB];
 #pragma unroll
     for (int u = 0; u < EPT; ++u) {
-      const int e = threadIdx.x + u * kLrThreads;
+      const int e = threadIdx.x + u * NT;
 #pragma unroll
       for (int k = 0; k < KB; ++k)
         v[u][k] = (e < P * P && b0 + k < nparts) ? part[(size_t)(b0 + k) * P * P + e] : 0.0;
@@ -235,92 +235,101 @@ __device__ __forceinline__ void lr_fill_sums(const double *__restrict__ part, in
   }
 #pragma unroll
   for (int u = 0; u < EPT; ++u) {
-    const int e = threadIdx.x + u * kLrThreads;
+    const int e = threadIdx.x + u * NT;
     if (e < P * P) M[(e / P) * (P + 1) + e % P] = acc[u];
   }
 }
 
 // One CTA: G = sum of the partials (in block order), shifted Cholesky
-// G + s I = L L^T, s = 1e-12 trace(G), and Linv = L^-1 (lower triangular).
+// G + s I = L L^T with s = 1e-12 trace(G), right-looking: column j of L and
+// the rank-one update of the trailing matrix by all threads, one barrier per
+// column (each entry's updates keep the column order of a left-looking
+// factorisation).  A zero block (trace 0) writes L = 0, which the solve
+// maps to zero rows.
+constexpr int kLrCholThreads = 512;
 template <int P>
-__global__ void __launch_bounds__(kLrThreads) lr_chol_kernel(const double *__restrict__ part,
-                                                             int nparts, double *__restrict__ Linv) {
+__global__ void __launch_bounds__(kLrCholThreads) lr_chol_kernel(const double *__restrict__ part,
+                                                                 int nparts, double *__restrict__ Lout) {
   extern __shared__ double lr_dyn[];
-  double(*G)[P + 1] = reinterpret_cast<double(*)[P + 1]>(lr_dyn);
-  double(*L)[P + 1] = reinterpret_cast<double(*)[P + 1]>(lr_dyn + P * (P + 1));
+  double(*A)[P + 1] = reinterpret_cast<double(*)[P + 1]>(lr_dyn);            // G + s I, updated
+  double(*Lm)[P + 1] = reinterpret_cast<double(*)[P + 1]>(lr_dyn + P * (P + 1));
   __shared__ double s_shift;
   const int tid = threadIdx.x;
-  lr_fill_sums<P>(part, nparts, &G[0][0]);
-  for (int e = tid; e < P * P; e += kLrThreads) L[e / P][e % P] = 0.0;
+  lr_fill_sums<P, kLrCholThreads>(part, nparts, &A[0][0]);
+  for (int e = tid; e < P * P; e += kLrCholThreads) Lm[e / P][e % P] = 0.0;
   __syncthreads();
   if (tid == 0) {
     double tr = 0.0;
-    for (int j = 0; j < P; ++j) tr += G[j][j];
+    for (int j = 0; j < P; ++j) tr += A[j][j];
     s_shift = 1e-12 * tr;
   }
   __syncthreads();
-  if (s_shift == 0.0) {             // a zero block: orth() maps it to zero
-    for (int e = tid; e < P * P; e += kLrThreads) Linv[e] = 0.0;
+  const double sh = s_shift;
+  if (sh == 0.0) {
+    for (int e = tid; e < P * P; e += kLrCholThreads) Lout[e] = 0.0;
     return;
   }
+  if (tid < P) A[tid][tid] += sh;
+  __syncthreads();
   for (int j = 0; j < P; ++j) {
-    if (tid == 0) {
-      double d = G[j][j] + s_shift;
-      for (int k = 0; k < j; ++k) d -= L[j][k] * L[j][k];
-      L[j][j] = sqrt(fmax(d, s_shift));
+    const double ljj = sqrt(fmax(A[j][j], sh));
+    const int nc = P - 1 - j;                    // rows below j
+    for (int e = tid; e < nc * (nc + 1); e += kLrCholThreads) {
+      const int i = j + 1 + e / (nc + 1), k = j + e % (nc + 1);   // k = j: the column itself
+      if (k > i) continue;
+      const double lij = A[i][j] / ljj;
+      if (k == j) {
+        Lm[i][j] = lij;
+      } else {
+        const double lkj = A[k][j] / ljj;
+        A[i][k] -= lij * lkj;
+      }
     }
-    __syncthreads();
-    for (int i = j + 1 + tid; i < P; i += kLrThreads) {
-      double v = G[i][j];
-      for (int k = 0; k < j; ++k) v -= L[i][k] * L[j][k];
-      L[i][j] = v / L[j][j];
-    }
+    if (tid == 0) Lm[j][j] = ljj;
     __syncthreads();
   }
-  // Linv column by column, L x = e_c by forward substitution: thread c owns
-  // column c of Li (in place of G, which is no longer read)
-  __syncthreads();
-  double(*Li)[P + 1] = G;
-  for (int cc = tid; cc < P; cc += kLrThreads)
-    for (int i = 0; i < P; ++i) {
-      double v = i == cc ? 1.0 : 0.0;
-      for (int k = cc; k < i; ++k) v -= L[i][k] * Li[k][cc];
-      Li[i][cc] = i < cc ? 0.0 : v / L[i][i];
-    }
-  __syncthreads();
-  for (int e = tid; e < P * P; e += kLrThreads) Linv[e] = Li[e / P][e % P];
+  for (int e = tid; e < P * P; e += kLrCholThreads) Lout[e] = Lm[e / P][e % P];
 }
 
-// Y[n][p] <- Y Linv^T (row y -> Linv y), in place: a CTA stages 32 rows in
-// shared memory and each thread forms p/8 of their outputs.
+// Y[n][p] <- Y L^-T (row y -> L^-1 y), in place, by forward substitution:
+// one thread per row, the row in registers, L in shared memory (FP32, its
+// reciprocal diagonal from fp64).  The dependency chain of a row is long
+// but the rows run side by side.
+constexpr int kLrSolveThreads = 64;
 template <int P>
-__global__ void __launch_bounds__(kLrThreads) lr_apply_linv_kernel(float *__restrict__ Y, int n,
-                                                                   const double *__restrict__ Linv) {
+__global__ void __launch_bounds__(kLrSolveThreads) lr_apply_solve_kernel(float *__restrict__ Y, int n,
+                                                                         const double *__restrict__ Lg) {
   __shared__ float Ls[P][P + 1];
-  __shared__ float ys[32][P + 1];
-  for (int e = threadIdx.x; e < P * P; e += kLrThreads) Ls[e / P][e % P] = (float)Linv[e];
-  for (long long r0 = (long long)blockIdx.x * 32; r0 < n; r0 += (long long)gridDim.x * 32) {
-    constexpr int LPT = 32 * P / kLrThreads;
-    float v[LPT];
-#pragma unroll
-    for (int u = 0; u < LPT; ++u) {
-      const int e = threadIdx.x + u * kLrThreads, rr = e / P;
-      v[u] = r0 + rr < n ? Y[r0 * P + e] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < LPT; ++u) {
-      const int e = threadIdx.x + u * kLrThreads;
-      ys[e / P][e % P] = v[u];
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < 32 * P; e += kLrThreads) {
-      const int rr = e / P, i = e - rr * P;
-      float s = 0.f;
-      for (int k = 0; k <= i; ++k) s = fmaf(Ls[i][k], ys[rr][k], s);
-      if (r0 + rr < n) Y[(r0 + rr) * P + i] = s;
-    }
+  __shared__ float dinv[P];
+  for (int e = threadIdx.x; e < P * P; e += kLrSolveThreads) Ls[e / P][e % P] = (float)Lg[e];
+  for (int i = threadIdx.x; i < P; i += kLrSolveThreads) {
+    const double d = Lg[i * P + i];
+    dinv[i] = d != 0.0 ? (float)(1.0 / d) : 0.f;
   }
+  __syncthreads();
+  const long long r = (long long)blockIdx.x * kLrSolveThreads + threadIdx.x;
+  if (r >= n) return;
+  float4 *row = reinterpret_cast<float4 *>(Y + r * P);
+  float y[P];
+#pragma unroll
+  for (int q = 0; q < P / 4; ++q) {
+    const float4 v = row[q];
+    y[4 * q] = v.x; y[4 * q + 1] = v.y; y[4 * q + 2] = v.z; y[4 * q + 3] = v.w;
+  }
+  // two partial sums per output halve the dependency chain
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    float s0 = y[i], s1 = 0.f;
+#pragma unroll
+    for (int k = 0; k + 1 < i; k += 2) {
+      s0 = fmaf(-Ls[i][k], y[k], s0);
+      s1 = fmaf(-Ls[i][k + 1], y[k + 1], s1);
+    }
+    if (i & 1) s0 = fmaf(-Ls[i][i - 1], y[i - 1], s0);
+    y[i] = (s0 + s1) * dinv[i];
+  }
+#pragma unroll
+  for (int q = 0; q < P / 4; ++q) row[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
 }
 
 // One CTA: eigen-decomposition of the symmetric G (sum of the partials) by
@@ -469,7 +478,7 @@ __global__ void __launch_bounds__(kLrThreads) lr_factor_kernel(
 
 namespace {
 struct LrLayout {
-  size_t X, Y, Z, mpart, part, linv, w, lam, total;
+  size_t X, Y, Z, mpart, part, chol, w, lam, total;
   int p, nparts;
 };
 int lr_p(int rank) { return rank + kLrOver <= 32 ? 32 : (rank + kLrOver <= 48 ? 48 : (rank + kLrOver <= 64 ? 64 : 80)); }
@@ -491,7 +500,7 @@ LrLayout lr_layout(int M, int K, int rank) {
   const size_t sl = (size_t)std::max((M + kLrSlice - 1) / kLrSlice, (K + kLrSlice - 1) / kLrSlice);
   L.mpart = take(sl * (size_t)std::max(M, K) * L.p * 4);   // split-product partials
   L.part = take((size_t)L.nparts * L.p * L.p * 8);
-  L.linv = take((size_t)L.p * L.p * 8);
+  L.chol = take((size_t)L.p * L.p * 8);
   L.w = take((size_t)L.p * L.p * 8);
   L.lam = take((size_t)L.p * 8);
   L.total = off;
@@ -505,7 +514,7 @@ cudaError_t lr_run(const LowrankArgs &a, const LrLayout &lay, cudaStream_t st, L
   float *Y = reinterpret_cast<float *>(ws + lay.Y);
   float *Z = reinterpret_cast<float *>(ws + lay.Z);
   double *part = reinterpret_cast<double *>(ws + lay.part);
-  double *linv = reinterpret_cast<double *>(ws + lay.linv);
+  double *chol = reinterpret_cast<double *>(ws + lay.chol);
   double *W = reinterpret_cast<double *>(ws + lay.w);
   double *lam = reinterpret_cast<double *>(ws + lay.lam);
   float *mpart = reinterpret_cast<float *>(ws + lay.mpart);
@@ -519,12 +528,12 @@ cudaError_t lr_run(const LowrankArgs &a, const LrLayout &lay, cudaStream_t st, L
       if ((err = L.launch("lr_gram", lr_gram_kernel<P>, dim3(np), dim3(kLrThreads), 0, st, false,
                           (const float *)B, n, part)) != cudaSuccess)
         return err;
-      if ((err = L.launch("lr_chol", lr_chol_kernel<P>, dim3(1), dim3(kLrThreads), dyn, st, false,
-                          (const double *)part, np, linv)) != cudaSuccess)
+      if ((err = L.launch("lr_chol", lr_chol_kernel<P>, dim3(1), dim3(kLrCholThreads), dyn, st,
+                          false, (const double *)part, np, chol)) != cudaSuccess)
         return err;
-      const int g = std::max(1, std::min((n + 31) / 32, 148 * 4));
-      if ((err = L.launch("lr_apply", lr_apply_linv_kernel<P>, dim3(g), dim3(kLrThreads), 0, st,
-                          false, B, n, (const double *)linv)) != cudaSuccess)
+      const int g = (n + kLrSolveThreads - 1) / kLrSolveThreads;
+      if ((err = L.launch("lr_apply", lr_apply_solve_kernel<P>, dim3(g), dim3(kLrSolveThreads), 0,
+                          st, false, B, n, (const double *)chol)) != cudaSuccess)
         return err;
     }
     return cudaSuccess;
