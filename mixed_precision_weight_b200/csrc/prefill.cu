@@ -317,7 +317,9 @@ __global__ void __launch_bounds__(256) pre_mat_kernel(PrefillParams p, long long
 }
 
 // ----------------------------------------------------------------- pre_gemm
-// Persistent: one CTA per SM walks output tiles (row tile fastest).  TMEM
+// Persistent: one CTA per SM walks output tiles, token tile fastest: a wave
+// of CTAs shares a few row tiles of A (each read from DRAM once) and all the
+// activation tiles, which are small enough to stay in L2 across waves.  TMEM
 // holds two accumulators of BN columns: the MMA warp fills one while the
 // epilogue warps drain the other (acc_full / acc_empty barriers).
 template <int BN>
@@ -328,6 +330,7 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
   uint8_t *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int A_STAGE = kPreBM * 128;
   constexpr int B_STAGE = BN * 128;
+  const int ntt = ntiles / nmt;      // token tiles
   uint8_t *sa = base;
   uint8_t *sb = base + kPreStages * A_STAGE;
   uint64_t *full = reinterpret_cast<uint64_t *>(sb + kPreStages * B_STAGE);
@@ -367,7 +370,7 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
       prefetch_tensormap(&mxc);
       long long gs = 0;                           // stage counter over all tiles
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % nmt) * kPreBM, n0 = (tile / nmt) * BN;
+        const int m0 = (tile / ntt) * kPreBM, n0 = (tile % ntt) * BN;
         for (int s = 0; s < S && ok; ++s, ++gs) {
           const int slot = (int)(gs % kPreStages);
           const uint32_t round = (uint32_t)(gs / kPreStages);
@@ -410,7 +413,7 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
     int li = 0;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++li) {
       const int ab = li & 1;
-      const int m0 = (tile % nmt) * kPreBM, n0 = (tile / nmt) * BN;
+      const int m0 = (tile / ntt) * kPreBM, n0 = (tile % ntt) * BN;
       if (!mbar_wait(&acc_full[ab], (li >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const int row = m0 + 32 * quarter + lane;
@@ -426,10 +429,13 @@ __global__ void __launch_bounds__(kPreThreads, 1) pre_gemm_kernel(
             const int tok = n0 + 16 * c + j;
             if (tok < p.T) {
               const float v = __uint_as_float(r[j]) + bv;
+              // streaming stores (evict-first): the output is written once and
+              // must not push the A and activation tiles out of L2
               if (p.y_bf16)
-                reinterpret_cast<uint16_t *>(p.y)[(size_t)tok * p.M + row] = f32_to_bf16_rn_bits(v);
+                __stcs(reinterpret_cast<unsigned short *>(p.y) + (size_t)tok * p.M + row,
+                       (unsigned short)f32_to_bf16_rn_bits(v));
               else
-                reinterpret_cast<float *>(p.y)[(size_t)tok * p.M + row] = v;
+                __stcs(reinterpret_cast<float *>(p.y) + (size_t)tok * p.M + row, v);
             }
           }
         }
