@@ -19,13 +19,15 @@
 #include "kernels.h"
 
 #include <algorithm>
+#include <cmath>
 
 namespace dvssq {
 
 constexpr int kLrOver = 16;          // oversampling p - r
 constexpr int kLrMaxP = 80;          // rank <= 64
-constexpr int kLrTile = 64;          // outputs (rows or columns of R) per CTA in the products
-constexpr int kLrSlice = 1024;       // inner-dimension slice per CTA in the products
+constexpr int kLrTile = 128;         // outputs (rows or columns of R) per CTA in the products
+constexpr int kLrSlice = 512;        // longest inner-dimension slice per CTA in the products
+constexpr int kLrMinSlice = 128;     // shortest
 constexpr int kLrChunk = 32;         // inner-dimension chunk staged in shared memory
 constexpr int kLrThreads = 256;
 constexpr int kLrGramRows = 128;     // rows per partial Gram matrix
@@ -48,11 +50,13 @@ __global__ void lr_gaussian_kernel(float *X, long long n, uint64_t seed) {
   }
 }
 
-// Split products with R, FP32 on the CUDA cores.  A CTA owns a tile of 64
+// Split products with R, FP32 on the CUDA cores.  A CTA owns a tile of 128
 // outputs (rows of R for R X, columns of R for R^T Q) x all p columns, over
-// one slice of kLrSlice along the inner dimension; each thread accumulates 4
-// outputs x p/16 columns (register blocking: one 16-byte load of R and p/16
-// of the small operand feed p/4 FMAs per step).  The next chunk of R and of the small operand is
+// one slice (a multiple of kLrChunk) along the inner dimension; thread (og, cg) = (tid / 8,
+// tid % 8) accumulates outputs 4 og .. 4 og + 3 x columns p/8 cg .. (register
+// blocking: one 16-byte load of R and p/8 values of the small operand feed
+// p/2 FMAs per step, and a warp's loads of a step are two shared-memory
+// wavefronts for 16 p FMAs).  The next chunk of R and of the small operand is
 // loaded into registers while the current chunk runs from shared memory.
 // Partial results go to part[slice][n][p], summed in slice order by
 // lr_reduce_kernel.
@@ -62,17 +66,18 @@ template <int P, int TRANS>
 __global__ void __launch_bounds__(kLrThreads) lr_mul_kernel(const float *__restrict__ R,
                                                             const float *__restrict__ B,
                                                             float *__restrict__ part, int M,
-                                                            int K) {
-  constexpr int PG = P / 16;                     // columns per thread
-  constexpr int RE = kLrChunk * kLrTile / kLrThreads;   // R values per thread and chunk (8)
+                                                            int K, int slice) {
+  constexpr int PG = P / 8;                      // columns per thread
+  static_assert(kLrThreads == 8 * (kLrTile / 4), "8 column groups x kLrTile / 4 output groups");
+  constexpr int RE = kLrChunk * kLrTile / kLrThreads;   // R values per thread and chunk (16)
   constexpr int XE = kLrChunk * P / kLrThreads;  // small-operand values per thread and chunk
   constexpr int RS = kLrTile + 8;                // padded row of the staged R chunk
   __shared__ __align__(16) float rs[kLrChunk][RS];      // [inner][out]
   __shared__ __align__(16) float bs[kLrChunk][P];
-  const int tid = threadIdx.x, og = tid >> 4, cg = tid & 15;
+  const int tid = threadIdx.x, og = tid >> 3, cg = tid & 7;
   const int n = TRANS ? K : M, inner = TRANS ? M : K;
   const int o0 = blockIdx.x * kLrTile;
-  const int t0 = blockIdx.y * kLrSlice, t1 = min(inner, t0 + kLrSlice);
+  const int t0 = blockIdx.y * slice, t1 = min(inner, t0 + slice);
   float acc[4][PG];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -119,8 +124,19 @@ __global__ void __launch_bounds__(kLrThreads) lr_mul_kernel(const float *__restr
       const float4 ra = *reinterpret_cast<const float4 *>(&rs[t][4 * og]);
       const float rv[4] = {ra.x, ra.y, ra.z, ra.w};
       float bv[PG];
+      if constexpr (PG % 4 == 0) {
 #pragma unroll
-      for (int j = 0; j < PG; ++j) bv[j] = bs[t][cg * PG + j];
+        for (int j = 0; j < PG; j += 4) {
+          const float4 b4 = *reinterpret_cast<const float4 *>(&bs[t][cg * PG + j]);
+          bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < PG; j += 2) {
+          const float2 b2 = *reinterpret_cast<const float2 *>(&bs[t][cg * PG + j]);
+          bv[j] = b2.x; bv[j + 1] = b2.y;
+        }
+      }
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -477,6 +493,13 @@ __global__ void __launch_bounds__(kLrThreads) lr_factor_kernel(
 }
 
 namespace {
+int lr_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
 struct LrLayout {
   size_t X, Y, Z, mpart, part, chol, w, lam, total;
   int p, nparts;
@@ -497,8 +520,11 @@ LrLayout lr_layout(int M, int K, int rank) {
   L.X = take((size_t)K * L.p * 4);          // X, then Z and Bt (K x p)
   L.Y = take((size_t)M * L.p * 4);          // Y / Q (M x p)
   L.Z = take((size_t)K * L.p * 4);          // Z (K x p)
-  const size_t sl = (size_t)std::max((M + kLrSlice - 1) / kLrSlice, (K + kLrSlice - 1) / kLrSlice);
-  L.mpart = take(sl * (size_t)std::max(M, K) * L.p * 4);   // split-product partials
+  // split-product partials: at most one slice per kLrMinSlice of the inner
+  // dimension for either product
+  const size_t rows = std::max((size_t)((K + kLrMinSlice - 1) / kLrMinSlice) * M,
+                               (size_t)((M + kLrMinSlice - 1) / kLrMinSlice) * K);
+  L.mpart = take(rows * L.p * 4);
   L.part = take((size_t)L.nparts * L.p * L.p * 8);
   L.chol = take((size_t)L.p * L.p * 8);
   L.w = take((size_t)L.p * L.p * 8);
@@ -541,9 +567,26 @@ cudaError_t lr_run(const LowrankArgs &a, const LrLayout &lay, cudaStream_t st, L
   // out = R in (TRANS 0, n = M) or R^T in (TRANS 1, n = K), split along the
   // inner dimension, then the slices summed in order
   auto mul = [&](auto kern, const float *in, float *out, int n, int inner) -> cudaError_t {
-    const int ns = (inner + kLrSlice - 1) / kLrSlice;
-    cudaError_t err = L.launch("lr_mul", kern, dim3((n + kLrTile - 1) / kLrTile, ns),
-                               dim3(kLrThreads), 0, st, false, a.R, in, mpart, M, K);
+    // slice length: a multiple of kLrChunk in [kLrMinSlice, kLrSlice] (the
+    // workspace holds the partials of the shortest), chosen so that the CTAs fill
+    // whole waves of the resident slots as nearly as possible
+    int occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kLrThreads, 0) != cudaSuccess ||
+        occ < 1)
+      occ = 1;
+    const double slots = (double)lr_sm_count() * occ;
+    const int tiles = (n + kLrTile - 1) / kLrTile;
+    int best = kLrSlice;
+    double best_eff = -1.0;
+    for (int sl = kLrMinSlice; sl <= kLrSlice; sl += kLrChunk) {
+      const int ns = (inner + sl - 1) / sl;
+      const double waves = tiles * (double)ns / slots;
+      const double eff = waves / std::ceil(waves);
+      if (eff > best_eff + 1e-9) { best_eff = eff; best = sl; }
+    }
+    const int ns = (inner + best - 1) / best;
+    cudaError_t err = L.launch("lr_mul", kern, dim3(tiles, ns), dim3(kLrThreads), 0, st, false,
+                               a.R, in, mpart, M, K, best);
     if (err != cudaSuccess) return err;
     const long long cnt = (long long)n * P;
     return L.launch("lr_reduce", lr_reduce_kernel, dim3(148 * 4), dim3(256), 0, st, false,
