@@ -81,6 +81,10 @@ def kernel_bytes(name, M, K, rank, n_sal, T):
 
 # The source files each kernel is built from: a recorded DRAM count stays valid
 # while these files are unchanged.
+# Roofline bars of the task: the decode GEMV kernels at 0.70 of measured HBM,
+# the prefill GEMM at 0.50 of the measured BF16 tensor peak.
+ROOFLINE_TARGETS = {"dec_row": 0.70, "dec_main": 0.70, "mlp_stack": 0.70, "pre_gemm": 0.50}
+
 KERNEL_SOURCES = {
     "enc_pass1": ("encode.cu", "fwht_group.cuh", "exact_sum.cuh"),
     "enc_pass2": ("encode.cu", "fwht_group.cuh", "exact_sum.cuh"),
@@ -998,6 +1002,11 @@ def measure(work, dv, torch, steps, warmup, world, device, local, key, use_graph
                     "frac": round(achieved / pk["hbm_gbs"], 4),
                     "traffic": dram_traffic(dom, key),
                     "algorithmic_bytes_per_launch": db}
+    # the task's bars: decode GEMV >= 0.70 of HBM, prefill GEMM >= 0.50 of the BF16 peak
+    target = ROOFLINE_TARGETS.get(dom)
+    if target is not None:
+        roofline["target_frac"] = target
+        roofline["frac_of_target"] = round(roofline["frac"] / target, 4)
     return dict(ms_step=ms_step, value=value, unit=unit, bytes_step=bytes_step, kernels=kernels,
                 roofline=roofline, launches=launches_measured, err=err, clocks=clk.summary(),
                 W=W, barrier=barrier, stream=stream)
