@@ -22,6 +22,8 @@
 //     accumulator of lane (g, q) holds row g's columns 8t + 2q + e, so the
 //     butterflies over e and t stay in registers and the two over q are quad
 //     shuffles; then the 1/sqrt(b) scale, BF16 rounding and 4-byte stores.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -35,6 +37,35 @@ constexpr int kMatRows = 8;                         // rows per warp tile
 constexpr int kMatRowsCta = kMatRows * kMatWarps;   // rows per CTA item
 constexpr int kMatMaxRank = 64;
 constexpr int kMatURow = kMatMaxRank * 2 + 16;      // U bytes per staged row (padded)
+
+// Packed FP32x2 arithmetic (sm_100a): two independent round-to-nearest
+// operations per instruction.
+__device__ __forceinline__ unsigned long long mat_f2u(float2 a) {
+  return (unsigned long long)__float_as_uint(a.x) | ((unsigned long long)__float_as_uint(a.y) << 32);
+}
+__device__ __forceinline__ float2 mat_u2f(unsigned long long u) {
+  return make_float2(__uint_as_float((uint32_t)u), __uint_as_float((uint32_t)(u >> 32)));
+}
+__device__ __forceinline__ float2 mat_add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(mat_f2u(a)), "l"(mat_f2u(b)));
+  return mat_u2f(r);
+}
+__device__ __forceinline__ float2 mat_sub2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(mat_f2u(a)), "l"(mat_f2u(b)));
+  return mat_u2f(r);
+}
+__device__ __forceinline__ float2 mat_mul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(mat_f2u(a)), "l"(mat_f2u(b)));
+  return mat_u2f(r);
+}
+__device__ __forceinline__ float2 mat_fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(mat_f2u(a)), "l"(mat_f2u(b)), "l"(mat_f2u(c)));
+  return mat_u2f(r);
+}
 
 __device__ __forceinline__ void mat_cp_async(void *smem, const void *gmem, int bytes) {
   if (bytes == 16)
@@ -264,41 +295,49 @@ __global__ void __launch_bounds__(kMatThreads, 3) materialize_kernel(const MatPa
       }
     }
     // Walsh-Hadamard transform along the b columns: bit 0 (e) and bits 3..
-    // (t) in registers, bits 1 and 2 (q) across the quad
+    // (t) in registers, bits 1 and 2 (q) across the quad.  After the e stage
+    // the (e = 0, 1) pair of every t runs as one packed FP32x2 operation; a
+    // quad stage is o + (+-1) v by one packed FMA (v times +-1 is exact, so
+    // the single rounding equals that of the scalar add or subtract).
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const float a0 = acc[t][0], a1 = acc[t][1];
       acc[t][0] = a0 + a1;
       acc[t][1] = a0 - a1;
     }
+    float2 v[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) v[t] = make_float2(acc[t][0], acc[t][1]);
 #pragma unroll
     for (int m = 1; m <= 2; m <<= 1) {
-      const bool upper = (q & m) != 0;
+      const float sg = (q & m) ? -1.0f : 1.0f;
+      const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float o = __shfl_xor_sync(0xffffffffu, acc[t][e], m);
-          acc[t][e] = upper ? o - acc[t][e] : acc[t][e] + o;
-        }
+      for (int t = 0; t < NT; ++t) {
+        float2 o;
+        o.x = __shfl_xor_sync(0xffffffffu, v[t].x, m);
+        o.y = __shfl_xor_sync(0xffffffffu, v[t].y, m);
+        v[t] = mat_fma2(v[t], sg2, o);
+      }
     }
 #pragma unroll
     for (int h = 1; h < NT; h <<= 1)
 #pragma unroll
       for (int t = 0; t < NT; ++t)
-        if (!(t & h))
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float a0 = acc[t][e], a1 = acc[t + h][e];
-            acc[t][e] = a0 + a1;
-            acc[t + h][e] = a0 - a1;
-          }
+        if (!(t & h)) {
+          const float2 a0 = v[t], a1 = v[t + h];
+          v[t] = mat_add2(a0, a1);
+          v[t + h] = mat_sub2(a0, a1);
+        }
     if (row < p.M) {
       uint32_t *dst = reinterpret_cast<uint32_t *>(p.W + (size_t)row * p.K + (size_t)kb * B) + q;
+      const float2 c2 = make_float2(p.c, p.c);
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
-        dst[4 * t] = (uint32_t)f32_to_bf16_rn_bits(acc[t][0] * p.c) |
-                     ((uint32_t)f32_to_bf16_rn_bits(acc[t][1] * p.c) << 16);
+      for (int t = 0; t < NT; ++t) {
+        const float2 w = mat_mul2(v[t], c2);
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(w.x, w.y);   // .x in the low half
+        dst[4 * t] = *reinterpret_cast<const uint32_t *>(&hb);
+      }
     }
     __syncwarp();
   }
