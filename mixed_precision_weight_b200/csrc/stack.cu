@@ -20,15 +20,18 @@
 //     through a ring of shared-memory slots (bulk copies of q4, s4, q8 and U
 //     rows per row tile).  Nothing it reads depends on activations, so it
 //     runs ahead across layer boundaries while the consumers wait.
-//   * The 15 consumer warps run two phases per block, each ending in a grid
-//     barrier: gate+up (x -> h) and down (h -> x).  After a barrier every CTA
+//   * The other 11 (consumer) warps run two phases per block, each ending in
+//     a grid barrier: gate+up (x -> h) and down (h -> x).  After a barrier every CTA
 //     reads the whole input vector, rotates it (one warp per Hadamard block,
 //     FP32 butterflies in registers and shuffles) into int16 with one scale
 //     per 64 columns, requantises the salient entries per 32-entry chunk, and
 //     runs its rows as exact int32 dot products by DP2A: even columns as
 //     bytes q + 8 (minus 8 times the unit's even-column activation sum), odd
 //     columns as the high nibble masked in place, a signed byte equal to
-//     16 q (the sum divided by 16 exactly); scaled per group in FP32.
+//     16 q (the sum divided by 16 exactly); scaled per group in FP32.  The
+//     row work is cut into items (rows x rounds of 32-column lane tasks) that
+//     the warps take from a shared counter; the warp that completes a tile's
+//     last item frees its ring slot.
 //   * The rank-r term needs t = V (H x) = (V H) x for all of x.  With
 //     (V H) precomputed once in FP32, each CTA adds the share of the entries
 //     it produced, t_c = (V H)[:, own] x[own], at the end of the producing
