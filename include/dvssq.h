@@ -363,9 +363,9 @@ typedef struct {
  * Supported stacks: every gate/up is inter x hidden and every down hidden x
  * inter with one Hadamard block size; hidden and inter multiples of 512;
  * n_sal a multiple of 32; rank a multiple of 8 and at most 32; and rows
- * small enough that the shared-memory weight ring holds at least one slot
- * per consumer warp (11; two rows of the down matrix per slot at least: the
- * Spark shapes, hidden 2560 / inter 10240, fit 11 slots of 13.8 KB).
+ * small enough that the shared-memory weight ring holds at least two slots
+ * (two rows of the down matrix per slot at least: the Spark shapes, hidden
+ * 2560 / inter 10240, fit 12 slots of 13.8 KB).
  * Others return UNSUPPORTED_SHAPE.                                         */
 DVSSQ_API dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers,
                                                       int32_t n_layers, size_t *bytes);

@@ -20,7 +20,7 @@
 //     through a ring of shared-memory slots (bulk copies of q4, s4, q8 and U
 //     rows per row tile).  Nothing it reads depends on activations, so it
 //     runs ahead across layer boundaries while the consumers wait.
-//   * The other 11 (consumer) warps run two phases per block, each ending in
+//   * The other 15 (consumer) warps run two phases per block, each ending in
 //     a grid barrier: gate+up (x -> h) and down (h -> x).  After a barrier every CTA
 //     reads the whole input vector, rotates it (one warp per Hadamard block,
 //     FP32 butterflies in registers and shuffles) into int16 with one scale
@@ -31,7 +31,8 @@
 //     16 q (the sum divided by 16 exactly); scaled per group in FP32.  The
 //     row work is cut into items (rows x rounds of 32-column lane tasks) that
 //     the warps take from a shared counter; the warp that completes a tile's
-//     last item frees its ring slot.
+//     last item frees its ring slot, and a warp ahead of the ring waits for
+//     its tile by the slot's tag as well as the mbarrier's parity.
 //   * The rank-r term needs t = V (H x) = (V H) x for all of x.  With
 //     (V H) precomputed once in FP32, each CTA adds the share of the entries
 //     it produced, t_c = (V H)[:, own] x[own], at the end of the producing
@@ -49,7 +50,7 @@
 
 namespace dvssq {
 
-constexpr int kStkWarps = 12;
+constexpr int kStkWarps = 16;
 constexpr int kStkThreads = 32 * kStkWarps;
 constexpr int kStkCons = kStkWarps - 1;           // consumer warps (warp 0 streams weights)
 constexpr int kStkConsThreads = 32 * kStkCons;
@@ -102,6 +103,39 @@ __device__ __forceinline__ bool stk_wait(uint64_t *bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64(), lim = wait_limit();
   while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > lim) {
+      set_error(kErrWaitMbarrier);
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+// The same wait for a ring slot that also requires the slot's tile tag: the
+// parity of an mbarrier cannot tell tile T from tile T - 2 NS, the tag can,
+// so consumer warps may run ahead of the ring by more than a turn.  The
+// producer writes a slot's tag only after the slot's previous tile was freed,
+// and the tag is read (acquire) before the parity is tested: a tag equal to
+// the wanted tile means the phases before it have completed, so the parity
+// then names this tile's phase alone.
+__device__ __forceinline__ int stk_tag_acquire(const int *tag) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];"
+               : "=r"(v)
+               : "r"(smem_u32(tag))
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool stk_wait_tile(uint64_t *bar, uint32_t parity, const int *tag,
+                                              int want, volatile int *abort) {
+  auto ready = [&]() { return stk_tag_acquire(tag) == want && mbar_try_wait(bar, parity); };
+  if (ready()) return true;
+  const long long t0 = clock64(), lim = wait_limit();
+  while (!ready()) {
     if (*abort) return false;
     if (clock64() - t0 > lim) {
       set_error(kErrWaitMbarrier);
@@ -298,6 +332,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   int *s_grab = reinterpret_cast<int *>(base + p.o_grab);        // next item of the phase
   StkPhase *sph = reinterpret_cast<StkPhase *>(base + p.o_ph);  // the current phase
   int *s_done = s_grab + 1;                                       // [nslots] items done per slot
+  int *s_tag = s_done + kStkMaxSlots;                             // [nslots] tile held per slot
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = p.G;
@@ -309,6 +344,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       s_done[s] = 0;
+      s_tag[s] = -1;
     }
     fence_mbarrier_init();
     *abort = 0;
@@ -338,6 +374,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
             uint8_t *dst = ring + (size_t)s * p.slot_bytes;
             const uint32_t bq = nr * kq, bs = nr * ks, b8 = nr * (uint32_t)m.n_sal;
             const uint32_t bu = nr * (uint32_t)m.r * 2u;
+            *(volatile int *)&s_tag[s] = (int)seq;
             mbar_arrive_expect_tx(&full[s], bq + bs + b8 + bu);
             bulk_g2s(dst, m.q4 + (size_t)i0 * kq, bq, &full[s]);
             bulk_g2s(dst + bq, reinterpret_cast<const uint8_t *>(m.s4) + (size_t)i0 * ks, bs,
@@ -643,10 +680,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     // RR rounds of one tile (RG = 4 for three-round items when the tile's rows
     // allow it, else 2).  The consumer warps take items from a shared
     // counter in (matrix, tile, item) order, which is the ring's order; the
-    // warp that completes a tile's last item frees its ring slot.  With at
-    // least as many slots as consumer warps, a warp never takes an item of a
-    // tile whose slot still holds the tile one ring turn earlier (the items
-    // of the slots in between would need more warps than there are).
+    // warp that completes a tile's last item frees its ring slot.  A warp
+    // that takes an item of a tile whose slot still holds an earlier tile
+    // waits for the slot's tag (stk_wait_tile).
     {
       // four-row items where the tile's rows allow it and every matrix of the
       // phase takes three-round items (three item shapes in all)
@@ -680,8 +716,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         const int tile = g / ipt, it = g - tile * ipt;
         const uint32_t tseq = seq + (uint32_t)((mi ? ntl_[0] : 0) + tile);
         const int s = (int)(tseq % (uint32_t)NS);
-        const bool got =
-            __all_sync(0xffffffffu, stk_wait(&full[s], (tseq / (uint32_t)NS) & 1u, abort));
+        const bool got = __all_sync(
+            0xffffffffu, stk_wait_tile(&full[s], (tseq / (uint32_t)NS) & 1u, s_tag + s, (int)tseq, abort));
         const int i0 = ph.a + tile * ph.tr;
         const int nr = min(ph.tr, ph.b - i0);
         const int nsal = mi ? nsal_[1] : nsal_[0], Km = mi ? K_[1] : K_[0];
@@ -878,14 +914,12 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
     p.o_vhs = take(std::max(max_rank * rg, 2 * max_rank * rd) * 4);
   }
   p.o_flag = take(16);
-  p.o_grab = take((1 + kStkMaxSlots) * 4);
+  p.o_grab = take((1 + 2 * kStkMaxSlots) * 4);
   p.o_ph = take((int)sizeof(StkPhase));
   const int fixed = off;
   const int room = kStkSmemLimit - 1024 - fixed - 2 * kStkMaxSlots * 8 - 128;
   p.nslots = std::min(kStkMaxSlots, room / p.slot_bytes);
-  // the consumer warps take items from a shared counter: a slot per warp at
-  // least keeps every taken item on the ring turn it waits for
-  if (p.nslots < kStkCons) return false;
+  if (p.nslots < 2) return false;
   p.o_full = take(p.nslots * 8);
   p.o_empty = take(p.nslots * 8);
   off = (off + 1023) & ~1023;
