@@ -56,6 +56,7 @@ constexpr int kStkCons = kStkWarps - 1;           // consumer warps (warp 0 stre
 constexpr int kStkConsThreads = 32 * kStkCons;
 constexpr int kStkMaxRank = 32;                   // rank <= 32: one U t term per lane
 constexpr int kStkMaxSlots = 24;
+constexpr int kStkShareRegs = 5;                 // t shares per lane and pair: G <= 160
 
 __device__ __forceinline__ void stk_consumer_sync() {
   asm volatile("bar.sync 2, %0;" ::"n"(kStkConsThreads) : "memory");
@@ -70,12 +71,16 @@ struct StackParams {
   const uint16_t *x;              // BF16 [H]
   uint16_t *y;                    // BF16 [H]: the running hidden state, then the output
   uint16_t *h;                    // BF16 [I]
-  float *tp;                      // t shares [3][kStkMaxRank][G]: gate, up, down
+  float *tp;                      // t shares [3][kStkMaxRank][Gp]: gate, up, down
   unsigned int *gbar;             // grid barrier counter, zero at launch
   // shared-memory offsets from the 1024-aligned base
   int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
       o_flag, o_grab, o_ph, o_vhs, smem_total;
 };
+
+// Stride of the t shares of one (matrix, rank index) pair: G rounded up to
+// whole 16-byte words, so that each pair's shares copy as 16-byte chunks.
+__host__ __device__ constexpr int stk_gp(int G) { return (G + 3) & ~3; }
 
 // Entries per matrix of the BF16 s8 staging: the own rows plus the partial
 // 16-byte words at both ends, rounded up to whole words.
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         for (int i = lane; i < n; i += 32) s = fmaf(row[i], vals[i], s);
 #pragma unroll
         for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) p.tp[((size_t)ph.oslot[j] * kStkMaxRank + k) * G + c] = s;
+        if (lane == 0) p.tp[((size_t)ph.oslot[j] * kStkMaxRank + k) * stk_gp(G) + c] = s;
       }
       off += ph.orank[j] * n;
     }
@@ -513,58 +518,30 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   auto run_phase = [&](const StkPhase &ph) {
     const int K = ph.K, nrows = ph.b - ph.a;
     if (ctid == 0) *s_grab = 0;    // the previous phase's rows ended before its last barrier
-    // input vector and t: the G shares of each (matrix, k), NP parts per
-    // pair summed in parallel, then the parts in order
-    // the input vector, four 16-byte loads per thread in flight at once (its
-    // producers are other CTAs: the loads go to L2 after the grid barrier)
-    for (int i0 = ctid; i0 < K / 8; i0 += 4 * kStkConsThreads) {
-      uint4 xv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * kStkConsThreads;
-        if (i < K / 8) xv[u] = __ldcg(reinterpret_cast<const uint4 *>(ph.src) + i);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * kStkConsThreads;
-        if (i < K / 8) reinterpret_cast<uint4 *>(xi)[i] = xv[u];
-      }
-    }
-    // t = the sum of the G CTAs' shares of each (matrix, rank index) pair.
-    // A warp takes up to four pairs (q = cw + 15 i); its lanes read the
-    // shares at lane + 32 u (coalesced, every load in flight at once), add
-    // them in u order and then by a fixed shuffle tree: deterministic.
+    // The input vector comes in by cp.async (the rotation waits for it); the
+    // G shares of each (matrix, rank index) pair are loaded into registers
+    // now and summed after the rotation and the salient step, so that their
+    // latency hides behind both.  Both were written by other CTAs before the
+    // grid barrier: the loads read L2 (.cg).  Warp cw takes the pairs
+    // q = cw + kStkCons i; its lanes hold the shares at lane + 32 u.
     const int r0m = ph.m[0].r, npair = r0m + (ph.nm > 1 ? ph.m[1].r : 0);
-    {
-      constexpr int QW = (2 * kStkMaxRank + kStkCons - 1) / kStkCons;   // pairs per warp
-      constexpr int UW = 8;                                              // G <= 256
-      float v[QW][UW];
+    const int Gp = stk_gp(G);
+    for (int i = ctid; i < K / 8; i += kStkConsThreads) stk_cp_async16(xi + 8 * i, ph.src + 8 * i);
+    stk_cp_async_commit();
+    constexpr int QW = (2 * kStkMaxRank + kStkCons - 1) / kStkCons;   // pairs per warp
+    float tsv[QW][kStkShareRegs];
 #pragma unroll
-      for (int i = 0; i < QW; ++i) {
-        const int q = cw + kStkCons * i;
-        const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
-        const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * G;
+    for (int i = 0; i < QW; ++i) {
+      const int q = cw + kStkCons * i;
+      const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
+      const float *src = p.tp + ((size_t)ph.tslot[mi] * kStkMaxRank + k) * Gp;
 #pragma unroll
-        for (int u = 0; u < UW; ++u) {
-          const int j = lane + 32 * u;
-          v[i][u] = (q < npair && j < G) ? __ldcg(src + j) : 0.0f;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < QW; ++i) {
-        float sum = 0.0f;
-#pragma unroll
-        for (int u = 0; u < UW; ++u) sum += v[i][u];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const int q = cw + kStkCons * i;
-        if (lane == 0 && q < npair) {
-          const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
-          tv[mi * kStkMaxRank + k] = sum;
-        }
+      for (int u = 0; u < kStkShareRegs; ++u) {
+        const int j = lane + 32 * u;
+        tsv[i][u] = (q < npair && j < G) ? __ldcg(src + j) : 0.0f;
       }
     }
-    stk_cp_async_wait_all();             // this phase's prefetched s8 and salient indices
+    stk_cp_async_wait_all();             // the prefetched s8 and salient indices, and x
     stk_consumer_sync();
 
     // rotate x: BF16 in, int16 (unit/chunk layout) with one scale per 64
@@ -671,6 +648,21 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         xsal[mi * p.max_nsal + 32 * j + 8 * stk_chunk(j, lane >> 3) + (lane & 7)] =
             (uint16_t)(qv & 0xFFFF);
         if (lane == 0) xss[mi * (p.max_nsal / 32) + j] = mx * (1.0f / 32767.0f);
+      }
+    }
+    // t = the sum of the G shares of each pair, in u order and then by a
+    // fixed shuffle tree (deterministic)
+#pragma unroll
+    for (int i = 0; i < QW; ++i) {
+      const int q = cw + kStkCons * i;
+      float sum = 0.0f;
+#pragma unroll
+      for (int u = 0; u < kStkShareRegs; ++u) sum += tsv[i][u];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0 && q < npair) {
+        const int mi = q < r0m ? 0 : 1, k = q - (mi ? r0m : 0);
+        tv[mi * kStkMaxRank + k] = sum;
       }
     }
     stk_consumer_sync();
@@ -790,7 +782,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         for (int i = lane; i < n; i += 32) sacc = fmaf(__ldg(row + i), vals[i], sacc);
 #pragma unroll
         for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
-        if (lane == 0) p.tp[((size_t)j * kStkMaxRank + k) * G + c] = sacc;
+        if (lane == 0) p.tp[((size_t)j * kStkMaxRank + k) * stk_gp(G) + c] = sacc;
       }
     }
   }
@@ -861,7 +853,7 @@ StkWs stk_ws_layout(const StackShapeInfo &si, int L, int G) {
   };
   w.desc = take((size_t)L * sizeof(StackLayerDesc));
   w.vh = take(si.vh_floats * sizeof(float));
-  w.tp = take((size_t)3 * kStkMaxRank * G * sizeof(float));
+  w.tp = take((size_t)3 * kStkMaxRank * stk_gp(G) * sizeof(float));
   w.gbar = take(256);
   w.h = take((size_t)si.I * 2);
   w.total = off;
@@ -869,7 +861,7 @@ StkWs stk_ws_layout(const StackShapeInfo &si, int L, int G) {
 }
 
 bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
-  if (G < 1 || G > 256) return false;        // the t-share sums read at most 256 shares
+  if (G < 1 || G > 32 * kStkShareRegs) return false;   // t shares a lane holds in registers
   const int L = (int)Ls.size();
   p.L = L;
   p.H = Ls[0].m[2].M;
