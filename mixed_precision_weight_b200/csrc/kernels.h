@@ -125,7 +125,7 @@ cudaError_t prepare_encode_kernels();
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t st, Launcher &L);
 
 // ------------------------------------------------------------- MLP stack ---
-struct StackMatDesc {           // one packed matrix (device pointers)
+struct alignas(16) StackMatDesc {   // one packed matrix (device pointers)
   const uint8_t *q4;
   const uint16_t *s4;
   const int32_t *sal_idx;

@@ -61,6 +61,12 @@ constexpr int kStkShareRegs = 5;                 // t shares per lane and pair: 
 __device__ __forceinline__ void stk_consumer_sync() {
   asm volatile("bar.sync 2, %0;" ::"n"(kStkConsThreads) : "memory");
 }
+// Barrier among consumer warps 1.. only: they prepare the next phase while
+// consumer warp 0 waits at the grid barrier.
+constexpr int kStkPrepThreads = kStkConsThreads - 32;
+__device__ __forceinline__ void stk_prep_sync() {
+  asm volatile("bar.sync 3, %0;" ::"n"(kStkPrepThreads) : "memory");
+}
 
 struct StackParams {
   const StackLayerDesc *layers;   // [L] in device memory
@@ -75,7 +81,7 @@ struct StackParams {
   unsigned int *gbar;             // grid barrier counter, zero at launch
   // shared-memory offsets from the 1024-aligned base
   int o_ring, o_full, o_empty, o_xi, o_xsc, o_xs8, o_xs, o_xss, o_sidx, o_t, o_s8, o_yv, o_vh,
-      o_flag, o_grab, o_ph, o_vhs, smem_total;
+      o_flag, o_grab, o_ph, o_ld, o_vhs, smem_total;
 };
 
 // Stride of the t shares of one (matrix, rank index) pair: G rounded up to
@@ -336,6 +342,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   volatile int *abort = reinterpret_cast<volatile int *>(base + p.o_flag);
   int *s_grab = reinterpret_cast<int *>(base + p.o_grab);        // next item of the phase
   StkPhase *sph = reinterpret_cast<StkPhase *>(base + p.o_ph);  // the current phase
+  StackLayerDesc *sld = reinterpret_cast<StackLayerDesc *>(base + p.o_ld);  // layers l, l + 1 at [l & 1]
   int *s_done = s_grab + 1;                                       // [nslots] items done per slot
   int *s_tag = s_done + kStkMaxSlots;                             // [nslots] tile held per slot
 
@@ -427,14 +434,29 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     return *s_live != 0;
   };
 
+  // Layer descriptors of layers l and l + 1 sit in shared memory (slot l & 1),
+  // copied by cp.async a phase ahead, so that building a phase descriptor at
+  // a grid barrier reads no global memory.
+  static_assert(sizeof(StackLayerDesc) % 16 == 0, "layer descriptors copy as 16-byte chunks");
+  auto fetch_layer = [&](int l) {
+    constexpr int n16 = (int)(sizeof(StackLayerDesc) / 16);
+    if (ctid < n16)
+      stk_cp_async16(reinterpret_cast<uint4 *>(sld + (l & 1)) + ctid,
+                     reinterpret_cast<const uint4 *>(p.layers + l) + ctid);
+    stk_cp_async_commit();
+  };
+
   // phase descriptors: layer l, kind 0 = gate and up (x -> h), 1 = down (h -> x).
   // One thread writes the descriptor to shared memory and the consumers read
   // it there: a per-thread copy would live in local memory, whose lines the
   // small L1 (shared memory takes the rest) loses to L2 between uses.
-  auto set_phase = [&](int l, int kind) {
-    if (ctid == 0) {
+  // `prep`: written by the first thread of consumer warp 1 and published to
+  // warps 1.. only (the grid-barrier path); else by consumer thread 0 to all.
+  auto set_phase = [&](int l, int kind, bool prep) {
+    if (ctid == (prep ? 32 : 0)) {
       StkPhase &ph = *sph;
-      const StackLayerDesc *Ld = p.layers + l;
+      const StackLayerDesc *Ld = sld + (l & 1);
+      const StackLayerDesc *Ln = sld + ((l + 1) & 1);
       if (kind == 0) {
         ph.nm = 2;
         ph.m[0] = Ld->m[0];
@@ -462,33 +484,35 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         ph.tslot[0] = 2;
         ph.nout = l + 1 < p.L ? 2 : 0;
         for (int j = 0; j < ph.nout; ++j) {
-          ph.ovh[j] = Ld[1].m[j].vh;
-          ph.oK[j] = Ld[1].m[j].K;
-          ph.orank[j] = Ld[1].m[j].r;
+          ph.ovh[j] = Ln->m[j].vh;
+          ph.oK[j] = Ln->m[j].K;
+          ph.orank[j] = Ln->m[j].r;
           ph.oslot[j] = j;
         }
       }
     }
-    stk_consumer_sync();
+    if (prep) stk_prep_sync();
+    else stk_consumer_sync();
   };
 
   // weight-side data of a phase, loaded while the grid barrier is pending:
   // INT8 scales of the own rows, salient indices, (V H) columns for the t shares
-  auto prefetch = [&](const StkPhase &ph) {
-    const int n = ph.b - ph.a;
+  // issued by threads t0.. of the consumers, nth of them
+  auto prefetch = [&](const StkPhase &ph, int t0, int nth) {
+    const int n = ph.b - ph.a, tt = ctid - t0;
     for (int mi = 0; mi < ph.nm; ++mi) {
       const StackMatDesc &m = ph.m[mi];
       if (m.n_sal == 0) continue;
       // the 16-byte words of s8 that hold rows [a, b) (M is a multiple of 8)
       const int w0 = ph.a >> 3, w1 = (ph.b + 7) >> 3;
-      for (int w = w0 + ctid; w < w1; w += kStkConsThreads)
+      for (int w = w0 + tt; w < w1; w += nth)
         stk_cp_async16(s8c + mi * s8_stride + 8 * (w - w0), m.s8 + 8 * w);
-      for (int e = 4 * ctid; e < m.n_sal; e += 4 * kStkConsThreads)
+      for (int e = 4 * tt; e < m.n_sal; e += 4 * nth)
         stk_cp_async16(sidx + mi * p.max_nsal + e, m.sal_idx + e);
     }
     int off = 0;
     for (int j = 0; j < ph.nout; ++j) {
-      for (int q = ctid; q < ph.orank[j] * n; q += kStkConsThreads) {
+      for (int q = tt; q < ph.orank[j] * n; q += nth) {
         const int k = q / n, i = q - k * n;
         stk_cp_async4(vhs + off + q, ph.ovh[j] + (size_t)k * ph.oK[j] + ph.a + i);
       }
@@ -767,9 +791,13 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   };
 
   // ---- prologue: t shares of layer 0's gate and up from x, entries [d_a, d_b)
-  set_phase(0, 0);
+  fetch_layer(0);
+  if (p.L > 1) fetch_layer(1);
+  stk_cp_async_wait_all();
+  stk_consumer_sync();
+  set_phase(0, 0, false);
   const StkPhase &ph = *sph;
-  prefetch(ph);
+  prefetch(ph, 0, kStkConsThreads);
   {
     const int n = d_b - d_a;
     for (int i = ctid; i < n; i += kStkConsThreads) vals[i] = bf16_bits_to_f32(p.x[d_a + i]);
@@ -795,6 +823,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
   // within the instruction caches).
   for (int step = 0; step < 2 * p.L; ++step) {
     const int l = step >> 1, kind = step & 1;
+    // layer l + 1 into the slot of layer l - 1, whose last phase descriptor
+    // was built at the previous barrier; it lands before this phase's rows
+    if (kind == 0 && l >= 1 && l + 1 < p.L && live) fetch_layer(l + 1);
     if (live) run_phase(ph);
     if (kind == 0) {
       // h = RN_bf16(gelu(g) u), g and u rounded to BF16 first
@@ -820,8 +851,12 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     if (step + 1 == 2 * p.L) break;     // the last block's output needs no t shares
     if (live) t_share_out(ph);
     grid_arrive();
-    set_phase(kind == 0 ? l : l + 1, kind ^ 1);
-    prefetch(ph);
+    // consumer warp 0 goes straight to the wait (its thread 0 polls); the
+    // other warps build the next phase's descriptor and issue its prefetch
+    if (cw >= 1) {
+      set_phase(kind == 0 ? l : l + 1, kind ^ 1, true);
+      prefetch(ph, 32, kStkPrepThreads);
+    }
     live = grid_wait() && live;
   }
 }
@@ -908,6 +943,7 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
   p.o_flag = take(16);
   p.o_grab = take((1 + 2 * kStkMaxSlots) * 4);
   p.o_ph = take((int)sizeof(StkPhase));
+  p.o_ld = take(2 * (int)sizeof(StackLayerDesc));
   const int fixed = off;
   const int room = kStkSmemLimit - 1024 - fixed - 2 * kStkMaxSlots * 8 - 128;
   p.nslots = std::min(kStkMaxSlots, room / p.slot_bytes);
