@@ -179,6 +179,10 @@ struct StkPhase {
   int nout;
   const float *ovh[2];
   int oK[2], orank[2], oslot[2];
+  // the rows' item plan (stk_plan_items): rows per item, items in all, and
+  // per matrix its items, items per tile, tiles, round groups and rounds
+  // per item
+  int rg, total, tot[2], ipt[2], ntl[2], nrg[2], rr[2];
 };
 
 __device__ __forceinline__ void stk_cp_async4(void *smem, const void *gmem) {
@@ -320,6 +324,30 @@ __device__ __forceinline__ void stk_item(const StkTileArgs a, int it, int lane) 
 __host__ __device__ __forceinline__ int stk_rr(int rounds) {
   const int n = (rounds + 3) / 4;
   return max(3, (rounds + n - 1) / n);
+}
+
+// The item plan of a phase, computed once by the thread that writes its
+// descriptor.  RG = 4 rows per item where the tile's rows allow it and every
+// matrix of the phase takes three-round items (three item shapes in all).
+__device__ __forceinline__ void stk_plan_items(StkPhase &ph) {
+  const int nrows = ph.b - ph.a;
+  int RG = ph.tr % 4 == 0 ? 4 : 2;
+  for (int mi = 0; mi < ph.nm; ++mi)
+    if (stk_rr((ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32) != 3) RG = 2;
+  ph.rg = RG;
+  ph.total = 0;
+  for (int mi = 0; mi < 2; ++mi) {
+    const bool on = mi < ph.nm;
+    const int K = on ? ph.m[mi].K : 32, nsal = on ? ph.m[mi].n_sal : 0;
+    const int rounds = (K / 32 + nsal / 32 + 31) / 32;
+    ph.rr[mi] = stk_rr(rounds);
+    ph.nrg[mi] = (rounds + ph.rr[mi] - 1) / ph.rr[mi];
+    ph.ntl[mi] = on ? (nrows + ph.tr - 1) / ph.tr : 0;
+    ph.ipt[mi] = (ph.tr / RG) * ph.nrg[mi];
+    const int nl = nrows - (ph.ntl[mi] - 1) * ph.tr;
+    ph.tot[mi] = on ? (ph.ntl[mi] - 1) * ph.ipt[mi] + ((nl + RG - 1) / RG) * ph.nrg[mi] : 0;
+    ph.total += ph.tot[mi];
+  }
 }
 
 template <int B>
@@ -490,6 +518,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
           ph.oslot[j] = j;
         }
       }
+      stk_plan_items(ph);
     }
     if (prep) stk_prep_sync();
     else stk_consumer_sync();
@@ -700,44 +729,25 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     // that takes an item of a tile whose slot still holds an earlier tile
     // waits for the slot's tag (stk_wait_tile).
     {
-      // four-row items where the tile's rows allow it and every matrix of the
-      // phase takes three-round items (three item shapes in all)
-      int RG = ph.tr % 4 == 0 ? 4 : 2;
-      for (int mi = 0; mi < ph.nm; ++mi)
-        if (stk_rr((ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32) != 3) RG = 2;
-      int nsal_[2], rk_[2], K_[2], nrg_[2], rr_[2], ntl_[2], ipt_[2], tot_[2];
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        const bool on = mi < ph.nm;
-        nsal_[mi] = on ? ph.m[mi].n_sal : 0;
-        rk_[mi] = on ? ph.m[mi].r : 0;
-        K_[mi] = on ? ph.m[mi].K : 32;
-        const int rounds = (K_[mi] / 32 + nsal_[mi] / 32 + 31) / 32;
-        rr_[mi] = stk_rr(rounds);
-        nrg_[mi] = (rounds + rr_[mi] - 1) / rr_[mi];
-        ntl_[mi] = on ? (nrows + ph.tr - 1) / ph.tr : 0;
-        ipt_[mi] = (ph.tr / RG) * nrg_[mi];
-        const int nl = nrows - (ntl_[mi] - 1) * ph.tr;
-        tot_[mi] = on ? (ntl_[mi] - 1) * ipt_[mi] + ((nl + RG - 1) / RG) * nrg_[mi] : 0;
-      }
-      const int total = tot_[0] + tot_[1];
+      const int RG = ph.rg, total = ph.total;
+      const int tot0 = ph.tot[0], ntl0 = ph.ntl[0];
       for (;;) {
         int gx = 0;
         if (lane == 0) gx = atomicAdd(s_grab, 1);
         gx = __shfl_sync(0xffffffffu, gx, 0);
         if (gx >= total) break;
-        const int mi = gx < tot_[0] ? 0 : 1;
-        const int g = gx - (mi ? tot_[0] : 0);
-        const int ipt = mi ? ipt_[1] : ipt_[0];
+        const int mi = gx < tot0 ? 0 : 1;
+        const int g = gx - (mi ? tot0 : 0);
+        const int ipt = ph.ipt[mi];
         const int tile = g / ipt, it = g - tile * ipt;
-        const uint32_t tseq = seq + (uint32_t)((mi ? ntl_[0] : 0) + tile);
+        const uint32_t tseq = seq + (uint32_t)((mi ? ntl0 : 0) + tile);
         const int s = (int)(tseq % (uint32_t)NS);
         const bool got = __all_sync(
             0xffffffffu, stk_wait_tile(&full[s], (tseq / (uint32_t)NS) & 1u, s_tag + s, (int)tseq, abort));
         const int i0 = ph.a + tile * ph.tr;
         const int nr = min(ph.tr, ph.b - i0);
-        const int nsal = mi ? nsal_[1] : nsal_[0], Km = mi ? K_[1] : K_[0];
-        const int nrg = mi ? nrg_[1] : nrg_[0], rr = mi ? rr_[1] : rr_[0];
+        const int nsal = ph.m[mi].n_sal, Km = ph.m[mi].K;
+        const int nrg = ph.nrg[mi], rr = ph.rr[mi];
         const int kq = Km / 2, ks = Km / 32;
         const uint8_t *q4s = ring + (size_t)s * p.slot_bytes;
         const uint8_t *s4s = q4s + nr * kq, *q8s = s4s + nr * ks;
@@ -749,7 +759,7 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         ta.xsu = xsu; ta.xsc = xsc; ta.xssm = xss + mi * (p.max_nsal / 32);
         ta.tvm = tv + mi * kStkMaxRank; ta.red = red;
         ta.kq = kq; ta.ks = ks; ta.nsal = nsal; ta.nu4 = Km / 32; ta.nu8 = nsal / 32;
-        ta.rk = mi ? rk_[1] : rk_[0];
+        ta.rk = ph.m[mi].r;
         ta.nr = nr; ta.nrg = nrg; ta.ra = i0 - ph.a; ta.mi = mi;
         ta.rows_max = rows_max; ta.rounds_max = rounds_max;
         if (got) {
@@ -769,15 +779,14 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
           }
         }
       }
-      seq += (uint32_t)(ntl_[0] + ntl_[1]);
+      seq += (uint32_t)(ph.ntl[0] + ph.ntl[1]);
     }
     stk_consumer_sync();
     // row results (round groups in order) back into red[mi][row][0]; a
     // matrix whose items span all rounds of a row has nothing to add
     bool more = false;
     for (int mi = 0; mi < ph.nm; ++mi) {
-      const int rounds = (ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32;
-      const int nrg = (rounds + stk_rr(rounds) - 1) / stk_rr(rounds);
+      const int nrg = ph.nrg[mi];
       if (nrg == 1) continue;
       more = true;
       for (int i = ctid; i < nrows; i += kStkConsThreads) {
