@@ -327,11 +327,14 @@ __host__ __device__ __forceinline__ int stk_rr(int rounds) {
 }
 
 // The item plan of a phase, computed once by the thread that writes its
-// descriptor.  RG = 4 rows per item where the tile's rows allow it and every
-// matrix of the phase takes three-round items (three item shapes in all).
+// descriptor.  RG = 5 (or 4) rows per item where the tile's rows allow it
+// and every matrix of the phase takes three-round items, else 2 (four item
+// shapes in all).  Five-row items cut a gate+up phase of the Spark shapes
+// (70 rows of each matrix per CTA) into 28 items, two even waves over the
+// 15 consumer warps, where four-row items made 36 (a third wave for 6).
 __device__ __forceinline__ void stk_plan_items(StkPhase &ph) {
   const int nrows = ph.b - ph.a;
-  int RG = ph.tr % 4 == 0 ? 4 : 2;
+  int RG = ph.tr % 5 == 0 ? 5 : ph.tr % 4 == 0 ? 4 : 2;
   for (int mi = 0; mi < ph.nm; ++mi)
     if (stk_rr((ph.m[mi].K / 32 + ph.m[mi].n_sal / 32 + 31) / 32) != 3) RG = 2;
   ph.rg = RG;
@@ -722,8 +725,8 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
 
     // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
     // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
-    // RR rounds of one tile (RG = 4 for three-round items when the tile's rows
-    // allow it, else 2).  The consumer warps take items from a shared
+    // RR rounds of one tile (RG = 5 or 4 for three-round items when the
+    // tile's rows allow it, else 2: stk_plan_items).  The consumer warps take items from a shared
     // counter in (matrix, tile, item) order, which is the ring's order; the
     // warp that completes a tile's last item frees its ring slot.  A warp
     // that takes an item of a tile whose slot still holds an earlier tile
@@ -763,7 +766,9 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
         ta.nr = nr; ta.nrg = nrg; ta.ra = i0 - ph.a; ta.mi = mi;
         ta.rows_max = rows_max; ta.rounds_max = rounds_max;
         if (got) {
-          if (RG == 4) {
+          if (RG == 5) {
+            stk_item<5, 3>(ta, it, lane);
+          } else if (RG == 4) {
             stk_item<4, 3>(ta, it, lane);
           } else {
             if (rr == 3) stk_item<2, 3>(ta, it, lane);
@@ -922,6 +927,9 @@ bool stk_plan(const std::vector<StackLayerDesc> &Ls, int G, StackParams &p) {
       rounds_max = std::max(rounds_max, (m.K / 32 + m.n_sal / 32 + 31) / 32);
     }
   p.tr_gu = std::max(2, (kStkSlotTarget / rb_gu) & ~1);
+  // gate/up tiles of six rows or more grow to a multiple of ten: two
+  // five-row items per tile (the Spark shapes: 8 -> 10 rows, 17.3 KB)
+  if (p.tr_gu >= 6) p.tr_gu = (p.tr_gu + 9) / 10 * 10;
   p.tr_d = std::max(2, (kStkSlotTarget / rb_d) & ~1);
   p.slot_bytes = (std::max(p.tr_gu * rb_gu, p.tr_d * rb_d) + 127) & ~127;
   p.max_rank = max_rank;
