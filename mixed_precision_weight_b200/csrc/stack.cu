@@ -726,11 +726,11 @@ __global__ void __launch_bounds__(kStkThreads, 1) mlp_stack_kernel(const StackPa
     // The rows.  A lane task is 32 columns of q4 (or 32 salient entries of
     // q8) of one row; a round is 32 consecutive tasks.  An item is RG rows x
     // RR rounds of one tile (RG = 5 or 4 for three-round items when the
-    // tile's rows allow it, else 2: stk_plan_items).  The consumer warps take items from a shared
-    // counter in (matrix, tile, item) order, which is the ring's order; the
-    // warp that completes a tile's last item frees its ring slot.  A warp
-    // that takes an item of a tile whose slot still holds an earlier tile
-    // waits for the slot's tag (stk_wait_tile).
+    // tile's rows allow it, else 2: stk_plan_items).  The consumer warps take
+    // items from a shared counter in (matrix, tile, item) order, which is the
+    // ring's order; the warp that completes a tile's last item frees its ring
+    // slot.  A warp that takes an item of a tile whose slot still holds an
+    // earlier tile waits for the slot's tag (stk_wait_tile).
     {
       const int RG = ph.rg, total = ph.total;
       const int tot0 = ph.tot[0], ntl0 = ph.ntl[0];
