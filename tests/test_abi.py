@@ -113,6 +113,78 @@ def test_fwht_argument_checks(dv):
     assert dv.lib.dvssq_fwht(P(264), P(256), 4, 512, 256, None) == 3
 
 
+def test_gelu_mul_argument_checks(dv):
+    P = ctypes.c_void_p
+    assert dv.lib.dvssq_gelu_mul(P(256), P(256), P(256), -1, None) == 1
+    assert dv.lib.dvssq_gelu_mul(P(256), P(256), P(256), 0, None) == 0   # no-op, no device
+    assert dv.lib.dvssq_gelu_mul(None, P(256), P(256), 8, None) == 1
+    assert dv.lib.dvssq_gelu_mul(P(256), P(264), P(256), 8, None) == 3
+
+
+def test_materialize_argument_checks(dv):
+    P = ctypes.c_void_p
+    s = _shape(dv)
+    w = dv._Weights(256, 256, 256, 256, 256, 256, 256)
+    assert dv.lib.dvssq_materialize(ctypes.byref(_shape(dv, block=64)), ctypes.byref(w), P(256), None) == 2
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), None, P(256), None) == 1
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), ctypes.byref(w), None, None) == 1
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), ctypes.byref(w), P(264), None) == 3
+    no_uv = dv._Weights(256, 256, 256, 256, 256, None, None)          # rank 8 needs U and V
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), ctypes.byref(no_uv), P(256), None) == 1
+    no_sal = dv._Weights(256, 256, None, None, 256, 256, 256)         # n_sal 64 needs sal_idx, q8
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), ctypes.byref(no_sal), P(256), None) == 1
+    bad_q4 = dv._Weights(264, 256, 256, 256, 256, 256, 256)
+    assert dv.lib.dvssq_materialize(ctypes.byref(s), ctypes.byref(bad_q4), P(256), None) == 3
+
+
+def test_lowrank_argument_checks(dv):
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    assert dv.lib.dvssq_lowrank_workspace_size(2560, 10240, 16, ctypes.byref(n)) == 0
+    small = n.value
+    assert small > 0
+    assert dv.lib.dvssq_lowrank_workspace_size(2560, 10240, 32, ctypes.byref(n)) == 0
+    assert n.value > small                                            # p = r + 16 columns
+    for M, K, r in ((2560, 10240, 4), (2560, 10240, 72), (2560, 10240, 12), (24, 10240, 16),
+                    (0, 10240, 16)):
+        assert dv.lib.dvssq_lowrank_workspace_size(M, K, r, ctypes.byref(n)) == 2, (M, K, r)
+    assert dv.lib.dvssq_lowrank_workspace_size(2560, 10240, 16, None) == 1
+    call = lambda R, it, ws, wsb: dv.lib.dvssq_lowrank(P(R), 2560, 10240, 16, it, 1, P(256), P(256),
+                                                       None, P(ws), wsb, None)
+    assert call(256, 65, 256, small) == 1                             # iterations 0..64
+    assert call(0, 4, 256, small) == 1                                # no residual
+    assert call(264, 4, 256, small) == 3                              # misaligned residual
+    assert call(256, 4, 272, small) == 3                              # workspace not 256-aligned
+    assert call(256, 4, 256, small - 16) == 4                         # workspace too small
+
+
+def test_bss_attention_argument_checks(dv):
+    P = ctypes.c_void_p
+    n = ctypes.c_size_t(0)
+    spark = dv.AttnShape(1, 16, 4, 256, 32768, 1.10, 12.0)
+    minicpm = dv.AttnShape(2, 16, 2, 128, 1000, 1.10, 12.0)
+    for sh in (spark, minicpm):
+        assert dv.lib.dvssq_bss_attention_workspace_size(ctypes.byref(sh), ctypes.byref(n)) == 0
+        assert n.value > 0
+    assert dv.lib.dvssq_bss_attention_workspace_size(ctypes.byref(spark), ctypes.byref(n)) == 0
+    need = n.value
+    bad = [dv.AttnShape(1, 12, 4, 256, 100, 1.1, 12.0),               # 3 query heads per KV head
+           dv.AttnShape(1, 16, 4, 64, 100, 1.1, 12.0),                # head_dim 64
+           dv.AttnShape(1, 16, 5, 128, 100, 1.1, 12.0),               # q_heads % kv_heads
+           dv.AttnShape(1, 16, 4, 256, 0, 1.1, 12.0)]                 # empty context
+    for sh in bad:
+        assert dv.lib.dvssq_bss_attention_workspace_size(ctypes.byref(sh), ctypes.byref(n)) == 2
+    for tau, haze in ((0.0, 12.0), (-1.0, 12.0), (1.1, float("nan"))):
+        sh = dv.AttnShape(1, 16, 4, 256, 100, tau, haze)
+        assert dv.lib.dvssq_bss_attention_workspace_size(ctypes.byref(sh), ctypes.byref(n)) == 1
+    call = lambda q, ws, wsb: dv.lib.dvssq_bss_attention(ctypes.byref(spark), P(q), P(256), P(256),
+                                                         P(256), P(ws), wsb, None)
+    assert call(0, 256, need) == 1
+    assert call(264, 256, need) == 3
+    assert call(256, 272, need) == 3
+    assert call(256, 256, need - 16) == 4
+
+
 def test_profile_api_without_launches(dv):
     dv.dvssq_profile_reset()
     dv.dvssq_profile_enable(True)
