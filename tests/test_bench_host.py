@@ -1,6 +1,7 @@
 """Host-side pieces of bench.py that need no GPU: the reference arm's refusal
-for workloads without a host step, and the source hash that keys the
-committed DRAM-traffic captures (comments and blank lines do not count)."""
+for workloads without a host step, the source hash that keys the committed
+DRAM-traffic captures (comments and blank lines do not count), the parsing
+of the clock samples, and the algorithmic bytes behind the roofline."""
 import contextlib
 import io
 import json
@@ -37,3 +38,39 @@ def test_every_traffic_record_names_a_kernel_with_sources():
         kernel = key.split("@")[0]
         assert kernel in bench.KERNEL_SOURCES, key
         assert ent["bytes_per_launch"] > 0 and len(ent["source_hash"]) == 16, key
+
+
+def test_clock_summary_parses_samples_and_reasons():
+    cs = bench.ClockSampler(0)
+    cs.out = "\n".join([
+        "1965, 1965, 812.4, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1950, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1965, 1965, 1001.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",   # unreadable
+        "short line",
+    ])
+    s = cs.summary()
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 3, "reasons": ["sw_power_cap"]}
+    cs.out = "1400, 1965, 700, 0x8, Not Active, Active, Not Active, Not Active"
+    assert cs.summary()["reasons"] == ["hw_thermal_slowdown"]
+    cs.out = ""
+    assert cs.summary() is None
+
+
+def test_roofline_bytes_follow_the_oracle_footprint():
+    # the decode GEMV's algorithmic bytes are the packed layer (the oracle's
+    # footprint, pinned to the pages' scorecard) minus U, which the tail reads
+    sys.path.insert(0, ROOT)
+    from oracle import dvssq_oracle as O
+    for M, K, r in ((2560, 10240, 16), (10240, 2560, 24), (512, 2048, 32), (8192, 2048, 24)):
+        n_sal = K // 8
+        assert bench.packed_bytes(M, K, r, n_sal) == O.packed_bytes(M, K, r, n_sal)
+        assert (bench.kernel_bytes("dec_row", M, K, r, n_sal, 1)
+                + bench.kernel_bytes("dec_tail", M, K, r, n_sal, 1)) == O.packed_bytes(M, K, r, n_sal)
+        assert bench.kernel_bytes("dec_main", M, K, r, n_sal, 16) == bench.kernel_bytes(
+            "dec_row", M, K, r, n_sal, 1)
+    # encode: W read once in BF16, the codes written once
+    M, K = 2560, 10240
+    assert bench.kernel_bytes("enc_pass1", M, K, 0, K // 8, 0) == M * K * 2
+    assert bench.kernel_bytes("enc_pass2", M, K, 16, K // 8, 0) == (
+        M * K * 2 + O.packed_bytes(M, K, 0, K // 8))
