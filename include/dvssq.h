@@ -365,7 +365,8 @@ typedef struct {
  * n_sal a multiple of 32; rank a multiple of 8 and at most 32; and rows
  * small enough that the shared-memory weight ring holds at least two slots
  * (two rows of the down matrix per slot at least: the Spark shapes, hidden
- * 2560 / inter 10240, fit 10 slots of 17.3 KB).
+ * 2560 / inter 10240, fit 10 slots of 17.3 KB).  The forward runs one CTA
+ * per SM on devices of at most 160 SMs (a B200 has 148).
  * Others return UNSUPPORTED_SHAPE.                                         */
 DVSSQ_API dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers,
                                                       int32_t n_layers, size_t *bytes);
