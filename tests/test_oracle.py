@@ -687,3 +687,19 @@ def test_bss_single_dominant_binding_returns_its_value():
     v = rng.standard_normal((1, 1, L, d))
     out = O.bss_attention(q, k, v)
     assert np.array_equal(out[0, 0], v[0, 0, 17])
+
+
+def test_bss_defaults_are_the_pages_constants():
+    import inspect
+    g = _read_kv("kv_bss.txt")
+    sig = inspect.signature(O.bss_attention)
+    assert sig.parameters["tau"].default == float(g["tau_focus"])
+    assert sig.parameters["haze"].default == float(g["haze_nats"])
+    assert abs(math.exp(-float(g["haze_nats"])) - float(g["exp_minus_haze"])) < 0.01e-6
+    # tau = 1.00 (KV-BSS off) with the haze off is plain attention: the same
+    # output as tau = 1.10 applied to a query scaled by 1 / 1.10
+    rng = np.random.default_rng(12)
+    q, k, v = rng.standard_normal((1, 2, 8)), rng.standard_normal((1, 1, 30, 8)), \
+        rng.standard_normal((1, 1, 30, 8))
+    off = O.bss_attention(q, k, v, tau=float(g["tau_off"]), haze=0.0)
+    assert np.allclose(off, O.bss_attention(q / float(g["tau_focus"]), k, v, haze=0.0), atol=1e-14)
