@@ -74,3 +74,22 @@ def test_roofline_bytes_follow_the_oracle_footprint():
     assert bench.kernel_bytes("enc_pass1", M, K, 0, K // 8, 0) == M * K * 2
     assert bench.kernel_bytes("enc_pass2", M, K, 16, K // 8, 0) == (
         M * K * 2 + O.packed_bytes(M, K, 0, K // 8))
+
+
+def test_reference_arm_line_keeps_the_contract():
+    # the oracle arm on the decode workload runs on the host cores (about 10 s)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(types.SimpleNamespace(workload="decode", steps=1, warmup=0), 1, 0)
+    line = json.loads(out.getvalue().strip().splitlines()[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "GB/s" and line["n_gpus"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "GB/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"].startswith("spark_down")
