@@ -371,6 +371,26 @@ typedef struct {
 DVSSQ_API dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers,
                                                       int32_t n_layers, size_t *bytes);
 
+/* The launch plan dvssq_mlp_stack_forward uses for these layers on a device
+ * of `sm_count` SMs (host only; no device is needed).  The forward runs one
+ * CTA per SM; warp 0 of each streams the CTA's weight rows into a ring of
+ * shared-memory slots and the other warps compute.
+ *   ctas          = sm_count
+ *   threads       per CTA
+ *   ring_slots    weight-ring slots, each slot_bytes long
+ *   rows_per_tile_gate_up, rows_per_tile_down   weight rows per ring slot
+ *   smem_bytes    dynamic shared memory per CTA
+ * Errors: INVALID_ARG (plan NULL, sm_count < 1, layers as for the workspace
+ * query), UNSUPPORTED_SHAPE (the layers, or tiles that leave the ring fewer
+ * than two slots, or sm_count above 160), MISALIGNED.                      */
+typedef struct {
+  int32_t ctas, threads, ring_slots, slot_bytes;
+  int32_t rows_per_tile_gate_up, rows_per_tile_down, smem_bytes;
+} dvssq_mlp_stack_plan;
+DVSSQ_API dvssq_status dvssq_mlp_stack_plan_query(const dvssq_mlp_layer *layers,
+                                                  int32_t n_layers, int32_t sm_count,
+                                                  dvssq_mlp_stack_plan *plan);
+
 /* Prepares `workspace` for dvssq_mlp_stack_forward on these layers: writes
  * the device table of the layers and, per matrix, (V H_K) in FP32 (the
  * blockwise FWHT of each row of V; H is symmetric).  Synchronises `stream`.

@@ -28,8 +28,8 @@ __all__ = [
     "dvssq_forward_workspace_size", "dvssq_linear_forward", "dvssq_linear_forward_static",
     "dvssq_materialize", "dvssq_lowrank_workspace_size", "dvssq_lowrank", "AttnShape",
     "dvssq_bss_attention_workspace_size", "dvssq_bss_attention", "dvssq_device_error", "STATIC_SCRATCH_BYTES", "MlpStack",
-    "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
-    "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
+    "dvssq_mlp_stack_workspace_size", "dvssq_mlp_stack_plan_query", "dvssq_mlp_stack_prepare",
+    "dvssq_mlp_stack_forward", "dvssq_profile_enable", "dvssq_profile_collect", "dvssq_profile_read",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
     "Y_F32", "Y_BF16", "PATH_AUTO", "PATH_DECODE", "PATH_PREFILL",
     "EXPORTED_SYMBOLS",
@@ -55,7 +55,7 @@ EXPORTED_SYMBOLS = (
     "dvssq_linear_forward", "dvssq_linear_forward_static", "dvssq_materialize",
     "dvssq_lowrank_workspace_size", "dvssq_lowrank", "dvssq_bss_attention_workspace_size",
     "dvssq_bss_attention", "dvssq_device_error", "dvssq_mlp_stack_workspace_size",
-    "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
+    "dvssq_mlp_stack_plan_query", "dvssq_mlp_stack_prepare", "dvssq_mlp_stack_forward",
     "dvssq_profile_enable",
     "dvssq_profile_collect", "dvssq_profile_count", "dvssq_profile_get",
     "dvssq_profile_reset", "dvssq_set_wait_limit", "dvssq_selftest_wait",
@@ -83,6 +83,13 @@ class _Weights(ctypes.Structure):
 
 class _MlpLayer(ctypes.Structure):
     _fields_ = [("shape", Shape * 3), ("w", _Weights * 3)]
+
+
+class _StackPlan(ctypes.Structure):
+    _fields_ = [("ctas", ctypes.c_int32), ("threads", ctypes.c_int32),
+                ("ring_slots", ctypes.c_int32), ("slot_bytes", ctypes.c_int32),
+                ("rows_per_tile_gate_up", ctypes.c_int32), ("rows_per_tile_down", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32)]
 
 
 class AttnShape(ctypes.Structure):
@@ -127,6 +134,8 @@ _sig = {
     "dvssq_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]),
     "dvssq_mlp_stack_workspace_size": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32,
                                                       ctypes.POINTER(ctypes.c_size_t)]),
+    "dvssq_mlp_stack_plan_query": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32,
+                                                  ctypes.c_int32, ctypes.POINTER(_StackPlan)]),
     "dvssq_mlp_stack_prepare": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32, _P,
                                                ctypes.c_size_t, _P]),
     "dvssq_mlp_stack_forward": (ctypes.c_int, [ctypes.POINTER(_MlpLayer), ctypes.c_int32, _P, _P,
@@ -391,6 +400,17 @@ def dvssq_mlp_stack_workspace_size(layers) -> int:
     _check(lib.dvssq_mlp_stack_workspace_size(arr, len(layers), ctypes.byref(n)),
            "dvssq_mlp_stack_workspace_size")
     return n.value
+
+
+def dvssq_mlp_stack_plan_query(layers, sm_count: int) -> dict:
+    """The forward's launch plan for these layers on a device of sm_count SMs
+    (host only): CTAs, threads per CTA, weight-ring slots and their bytes, weight
+    rows per slot for gate/up and for down, dynamic shared memory per CTA."""
+    arr = _mlp_layers(layers)
+    plan = _StackPlan()
+    _check(lib.dvssq_mlp_stack_plan_query(arr, len(layers), int(sm_count), ctypes.byref(plan)),
+           "dvssq_mlp_stack_plan_query")
+    return {name: getattr(plan, name) for name, _ in _StackPlan._fields_}
 
 
 def dvssq_mlp_stack_prepare(layers, workspace: torch.Tensor, stream=None):

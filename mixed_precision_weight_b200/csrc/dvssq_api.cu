@@ -440,6 +440,25 @@ dvssq_status dvssq_mlp_stack_workspace_size(const dvssq_mlp_layer *layers, int32
   return DVSSQ_OK;
 }
 
+dvssq_status dvssq_mlp_stack_plan_query(const dvssq_mlp_layer *layers, int32_t n_layers,
+                                        int32_t sm_count, dvssq_mlp_stack_plan *plan) {
+  if (plan == nullptr || sm_count < 1) return DVSSQ_ERR_INVALID_ARG;
+  std::vector<StackMatDesc> mats;
+  StackShapeInfo si{};
+  dvssq_status s = stack_descs(layers, n_layers, mats, si);
+  if (s != DVSSQ_OK) return s;
+  StackPlanInfo pi{};
+  if (!stack_plan_info(mats.data(), n_layers, sm_count, pi)) return DVSSQ_ERR_UNSUPPORTED_SHAPE;
+  plan->ctas = pi.ctas;
+  plan->threads = pi.threads;
+  plan->ring_slots = pi.slots;
+  plan->slot_bytes = pi.slot_bytes;
+  plan->rows_per_tile_gate_up = pi.tr_gu;
+  plan->rows_per_tile_down = pi.tr_d;
+  plan->smem_bytes = pi.smem;
+  return DVSSQ_OK;
+}
+
 dvssq_status dvssq_mlp_stack_prepare(const dvssq_mlp_layer *layers, int32_t n_layers,
                                      void *workspace, size_t workspace_bytes, void *stream) {
   std::vector<StackMatDesc> mats;

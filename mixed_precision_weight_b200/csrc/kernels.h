@@ -145,6 +145,12 @@ struct StackShapeInfo {
 };
 bool stack_shape_info(const StackMatDesc *mats, int L, StackShapeInfo &si);
 size_t stack_workspace_bytes(const StackShapeInfo &si, int L);
+// The forward's launch plan for G SMs (host only): false when the stack's
+// tiles do not fit the shared-memory ring or G is out of range.
+struct StackPlanInfo {
+  int ctas, threads, slots, slot_bytes, tr_gu, tr_d, smem;
+};
+bool stack_plan_info(const StackMatDesc *mats, int L, int G, StackPlanInfo &out);
 cudaError_t stack_prepare(StackMatDesc *mats, int L, const StackShapeInfo &si, void *ws,
                           cudaStream_t st, Launcher &Lc);
 cudaError_t launch_mlp_stack(const StackMatDesc *mats, int L, const StackShapeInfo &si,

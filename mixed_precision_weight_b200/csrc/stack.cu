@@ -1000,6 +1000,22 @@ size_t stack_workspace_bytes(const StackShapeInfo &si, int L) {
   return stk_ws_layout(si, L, std::max(1, stk_sm_count())).total;
 }
 
+bool stack_plan_info(const StackMatDesc *mats, int L, int G, StackPlanInfo &out) {
+  std::vector<StackLayerDesc> Ls((size_t)L);
+  for (int l = 0; l < L; ++l)
+    for (int mi = 0; mi < 3; ++mi) Ls[(size_t)l].m[mi] = mats[3 * l + mi];
+  StackParams p{};
+  if (!stk_plan(Ls, G, p)) return false;
+  out.ctas = G;
+  out.threads = kStkThreads;
+  out.slots = p.nslots;
+  out.slot_bytes = p.slot_bytes;
+  out.tr_gu = p.tr_gu;
+  out.tr_d = p.tr_d;
+  out.smem = p.smem_total;
+  return true;
+}
+
 cudaError_t stack_prepare(StackMatDesc *mats, int L, const StackShapeInfo &si, void *ws,
                           cudaStream_t st, Launcher &Lc) {
   const int G = stk_sm_count();

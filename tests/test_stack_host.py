@@ -91,3 +91,32 @@ def test_rejects_bad_layer_tables(dv, case, expected):
         packed.q4 = base[off:off + packed.q4.numel()].view(packed.q4.shape)
         layers = [((shape, packed), u, d)]
     assert _status(dv, layers) == expected
+
+
+def test_plan_query_for_the_spark_stack(dv):
+    # 36 Spark blocks (hidden 2560, intermediate 10240, n_sal = K / 8; ranks
+    # 16 and 24 as in the bench's stack) on a B200's 148 SMs
+    layers = [_layer(dv, 2560, 10240, ranks=(r, r, r)) for r in [16] * 14 + [24] * 15 + [16] * 7]
+    p = dv.dvssq_mlp_stack_plan_query(layers, 148)
+    assert p["ctas"] == 148 and p["threads"] == 512
+    # gate/up rows are 1280 + 80 + 320 + 2 r bytes: ten of them per slot; down
+    # rows 6768 bytes at r = 24: two per slot, inside the same slot size
+    assert p["rows_per_tile_gate_up"] == 10 and p["rows_per_tile_down"] == 2
+    assert p["slot_bytes"] >= 10 * (1280 + 80 + 320 + 2 * 24)
+    assert p["slot_bytes"] >= 2 * (5120 + 320 + 1280 + 2 * 24)
+    assert p["ring_slots"] >= 2
+    assert p["ring_slots"] * p["slot_bytes"] < p["smem_bytes"] <= 232448   # 227 KB opt-in
+    # the plan does not depend on the SM count up to the limit, and stops there
+    assert dv.dvssq_mlp_stack_plan_query(layers, 160)["ring_slots"] == p["ring_slots"]
+    for sm, status in ((161, UNSUPPORTED_SHAPE), (0, INVALID_ARG)):
+        with pytest.raises(dv.DvssqError) as e:
+            dv.dvssq_mlp_stack_plan_query(layers, sm)
+        assert e.value.status == status
+
+
+def test_plan_query_rejects_what_the_workspace_query_rejects(dv):
+    g, u, d = _layer(dv, 512, 1024)
+    assert dv.dvssq_mlp_stack_plan_query([(g, u, d)], 148)["ring_slots"] >= 2
+    with pytest.raises(dv.DvssqError) as e:
+        dv.dvssq_mlp_stack_plan_query([(d, u, g)], 148)
+    assert e.value.status == UNSUPPORTED_SHAPE
